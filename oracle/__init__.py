@@ -1,0 +1,8 @@
+"""CPU oracle (test infrastructure only; never imported by the product path)."""
+
+from .paged_attention import (ORACLE, PagedAttentionOracle, attend, copy_blocks,
+                              decode, decode_one, gather, merge, partial,
+                              write_kv)
+
+__all__ = ["ORACLE", "PagedAttentionOracle", "attend", "copy_blocks", "decode",
+           "decode_one", "gather", "merge", "partial", "write_kv"]
