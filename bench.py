@@ -1,0 +1,488 @@
+"""Benchmark of the paged-KV decode step on B200.
+
+One step = the whole hot path over one batch: copy-on-write block copies (when
+the workload has them), the new-token KV write, and paged decode attention for
+every sequence and query head. Inputs are resident in HBM before timing
+starts; every workload's KV bytes exceed the 126 MB L2, so no flush is needed
+between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mha|gqa|prefix_cow|long|tiny]
+                    [--impl ours|reference] [--block-size BS] [--path auto|simt|tc]
+
+Under torchrun (N > 1) every rank runs its own independent batch (different
+seed) on its own GPU: decode of different sequences needs no exchange, so the
+scaling is weak and no collective touches the data path; the step time is the
+max over ranks. Rank 0 prints one JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+from pathlib import Path
+
+import numpy as np
+import torch
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+METRIC = "paged decode: effective KV-read HBM GB/s (% of B200 peak), seq-steps/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="mha")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--block-size", type=int, default=0)
+    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
+    ap.add_argument("--split", type=int, default=0)
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (control path only)
+# ---------------------------------------------------------------------------
+
+def dist_setup(n):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# workload
+# ---------------------------------------------------------------------------
+
+def make_batch(name, device, rank, block_size):
+    from paged_kv_cache_339_b200 import workloads as W
+    fn = W.FULL[name]
+    seed = {"tiny": 1001, "mha": 1002, "gqa": 1003, "prefix_cow": 1004, "long": 1005}[name]
+    kw = {"seed": seed + 100 * rank}
+    if block_size and name in ("mha", "gqa", "long"):
+        kw["block_size"] = block_size
+    return fn(device, **kw)
+
+
+def config_of(b, name, l2_note):
+    G = b.num_q_heads // b.num_kv_heads
+    lens = b.context_lens.cpu()
+    return {
+        "workload": b.name, "num_seqs": b.num_seqs, "num_q_heads": b.num_q_heads,
+        "num_kv_heads": b.num_kv_heads, "group": G, "head_dim": b.head_dim,
+        "block_size": b.block_size, "num_blocks": b.num_blocks,
+        "context_len_mean": round(float(lens.float().mean()), 1),
+        "context_len_max": int(lens.max()), "cow_pairs": int(b.cow_pairs.shape[0]),
+        "kv_bytes_per_step": b.kv_bytes_logical(), "l2": l2_note,
+    }
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.out = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.15)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out = ""
+
+    def summary(self):
+        if not self.out:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# our implementation
+# ---------------------------------------------------------------------------
+
+def step_fn(b, ops, out, ws, split, path, stream):
+    max_ctx = b.max_context_len
+
+    def step():
+        n = 0
+        if b.cow_pairs.numel():
+            ops.pa_copy_blocks(b.k_cache, b.v_cache, b.cow_pairs, stream=stream)
+            n += 1
+        ops.pa_write_kv(b.k_cache, b.v_cache, b.key, b.value, b.slot_mapping, stream=stream)
+        ops.pa_decode(out, b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, max_ctx,
+                      b.scale, ws, split_tokens=split, path=path, stream=stream)
+        return n + 1 + 3   # write, plan, decode, merge
+    return step
+
+
+def time_device(step, K, W, stream, use_graph, world):
+    """Device time of K steps (CUDA events on the launching stream)."""
+    launches = 0
+    with torch.cuda.stream(stream):
+        for _ in range(W):
+            launches = step()
+        torch.cuda.synchronize()
+        graph = None
+        if use_graph:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=stream):
+                step()
+            for _ in range(2):
+                graph.replay()
+            torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            if graph is not None:
+                graph.replay()
+            else:
+                step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    ms = e0.elapsed_time(e1)
+    del graph
+    return ms / K, launches
+
+
+def time_decode_only(b, ops, out, ws, split, path, stream, K):
+    """Average duration of the decode call alone (plan + main + merge kernels)
+    and of the main kernel share, with events around each call."""
+    max_ctx = b.max_context_len
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            ops.pa_decode(out, b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens,
+                          max_ctx, b.scale, ws, split_tokens=split, path=path, stream=stream)
+        torch.cuda.synchronize()
+        for a, z in ev:
+            a.record(stream)
+            ops.pa_decode(out, b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens,
+                          max_ctx, b.scale, ws, split_tokens=split, path=path, stream=stream)
+            z.record(stream)
+        torch.cuda.synchronize()
+    ts = [a.elapsed_time(z) for a, z in ev]
+    return statistics.median(ts), ts
+
+
+def time_e2e(b, ops, ws, split, path, stream, K, W):
+    """Same metric through the public API from pinned host buffers: every step
+    copies its inputs host->device and reads the result back."""
+    host = {k: getattr(b, k).cpu().pin_memory() for k in
+            ("q", "key", "value", "slot_mapping", "block_tables", "context_lens", "cow_pairs")}
+    dev = {k: torch.empty_like(v, device="cuda") for k, v in host.items()}
+    out = torch.empty(b.q.shape, dtype=torch.float32, device="cuda")
+    out_h = torch.empty(b.q.shape, dtype=torch.float32).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_h.numel() * 4
+    max_ctx = b.max_context_len
+
+    def step():
+        for k in host:
+            dev[k].copy_(host[k], non_blocking=True)
+        if dev["cow_pairs"].numel():
+            ops.pa_copy_blocks(b.k_cache, b.v_cache, dev["cow_pairs"], stream=stream)
+        ops.pa_write_kv(b.k_cache, b.v_cache, dev["key"], dev["value"], dev["slot_mapping"],
+                        stream=stream)
+        ops.pa_decode(out, dev["q"], b.k_cache, b.v_cache, dev["block_tables"],
+                      dev["context_lens"], max_ctx, b.scale, ws, split_tokens=split, path=path,
+                      stream=stream)
+        out_h.copy_(out, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(W):
+            step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / K, h2d, d2h
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in sorted((ROOT / "paged_kv_cache_339_b200" / "csrc").glob("*")):
+        if f.suffix in (".cu", ".cuh", ".h"):
+            h.update(f.read_bytes())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profile(workload, kernel_hash):
+    """DRAM bytes per launch of the decode kernel from the committed ncu
+    summary, if it was taken on the current kernel sources."""
+    f = ROOT / "profiles" / "decode_traffic.json"
+    if not f.exists():
+        return None
+    try:
+        d = json.loads(f.read_text())
+        e = d.get(workload)
+        if e and e.get("kernel_source_hash") == kernel_hash:
+            return e.get("dram_bytes_per_launch")
+    except (ValueError, OSError):
+        pass
+    return None
+
+
+def measured_peak():
+    f = ROOT / "MEASURED_PEAKS.json"
+    try:
+        d = json.loads(f.read_text())
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, ValueError, KeyError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(b, seconds):
+    """Run the fp64 oracle on the first sequences of the batch (all heads) until
+    about `seconds` of CPU work; returns (KV bytes covered, seconds, seqs)."""
+    from oracle import ORACLE
+    from threadpoolctl import threadpool_info
+    BS = b.block_size
+    G = b.num_q_heads // b.num_kv_heads
+    done_bytes, spent, nseq = 0, 0.0, 0
+    e = b.elem_bytes
+    for i in range(b.num_seqs):
+        L = int(b.context_lens[i])
+        nb = (L + BS - 1) // BS
+        rows = b.block_tables[i, :nb].long()
+        kc = b.k_cache[rows].to(torch.float32).cpu().numpy().astype(np.float64)
+        vc = b.v_cache[rows].to(torch.float32).cpu().numpy().astype(np.float64)
+        q = b.q[i].to(torch.float32).cpu().numpy().astype(np.float64)
+        t0 = time.perf_counter()
+        tab = np.arange(nb)
+        for h in range(b.num_q_heads):
+            ORACLE.decode_one(q[h], kc, vc, tab, L, h, b.num_q_heads, b.scale)
+        spent += time.perf_counter() - t0
+        done_bytes += 2 * L * b.num_kv_heads * b.head_dim * e
+        nseq += 1
+        if spent >= seconds:
+            break
+    threads = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    return done_bytes, spent, nseq, threads
+
+
+# ---------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local):
+    from paged_kv_cache_339_b200 import build as pa_build
+    pa_build.build()
+    from paged_kv_cache_339_b200 import ops
+    path = {"auto": ops.PA_PATH_AUTO, "simt": ops.PA_PATH_SIMT, "tc": ops.PA_PATH_TCGEN05}[args.path]
+    b = make_batch(args.workload, "cuda", rank, args.block_size)
+    kv_bytes = b.kv_bytes_logical()
+    B, Hq, D = b.q.shape
+    ws = ops.decode_workspace(B, Hq, D, b.max_context_len, b.block_size, args.split)
+    out = torch.empty((B, Hq, D), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.Stream()
+    step = step_fn(b, ops, out, ws, args.split, path, stream)
+    W = max(args.warmup, 3)
+
+    with ClockSampler(local) as clk:
+        ms, per_step = time_device(step, args.steps, W, stream, not args.no_graph, world)
+    ms = max_over_ranks(ms, world)
+    torch.cuda.synchronize()
+    status = ops.pa_decode_status(ws, stream)
+    dec_ms, _ = time_decode_only(b, ops, out, ws, args.split, path, stream, max(10, args.steps))
+    e2e_ms, h2d, d2h = time_e2e(b, ops, ws, args.split, path, stream, max(5, args.steps // 2), 3)
+    e2e_ms = max_over_ranks(e2e_ms, world)
+
+    peak, peak_kind = measured_peak()
+    gbps = kv_bytes * world / (ms * 1e-3) / 1e9
+    dec_gbps = kv_bytes / (dec_ms * 1e-3) / 1e9
+    khash = kernel_source_hash()
+    res = {
+        "metric": METRIC, "value": round(gbps, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": W, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": {torch.bfloat16: "bf16", torch.float16: "f16", torch.float32: "f32"}[b.dtype],
+        "data": "synthetic (seeded N(0,1) K/V/Q, shuffled block placement)",
+        "config": config_of(b, args.workload,
+                            f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of KV read per step"),
+        "seq_steps_per_s": round(B * world / (ms * 1e-3), 1),
+        "pct_of_peak": round(100.0 * gbps / world / peak, 2),
+        "pct_of_nominal_8tbs": round(100.0 * gbps / world / 8000.0, 2),
+        "decode_status": int(status),
+        "gpu_launches": per_step * args.steps,
+        "roofline": {
+            "bound": "hbm", "kernel": "pa_decode (plan + decode main + merge)",
+            "achieved": round(dec_gbps, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(dec_gbps / peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
+            "algorithmic_bytes_per_launch": kv_bytes,
+            "launch_ms": round(dec_ms, 5),
+            "traffic": traffic_from_profile(b.name, khash),
+            "kernel_source_hash": khash,
+        },
+        "e2e": {"value": round(kv_bytes * world / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h)},
+        "clocks": clk.summary(),
+        "graph": not args.no_graph,
+    }
+    if not args.no_secondary and world == 1 and args.workload == "mha":
+        sec = {}
+        for name in ("gqa", "long"):
+            del b
+            torch.cuda.empty_cache()
+            b = make_batch(name, "cuda", rank, 0)
+            B2, Hq2, D2 = b.q.shape
+            ws2 = ops.decode_workspace(B2, Hq2, D2, b.max_context_len, b.block_size, 0)
+            out2 = torch.empty((B2, Hq2, D2), dtype=torch.float32, device="cuda")
+            st2 = step_fn(b, ops, out2, ws2, 0, ops.PA_PATH_AUTO, stream)
+            ms2, _ = time_device(st2, max(10, args.steps // 2), 3, stream, not args.no_graph, 1)
+            d2, _ = time_decode_only(b, ops, out2, ws2, 0, ops.PA_PATH_AUTO, stream, 10)
+            kb = b.kv_bytes_logical()
+            sec[b.name] = {"step_gbps": round(kb / (ms2 * 1e-3) / 1e9, 1),
+                           "decode_gbps": round(kb / (d2 * 1e-3) / 1e9, 1),
+                           "frac_of_measured_peak": round(kb / (d2 * 1e-3) / 1e9 / peak, 4),
+                           "ms_per_step": round(ms2, 5),
+                           "status": ops.pa_decode_status(ws2, stream)}
+            del ws2, out2
+        res["secondary"] = sec
+        del b
+        torch.cuda.empty_cache()
+        b = make_batch(args.workload, "cuda", rank, args.block_size)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        nbytes, secs, nseq, threads = oracle_sample(b, args.cpu_seconds)
+        res["cpu_baseline"] = {
+            "value": round(nbytes / secs / 1e9, 4), "unit": "GB/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"fp64 NumPy oracle, decode of the first {nseq} of {b.num_seqs} "
+                      f"sequences (all {b.num_q_heads} heads), {secs:.1f} s",
+        }
+    return res
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: same workload, bounded sample per step."""
+    if rank != 0:
+        return None
+    b = make_batch(args.workload, "cuda" if torch.cuda.is_available() else "cpu", 0,
+                   args.block_size)
+    per = max(args.cpu_seconds / max(args.steps, 1), 0.5)
+    for _ in range(min(args.warmup, 1)):
+        oracle_sample(b, 0.1)
+    tot_b, tot_s, seqs, threads = 0, 0.0, 0, 1
+    for _ in range(args.steps):
+        nb, s, n, threads = oracle_sample(b, per)
+        tot_b += nb
+        tot_s += s
+        seqs = n
+    v = tot_b / tot_s / 1e9
+    return {
+        "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * tot_s / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": config_of(b, args.workload, "host memory"),
+        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": threads,
+                         "kind": "oracle",
+                         "sample": f"each step: decode of the first {seqs} sequences, all heads"},
+        "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            res = run_reference(args, rank, world)
+        else:
+            res = run_ours(args, rank, world, local)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,202 @@
+/*
+ * pa.h - C ABI of the paged KV-cache decode library (libpagedattn.so).
+ *
+ * The KV cache is a pool of fixed-size physical blocks, each holding the keys
+ * and values of `block_size` tokens; every sequence keeps a block table that
+ * lists, in logical order, which physical blocks hold it, and the attention
+ * kernel follows that table instead of assuming the sequence is laid out end
+ * to end ("Paged Attention: Virtual Memory for the KV Cache", section "The fix
+ * borrowed from operating systems"; glossary "Paged attention", section "What
+ * is Paged Attention?").
+ *
+ * Three device operations:
+ *   pa_write_kv    - store each new token's K and V into its slot;
+ *   pa_copy_blocks - copy whole blocks: the copy-on-write step when a sequence
+ *                    diverges inside a shared block;
+ *   pa_decode      - single-query attention of every sequence over its paged
+ *                    context.
+ *
+ * Conventions for every call:
+ *   - All array pointers are caller-owned DEVICE memory (in practice PyTorch
+ *     tensors). The library never allocates, frees or synchronises device
+ *     memory; it only enqueues kernels on `stream` (0 = legacy default stream).
+ *   - Argument checks run on the host, synchronously, before anything is
+ *     enqueued; a rejected call has enqueued nothing. Errors that depend on
+ *     device data are the caller's contract, but never lead to an access
+ *     outside the caller's buffers: pa_write_kv / pa_copy_blocks skip slots and
+ *     blocks outside the pool; pa_decode reads block 0 in place of a table
+ *     entry outside the pool and writes zero rows for a sequence whose length
+ *     is negative or exceeds max_context_len or its table, and records
+ *     PA_ERR_INVALID_ARG in its status word (pa_decode_status).
+ *   - A launch failure is reported as PA_ERR_CUDA; pa_last_cuda_error() gives
+ *     the CUDA error string of the most recent such failure on this thread.
+ *   - Every array must be 16-byte aligned and densely packed in the layout
+ *     given (row-major, innermost index last).
+ */
+#ifndef PAGED_KV_CACHE_PA_H
+#define PAGED_KV_CACHE_PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Opaque CUDA stream handle (a cudaStream_t). */
+typedef void* pa_stream_t;
+
+typedef enum {
+  PA_F32 = 0,
+  PA_F16 = 1,
+  PA_BF16 = 2
+} pa_dtype;
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,          /* null pointer, negative size, bad shape */
+  PA_ERR_UNSUPPORTED = 2,          /* dtype / head_dim / block_size not built */
+  PA_ERR_MISALIGNED = 3,           /* a pointer is not 16-byte aligned */
+  PA_ERR_WORKSPACE_TOO_SMALL = 4,  /* see pa_decode_workspace_size */
+  PA_ERR_CUDA = 5,                 /* a CUDA call failed; see pa_last_cuda_error */
+  PA_ERR_DEVICE_TIMEOUT = 6        /* a kernel gave up waiting (see pa_decode_status) */
+} pa_status;
+
+/*
+ * The two pools of one layer's cache. Both have shape
+ *   [num_blocks, num_kv_heads, block_size, head_dim]
+ * and element type `dtype`: slot s (token) of the pool lives in block
+ * s / block_size at offset s % block_size; inside a block, each KV head's
+ * block_size x head_dim tile is contiguous.
+ * Supported: dtype F32/F16/BF16, head_dim 64/128, block_size 8/16/32
+ * (the block sizes the pages call typical: "Paged Attention as a Memory
+ * Manager", "Virtual Memory as the Blueprint").
+ */
+typedef struct {
+  void* k_cache;
+  void* v_cache;
+  int32_t num_blocks;
+  int32_t num_kv_heads;
+  int32_t block_size;
+  int32_t head_dim;
+  pa_dtype dtype;
+} pa_kv_cache;
+
+/*
+ * pa_write_kv - store new tokens' keys and values into their slots.
+ *
+ * A sequence fills its current block and takes a new one only when it needs
+ * one ("The fix borrowed from operating systems"); the host decides the slot,
+ * this call only stores. For token t (0 <= t < num_tokens) and KV head h:
+ *   k_cache[slot / BS][h][slot % BS][:] = key[t][h][:]   (same for V)
+ * with slot = slot_mapping[t]; a negative slot skips the token (padding).
+ *
+ *   key, value    device [num_tokens, num_kv_heads, head_dim], cache dtype
+ *   slot_mapping  device int64 [num_tokens]; slots must be distinct within a
+ *                 call and < num_blocks * block_size
+ * Bit-exact copy. num_tokens == 0 is a no-op returning PA_OK.
+ */
+pa_status pa_write_kv(const pa_kv_cache* cache, const void* key,
+                      const void* value, const int64_t* slot_mapping,
+                      int32_t num_tokens, pa_stream_t stream);
+
+/*
+ * pa_copy_blocks - copy-on-write block copies.
+ *
+ * When a sequence is about to write into a block it shares, it first gets its
+ * own copy of that block ("Paged Attention: Virtual Memory for the KV Cache",
+ * section "Sharing comes almost for free"). For each pair p:
+ *   k_cache[dst] = k_cache[src]; v_cache[dst] = v_cache[src]   (all heads)
+ * with (src, dst) = (block_pairs[2p], block_pairs[2p + 1]).
+ *
+ *   block_pairs  device int64 [num_pairs][2]; every dst distinct and never a
+ *                src in the same call (otherwise the result is order-dependent)
+ * Bit-exact copy. num_pairs == 0 is a no-op returning PA_OK.
+ */
+pa_status pa_copy_blocks(const pa_kv_cache* cache, const int64_t* block_pairs,
+                         int32_t num_pairs, pa_stream_t stream);
+
+/* Kernel choice for pa_decode (see pa_decode_options.path). */
+typedef enum {
+  PA_PATH_AUTO = 0,   /* tensor-core path when it applies, else CUDA cores */
+  PA_PATH_SIMT = 1,   /* CUDA-core kernel for every supported shape */
+  PA_PATH_TCGEN05 = 2 /* tensor-core kernel; PA_ERR_UNSUPPORTED if it cannot run */
+} pa_decode_path;
+
+typedef struct {
+  /* Tokens per work item (context split). 0 = chosen on the device from the
+     actual context lengths (a multiple of 128, at least 256, and at most 64
+     splits per sequence for max_context_len). Otherwise a positive multiple
+     of block_size with ceil(max_context_len / split_tokens) <= 256. */
+  int32_t split_tokens;
+  int32_t path;        /* a pa_decode_path */
+} pa_decode_options;
+
+/*
+ * pa_decode_workspace_size - bytes of device workspace pa_decode needs for the
+ * given shapes (work list, one partial result per (sequence, query head,
+ * split), status word). split_tokens as in pa_decode_options.
+ */
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
+                                int32_t head_dim, int32_t max_context_len,
+                                int32_t block_size, int32_t split_tokens);
+
+/*
+ * pa_decode - paged single-query decode attention.
+ *
+ * For sequence i, query head h (0 <= h < num_q_heads) and KV head
+ * kv = h / (num_q_heads / num_kv_heads) (consecutive query heads share a KV
+ * head: grouped-query attention, "Paged Attention: Virtual Memory for the KV
+ * Cache", "What it does not fix"):
+ *   K_j = k_cache[bt[i][j / BS]][kv][j % BS][:],  V_j likewise,  j < L_i
+ *   s_j = scale * <q[i][h], K_j>
+ *   out[i][h] = sum_j exp(s_j - max s) V_j / sum_j exp(s_j - max s)
+ * with bt = block_tables, L_i = context_lens[i]; L_i == 0 gives a zero row.
+ * The sequence is read through its table as if it were contiguous (glossary
+ * "Paged attention", "What is Paged Attention?"). The pages never write the
+ * formula; this is the plain scaled dot-product reading.
+ *
+ *   out           device fp32 [num_seqs, num_q_heads, head_dim]
+ *   q             device [num_seqs, num_q_heads, head_dim], cache dtype
+ *   block_tables  device int32 [num_seqs, bt_stride]
+ *   context_lens  device int32 [num_seqs]; each <= max_context_len and
+ *                 <= bt_stride * block_size
+ *   max_context_len host-known upper bound of context_lens (sizes the split
+ *                 grid and the workspace)
+ *   opts          may be NULL (= split chosen on the device, path AUTO)
+ *   workspace     device buffer of >= pa_decode_workspace_size(...) bytes,
+ *                 16-byte aligned; owned by the caller, used by one call at a
+ *                 time (two calls that overlap on the GPU must not share it).
+ * Accumulation and softmax are fp32; the tensor-core path keeps the
+ * probabilities at ~16 significant bits (two 16-bit terms).
+ */
+pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
+                    const int32_t* block_tables, int32_t bt_stride,
+                    const int32_t* context_lens, int32_t num_seqs,
+                    int32_t num_q_heads, int32_t max_context_len, float scale,
+                    const pa_decode_options* opts, void* workspace,
+                    size_t workspace_bytes, pa_stream_t stream);
+
+/*
+ * pa_decode_status - read back (synchronously, on `stream`) the device status
+ * word the last pa_decode using `workspace` left: PA_OK, or
+ * PA_ERR_DEVICE_TIMEOUT if one of its kernels stopped waiting on a barrier
+ * after its time limit and returned early (its output is then invalid).
+ * The word is cleared on every pa_decode. Returns PA_ERR_CUDA if the copy fails.
+ */
+pa_status pa_decode_status(const void* workspace, pa_stream_t stream);
+
+/* Human-readable name of a status code (static string). */
+const char* pa_status_string(pa_status status);
+
+/* CUDA error string of the last PA_ERR_CUDA on this thread ("" if none). */
+const char* pa_last_cuda_error(void);
+
+/* Library version string. */
+const char* pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGED_KV_CACHE_PA_H */

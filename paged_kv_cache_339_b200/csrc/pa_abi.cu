@@ -1,0 +1,276 @@
+// C-ABI entry points (include/pa.h): host-side argument checks, dispatch,
+// launch. No device memory is allocated or freed here.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/pa.h"
+#include "pa_internal.h"
+
+namespace pa {
+
+namespace {
+
+thread_local char g_cuda_error[256] = "";
+
+pa_status cuda_fail(cudaError_t e) {
+  std::snprintf(g_cuda_error, sizeof(g_cuda_error), "%s: %s",
+                cudaGetErrorName(e), cudaGetErrorString(e));
+  return PA_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+pa_status check_cache(const pa_kv_cache* c) {
+  if (c == nullptr || c->k_cache == nullptr || c->v_cache == nullptr) return PA_ERR_INVALID_ARG;
+  if (c->num_blocks <= 0 || c->num_kv_heads <= 0 || c->block_size <= 0 || c->head_dim <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (c->dtype != PA_F32 && c->dtype != PA_F16 && c->dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (c->head_dim != 64 && c->head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (c->block_size != 8 && c->block_size != 16 && c->block_size != 32) return PA_ERR_UNSUPPORTED;
+  if (!aligned16(c->k_cache) || !aligned16(c->v_cache)) return PA_ERR_MISALIGNED;
+  return PA_OK;
+}
+
+int elem_bytes(int dtype) { return dtype == PA_F32 ? 4 : 2; }
+
+// Persistent-grid sizes, computed once per (device, kernel flavour).
+struct CtaCache {
+  std::mutex mu;
+  int dev = -1;
+  int simt[3][2][3] = {};   // [dtype][head_dim 64/128][gpw 1/2/4]
+  int tc[3][17] = {};       // [dtype][group]
+};
+CtaCache g_ctas;
+
+cudaError_t cached_ctas(bool tc, int dtype, int head_dim, int group, int* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_ctas.mu);
+  if (g_ctas.dev != dev) {
+    std::memset(g_ctas.simt, 0, sizeof(g_ctas.simt));
+    std::memset(g_ctas.tc, 0, sizeof(g_ctas.tc));
+    g_ctas.dev = dev;
+  }
+  int* slot;
+  if (tc) {
+    slot = &g_ctas.tc[dtype][group];
+  } else {
+    const int gpw = group == 1 ? 0 : (group == 2 ? 1 : 2);
+    slot = &g_ctas.simt[dtype][head_dim == 64 ? 0 : 1][gpw];
+  }
+  if (*slot == 0) {
+    e = tc ? tc_num_ctas(dtype, group, slot) : simt_num_ctas(dtype, head_dim, group, slot);
+    if (e != cudaSuccess) {
+      *slot = 0;
+      return e;
+    }
+  }
+  *out = *slot;
+  return cudaSuccess;
+}
+
+constexpr int kItemsPerCta = 12;
+
+}  // namespace
+
+int num_sms() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" {
+
+pa_status pa_write_kv(const pa_kv_cache* cache, const void* key, const void* value,
+                      const int64_t* slot_mapping, int32_t num_tokens, pa_stream_t stream) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (num_tokens < 0) return PA_ERR_INVALID_ARG;
+  if (num_tokens == 0) return PA_OK;
+  if (key == nullptr || value == nullptr || slot_mapping == nullptr) return PA_ERR_INVALID_ARG;
+  if (!aligned16(key) || !aligned16(value) || (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+    return PA_ERR_MISALIGNED;
+  const int32_t row_bytes = cache->head_dim * elem_bytes(cache->dtype);
+  const int64_t num_slots = static_cast<int64_t>(cache->num_blocks) * cache->block_size;
+  cudaError_t e = launch_write_kv(cache->k_cache, cache->v_cache, key, value, slot_mapping,
+                                  num_tokens, cache->num_kv_heads, cache->block_size, row_bytes,
+                                  num_slots, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : cuda_fail(e);
+}
+
+pa_status pa_copy_blocks(const pa_kv_cache* cache, const int64_t* block_pairs, int32_t num_pairs,
+                         pa_stream_t stream) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (num_pairs < 0) return PA_ERR_INVALID_ARG;
+  if (num_pairs == 0) return PA_OK;
+  if (block_pairs == nullptr) return PA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(block_pairs) & 7u) return PA_ERR_MISALIGNED;
+  const int64_t block_bytes = static_cast<int64_t>(cache->num_kv_heads) * cache->block_size *
+                              cache->head_dim * elem_bytes(cache->dtype);
+  cudaError_t e = launch_copy_blocks(cache->k_cache, cache->v_cache, block_pairs, num_pairs,
+                                     block_bytes, cache->num_blocks,
+                                     static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : cuda_fail(e);
+}
+
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+                                int32_t max_context_len, int32_t block_size,
+                                int32_t split_tokens) {
+  (void)block_size;
+  if (num_seqs < 0 || num_q_heads < 0 || head_dim < 0 || max_context_len < 0) return 0;
+  return ws_layout(num_seqs, num_q_heads, head_dim, max_context_len, split_tokens).total;
+}
+
+pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
+                    const int32_t* block_tables, int32_t bt_stride, const int32_t* context_lens,
+                    int32_t num_seqs, int32_t num_q_heads, int32_t max_context_len, float scale,
+                    const pa_decode_options* opts, void* workspace, size_t workspace_bytes,
+                    pa_stream_t stream) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (num_seqs < 0 || num_q_heads <= 0 || max_context_len < 0) return PA_ERR_INVALID_ARG;
+  if (num_q_heads % cache->num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+  const int group = num_q_heads / cache->num_kv_heads;
+  if (group > 16) return PA_ERR_UNSUPPORTED;
+  if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+  const int32_t split = opts ? opts->split_tokens : 0;
+  const int32_t path = opts ? opts->path : PA_PATH_AUTO;
+  if (split < 0 || path < PA_PATH_AUTO || path > PA_PATH_TCGEN05) return PA_ERR_INVALID_ARG;
+  if (split > 0) {
+    if (split % cache->block_size != 0) return PA_ERR_INVALID_ARG;
+    if (max_context_len > 0 && ceil_div(max_context_len, split) > kMaxSplits)
+      return PA_ERR_INVALID_ARG;
+  }
+  if (num_seqs == 0) return PA_OK;
+  if (out == nullptr || q == nullptr || block_tables == nullptr || context_lens == nullptr ||
+      workspace == nullptr)
+    return PA_ERR_INVALID_ARG;
+  if (bt_stride <= 0) return PA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(max_context_len) > static_cast<int64_t>(bt_stride) * cache->block_size)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(workspace) ||
+      (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
+      (reinterpret_cast<uintptr_t>(context_lens) & 3u))
+    return PA_ERR_MISALIGNED;
+  const WsLayout lay = ws_layout(num_seqs, num_q_heads, cache->head_dim, max_context_len, split);
+  if (workspace_bytes < lay.total) return PA_ERR_WORKSPACE_TOO_SMALL;
+
+  const bool tc_ok = tc_supported(cache->dtype, cache->head_dim, group);
+  bool use_tc = false;
+  if (path == PA_PATH_TCGEN05) {
+    if (!tc_ok) return PA_ERR_UNSUPPORTED;
+    use_tc = true;
+  } else if (path == PA_PATH_AUTO) {
+    use_tc = tc_ok;
+  }
+  if (!use_tc && !simt_supported(cache->dtype, cache->head_dim, group)) return PA_ERR_UNSUPPORTED;
+
+  int ctas = 0;
+  cudaError_t e = cached_ctas(use_tc, cache->dtype, cache->head_dim, group, &ctas);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+
+  PlanParams pp;
+  pp.context_lens = context_lens;
+  pp.out = out;
+  pp.ws = ws;
+  pp.pairs_off = lay.pairs_off;
+  pp.nsplit_off = lay.nsplit_off;
+  pp.num_seqs = num_seqs;
+  pp.num_q_heads = num_q_heads;
+  pp.num_kv_heads = cache->num_kv_heads;
+  pp.head_dim = cache->head_dim;
+  pp.bt_stride = bt_stride;
+  pp.block_size = cache->block_size;
+  pp.max_context_len = max_context_len;
+  pp.split_tokens = split;
+  pp.min_split = split > 0 ? split : auto_min_split(max_context_len);
+  pp.max_splits = lay.max_splits;
+  pp.num_ctas = ctas;
+  pp.items_per_cta = kItemsPerCta;
+  e = launch_plan(pp, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+
+  DecodeParams dp;
+  dp.k_cache = cache->k_cache;
+  dp.v_cache = cache->v_cache;
+  dp.q = q;
+  dp.out = out;
+  dp.block_tables = block_tables;
+  dp.ws = ws;
+  dp.pairs_off = lay.pairs_off;
+  dp.ml_off = lay.ml_off;
+  dp.o_off = lay.o_off;
+  dp.bt_stride = bt_stride;
+  dp.num_blocks = cache->num_blocks;
+  dp.num_kv_heads = cache->num_kv_heads;
+  dp.num_q_heads = num_q_heads;
+  dp.head_dim = cache->head_dim;
+  dp.block_size = cache->block_size;
+  dp.num_seqs = num_seqs;
+  dp.max_splits = lay.max_splits;
+  dp.scale_log2 = scale * 1.4426950408889634f;
+  dp.dtype = cache->dtype;
+  e = use_tc ? launch_decode_tc(dp, ctas, s) : launch_decode_simt(dp, ctas, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+
+  MergeParams mp;
+  mp.out = out;
+  mp.ws = ws;
+  mp.nsplit_off = lay.nsplit_off;
+  mp.ml_off = lay.ml_off;
+  mp.o_off = lay.o_off;
+  mp.num_seqs = num_seqs;
+  mp.num_q_heads = num_q_heads;
+  mp.num_kv_heads = cache->num_kv_heads;
+  mp.head_dim = cache->head_dim;
+  mp.max_splits = lay.max_splits;
+  e = launch_merge(mp, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return PA_OK;
+}
+
+pa_status pa_decode_status(const void* workspace, pa_stream_t stream) {
+  if (workspace == nullptr) return PA_ERR_INVALID_ARG;
+  int32_t word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost,
+                                  static_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess) e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return static_cast<pa_status>(word);
+}
+
+const char* pa_status_string(pa_status status) {
+  switch (status) {
+    case PA_OK: return "PA_OK";
+    case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG: invalid argument";
+    case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED: shape or dtype not supported";
+    case PA_ERR_MISALIGNED: return "PA_ERR_MISALIGNED: pointer not 16-byte aligned";
+    case PA_ERR_WORKSPACE_TOO_SMALL: return "PA_ERR_WORKSPACE_TOO_SMALL: workspace too small";
+    case PA_ERR_CUDA: return "PA_ERR_CUDA: CUDA call failed";
+    case PA_ERR_DEVICE_TIMEOUT: return "PA_ERR_DEVICE_TIMEOUT: a kernel gave up waiting";
+  }
+  return "unknown pa_status";
+}
+
+const char* pa_last_cuda_error(void) { return g_cuda_error; }
+
+const char* pa_version(void) { return "pagedattn 0.1.0 (sm_100a)"; }
+
+}  // extern "C"

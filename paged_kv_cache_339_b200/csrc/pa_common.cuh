@@ -1,0 +1,213 @@
+// Device helpers shared by the paged-KV kernels (sm_100a only).
+//
+// Everything asynchronous here is a plain CTA-local form: bulk copies and TMA
+// tensor loads write this CTA's shared memory, completion is tracked by
+// mbarrier transaction counts, and no copy uses cluster multicast.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pa_workspace.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "this library is built for sm_100a only"
+#endif
+
+namespace pa {
+
+// Time limit of every barrier wait in the kernels (nanoseconds). A correct
+// launch never comes near it; if a wait does run out, the kernel records
+// PA_ERR_DEVICE_TIMEOUT in the workspace status word and returns early.
+constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long global_timer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar,
+                                                      uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(
+                   smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait until the phase with the given parity of `bar` has completed, for at
+// most kWaitLimitNs. On time-out (or when another role of the CTA already
+// gave up, `abrt` != 0) it records the status, raises `abrt` and returns
+// false; callers then leave their loops.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          volatile int* abrt,
+                                          int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 31u) == 0) {
+      if (*abrt) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        *abrt = 1;
+        atomicExch(status, 6 /* PA_ERR_DEVICE_TIMEOUT */);
+        return false;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Bulk copies global -> this CTA's shared memory (no multicast)
+// ---------------------------------------------------------------------------
+// Contiguous bytes; dst/src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src,
+                                         uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// 2-D tiled TMA load of the box at (x, y) of `tmap` (x innermost, in
+// elements; x * element size must be a multiple of 16 bytes).
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tmap,
+                                            int32_t x, int32_t y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::"
+      "complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y),
+      "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* tmap) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap))
+               : "memory");
+}
+
+// Generic-proxy writes to shared memory made visible to the async proxy
+// (tensor core / TMA) before they read or overwrite it.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Named barrier among `nthreads` threads (id 0 is __syncthreads).
+__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Element conversions (exact widening to fp32)
+// ---------------------------------------------------------------------------
+template <typename T>
+struct Elem;
+
+template <>
+struct Elem<float> {
+  static constexpr int kBytes = 4;
+  __device__ static __forceinline__ void unpack4(const uint4& v, float* f) {
+    f[0] = __uint_as_float(v.x);
+    f[1] = __uint_as_float(v.y);
+    f[2] = __uint_as_float(v.z);
+    f[3] = __uint_as_float(v.w);
+  }
+  __device__ static __forceinline__ float load1(const void* p) {
+    return *reinterpret_cast<const float*>(p);
+  }
+};
+
+template <>
+struct Elem<__nv_bfloat16> {
+  static constexpr int kBytes = 2;
+  // bf16 -> fp32 is a 16-bit left shift of the bit pattern.
+  __device__ static __forceinline__ void unpack2(uint32_t w, float* f) {
+    f[0] = __uint_as_float(w << 16);
+    f[1] = __uint_as_float(w & 0xffff0000u);
+  }
+  __device__ static __forceinline__ float load1(const void* p) {
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(p));
+  }
+};
+
+template <>
+struct Elem<__half> {
+  static constexpr int kBytes = 2;
+  __device__ static __forceinline__ void unpack2(uint32_t w, float* f) {
+    __half2 h = *reinterpret_cast<__half2*>(&w);
+    float2 x = __half22float2(h);
+    f[0] = x.x;
+    f[1] = x.y;
+  }
+  __device__ static __forceinline__ float load1(const void* p) {
+    return __half2float(*reinterpret_cast<const __half*>(p));
+  }
+};
+
+// Unpack a 16-byte vector into fp32 values: 4 (fp32) or 8 (16-bit types).
+template <typename T>
+__device__ __forceinline__ void unpack16(const uint4& v, float* f) {
+  if constexpr (sizeof(T) == 4) {
+    Elem<float>::unpack4(v, f);
+  } else {
+    Elem<T>::unpack2(v.x, f + 0);
+    Elem<T>::unpack2(v.y, f + 2);
+    Elem<T>::unpack2(v.z, f + 4);
+    Elem<T>::unpack2(v.w, f + 6);
+  }
+}
+
+// Work-item record written by the planning kernel: one per (sequence, split);
+// the KV-head index is folded into the claimed item number.
+struct __align__(16) WorkPair {
+  int32_t seq;
+  int32_t split;
+  int32_t t_begin;  // first token of the range
+  int32_t t_end;    // one past the last token; the sequence has one split
+                    // iff split == 0 and t_end == context length (flag below)
+};
+constexpr int32_t kSingleFlag = 1 << 30;  // set in `split` when the item is the
+                                          // whole sequence (output written directly)
+
+}  // namespace pa

@@ -1,0 +1,76 @@
+// Host-side declarations shared by the C-ABI shim and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "pa_workspace.h"
+
+namespace pa {
+
+struct PlanParams {
+  const int32_t* context_lens;
+  float* out;
+  uint8_t* ws;
+  size_t pairs_off, nsplit_off;
+  int32_t num_seqs, num_q_heads, num_kv_heads, head_dim;
+  int32_t bt_stride, block_size, max_context_len;
+  int32_t split_tokens;   // explicit split, or 0 = choose on the device
+  int32_t min_split;      // lower bound of an automatic split
+  int32_t max_splits;
+  int32_t num_ctas;       // persistent CTAs of the decode kernel
+  int32_t items_per_cta;  // target work items per CTA (automatic split)
+};
+
+struct MergeParams {
+  float* out;
+  const uint8_t* ws;
+  size_t nsplit_off, ml_off, o_off;
+  int32_t num_seqs, num_q_heads, num_kv_heads, head_dim, max_splits;
+};
+
+// Everything a decode main kernel needs; filled by the C-ABI shim.
+struct DecodeParams {
+  const void* k_cache;
+  const void* v_cache;
+  const void* q;
+  float* out;
+  const int32_t* block_tables;
+  uint8_t* ws;
+  size_t pairs_off, ml_off, o_off;
+  int32_t bt_stride, num_blocks, num_kv_heads, num_q_heads, head_dim,
+      block_size, num_seqs, max_splits;
+  float scale_log2;  // scale * log2(e): scores kept in log2 units
+  int32_t dtype;     // pa_dtype
+};
+
+cudaError_t launch_plan(const PlanParams& p, cudaStream_t stream);
+cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream);
+
+// CUDA-core decode. Returns cudaErrorInvalidValue for an unsupported shape.
+bool simt_supported(int dtype, int head_dim, int group);
+cudaError_t simt_num_ctas(int dtype, int head_dim, int group, int* num_ctas);
+cudaError_t launch_decode_simt(const DecodeParams& p, int num_ctas,
+                               cudaStream_t stream);
+
+// Tensor-core (tcgen05) decode for 16-bit KV, head_dim 128, 4 <= G <= 16.
+bool tc_supported(int dtype, int head_dim, int group);
+cudaError_t tc_num_ctas(int dtype, int group, int* num_ctas);
+cudaError_t launch_decode_tc(const DecodeParams& p, int num_ctas,
+                             cudaStream_t stream);
+
+// KV write and block copy.
+cudaError_t launch_write_kv(void* k_cache, void* v_cache, const void* key,
+                            const void* value, const int64_t* slots,
+                            int32_t num_tokens, int32_t num_kv_heads,
+                            int32_t block_size, int32_t row_bytes,
+                            int64_t num_slots, cudaStream_t stream);
+cudaError_t launch_copy_blocks(void* k_cache, void* v_cache,
+                               const int64_t* pairs, int32_t num_pairs,
+                               int64_t block_bytes, int32_t num_blocks,
+                               cudaStream_t stream);
+
+int num_sms();
+
+}  // namespace pa

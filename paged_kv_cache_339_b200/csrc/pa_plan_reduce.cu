@@ -1,0 +1,228 @@
+// Work planning and split-context merge for pa_decode.
+//
+// plan_kernel (one CTA) reads the context lengths, checks them, picks the
+// split size, and writes the list of (sequence, split) work pairs in
+// split-major order (every sequence's first split, then every second split,
+// ...), so the persistent decode kernels claim the longest ranges first.
+//
+// merge_kernel combines the partial softmax results of sequences that were
+// split: with per-split running max m_p (log2 units), sum l_p and
+// unnormalised accumulator a_p,
+//   M = max_p m_p,  L = sum_p l_p 2^(m_p - M),  o = sum_p a_p 2^(m_p - M) / L.
+// This regrouping is exact algebra on the softmax sums; the pages do not
+// discuss splitting a context.
+#include "pa_common.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+
+namespace {
+
+constexpr int kPlanThreads = 1024;
+
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  return v;
+}
+
+// Exclusive scan of one int per thread over the CTA; returns the prefix and
+// writes the total to *total (all threads).
+__device__ int block_excl_scan(int v, int* scratch, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int inc = warp_incl_scan(v, lane);
+  if (lane == 31) scratch[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < (kPlanThreads / 32) ? scratch[lane] : 0;
+    int wi = warp_incl_scan(w, lane);
+    scratch[32 + lane] = wi - w;
+    if (lane == 31) scratch[64] = wi;
+  }
+  __syncthreads();
+  int res = scratch[32 + warp] + inc - v;
+  *total = scratch[64];
+  __syncthreads();
+  return res;
+}
+
+__global__ void __launch_bounds__(kPlanThreads, 1)
+    plan_kernel(PlanParams p) {
+  __shared__ long long s_sum[32];
+  __shared__ int s_max[32];
+  __shared__ int s_bad[32];
+  __shared__ int s_scan[96];
+  __shared__ int s_split;
+  __shared__ int s_maxn;
+
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(p.ws);
+  WorkPair* pairs = reinterpret_cast<WorkPair*>(p.ws + p.pairs_off);
+  int32_t* nsplit = reinterpret_cast<int32_t*>(p.ws + p.nsplit_off);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t cap = static_cast<int64_t>(p.bt_stride) * p.block_size;
+
+  // 1. validate lengths, total and maximum
+  long long tot = 0;
+  int mx = 0, bad = 0;
+  for (int i = tid; i < p.num_seqs; i += kPlanThreads) {
+    const int L = p.context_lens[i];
+    if (L < 0 || L > p.max_context_len || L > cap) {
+      bad = 1;
+    } else {
+      tot += L;
+      mx = max(mx, L);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    tot += __shfl_xor_sync(0xffffffffu, tot, o);
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    bad |= __shfl_xor_sync(0xffffffffu, bad, o);
+  }
+  if (lane == 0) {
+    s_sum[warp] = tot;
+    s_max[warp] = mx;
+    s_bad[warp] = bad;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    long long t = 0;
+    int m = 0, b = 0;
+    for (int w = 0; w < kPlanThreads / 32; ++w) {
+      t += s_sum[w];
+      m = max(m, s_max[w]);
+      b |= s_bad[w];
+    }
+    int S = p.split_tokens;
+    if (S <= 0) {
+      // Aim for ~items_per_cta work items per persistent CTA.
+      long long per_cta = (t * p.num_kv_heads + p.num_ctas - 1) / p.num_ctas;
+      long long want = (per_cta + p.items_per_cta - 1) / p.items_per_cta;
+      want = (want + kAutoSplitQuantum - 1) / kAutoSplitQuantum * kAutoSplitQuantum;
+      if (want < p.min_split) want = p.min_split;
+      if (want > (1 << 30)) want = 1 << 30;
+      S = static_cast<int>(want);
+    }
+    s_split = S;
+    s_maxn = m > 0 ? (m + S - 1) / S : 0;
+    hdr->status = b ? 1 /* PA_ERR_INVALID_ARG */ : 0;
+    hdr->split_tokens = S;
+    hdr->max_splits = p.max_splits;
+  }
+  __syncthreads();
+  const int S = s_split;
+  const int maxn = min(s_maxn, p.max_splits);
+
+  // 2. splits per sequence; sequences with nothing to attend to get zero rows
+  for (int i = tid; i < p.num_seqs; i += kPlanThreads) {
+    const int L = p.context_lens[i];
+    const bool ok = !(L < 0 || L > p.max_context_len || L > cap);
+    const int n = (ok && L > 0) ? (L + S - 1) / S : 0;
+    nsplit[i] = n;
+    if (n == 0) {
+      float4* row = reinterpret_cast<float4*>(
+          p.out + static_cast<size_t>(i) * p.num_q_heads * p.head_dim);
+      const int n4 = p.num_q_heads * p.head_dim / 4;
+      for (int e = 0; e < n4; ++e) row[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  __syncthreads();
+
+  // 3. split-major pair list
+  int base = 0;
+  for (int s = 0; s < maxn; ++s) {
+    for (int i0 = 0; i0 < p.num_seqs; i0 += kPlanThreads) {
+      const int i = i0 + tid;
+      int n = 0, L = 0;
+      if (i < p.num_seqs) {
+        n = nsplit[i];
+        L = p.context_lens[i];
+      }
+      const int f = (n > s) ? 1 : 0;
+      int count;
+      const int rank = block_excl_scan(f, s_scan, &count);
+      if (f) {
+        WorkPair w;
+        w.seq = i;
+        w.split = s | (n == 1 ? kSingleFlag : 0);
+        w.t_begin = s * S;
+        w.t_end = min(L, (s + 1) * S);
+        pairs[base + rank] = w;
+      }
+      base += count;
+    }
+  }
+  if (tid == 0) {
+    hdr->num_pairs = base;
+    hdr->num_items = base * p.num_kv_heads;
+    hdr->work_counter = 0;
+  }
+}
+
+constexpr int kMergeThreads = 256;
+
+__global__ void __launch_bounds__(kMergeThreads)
+    merge_kernel(MergeParams p) {
+  extern __shared__ float s_w[];  // [G][max_splits] normalised weights
+  const int seq = blockIdx.x / p.num_kv_heads;
+  const int kvh = blockIdx.x % p.num_kv_heads;
+  const int32_t* nsplit = reinterpret_cast<const int32_t*>(p.ws + p.nsplit_off);
+  const int n = nsplit[seq];
+  if (n <= 1) return;
+  const int G = p.num_q_heads / p.num_kv_heads;
+  const float2* ml = reinterpret_cast<const float2*>(p.ws + p.ml_off);
+  const float* po = reinterpret_cast<const float*>(p.ws + p.o_off);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+  for (int g = warp; g < G; g += kMergeThreads / 32) {
+    const size_t row = static_cast<size_t>(seq) * p.num_q_heads + kvh * G + g;
+    const float2* r = ml + row * p.max_splits;
+    float M = -INFINITY;
+    for (int s = lane; s < n; s += 32) M = fmaxf(M, r[s].x);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.f;
+    for (int s = lane; s < n; s += 32) L += r[s].y * exp2f(r[s].x - M);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    const float inv = 1.0f / L;
+    for (int s = lane; s < n; s += 32) s_w[g * p.max_splits + s] = exp2f(r[s].x - M) * inv;
+  }
+  __syncthreads();
+  const int D = p.head_dim;
+  for (int idx = threadIdx.x; idx < G * D; idx += kMergeThreads) {
+    const int g = idx / D, d = idx % D;
+    const size_t row = static_cast<size_t>(seq) * p.num_q_heads + kvh * G + g;
+    const float* src = po + row * p.max_splits * D + d;
+    const float* w = s_w + g * p.max_splits;
+    float acc = 0.f;
+    for (int s = 0; s < n; ++s) acc = fmaf(w[s], src[static_cast<size_t>(s) * D], acc);
+    p.out[row * D + d] = acc;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_plan(const PlanParams& p, cudaStream_t stream) {
+  plan_kernel<<<1, kPlanThreads, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream) {
+  if (p.max_splits <= 1 || p.num_seqs == 0) return cudaSuccess;
+  const int G = p.num_q_heads / p.num_kv_heads;
+  const size_t smem = static_cast<size_t>(G) * p.max_splits * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(
+        merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  merge_kernel<<<p.num_seqs * p.num_kv_heads, kMergeThreads, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace pa
