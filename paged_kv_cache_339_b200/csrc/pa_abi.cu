@@ -170,7 +170,9 @@ pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
   const WsLayout lay = ws_layout(num_seqs, num_q_heads, cache->head_dim, max_context_len, split);
   if (workspace_bytes < lay.total) return PA_ERR_WORKSPACE_TOO_SMALL;
 
-  const bool tc_ok = tc_supported(cache->dtype, cache->head_dim, group);
+  // the tensor-core kernel loads query tiles of 16 rows: it needs >= 16 query rows
+  const bool tc_ok = tc_supported(cache->dtype, cache->head_dim, group) &&
+                     static_cast<int64_t>(num_seqs) * num_q_heads >= 16;
   bool use_tc = false;
   if (path == PA_PATH_TCGEN05) {
     if (!tc_ok) return PA_ERR_UNSUPPORTED;

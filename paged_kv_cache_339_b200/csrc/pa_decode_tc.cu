@@ -1,9 +1,598 @@
-// Tensor-core decode (placeholder until the tcgen05 kernel lands).
+// Paged decode on the 5th-generation tensor cores (tcgen05), for 16-bit KV,
+// head_dim 128 and 4..16 query heads per KV head. With grouped-query
+// attention ("Paged Attention: Virtual Memory for the KV Cache", "What it does
+// not fix") the G query heads that share a KV head form a real dense tile, so
+// the two contractions of a 128-token chunk run as MMAs:
+//
+//   S^T[128 tok, 16] = K[128 tok, 128 d] . Q^T[128 d, 16]     (A = K, K-major)
+//   O^T[128 d, NPV]  = V^T[128 d, 128 tok] . P^T[128 tok, NPV] (A = V^T, MN-major)
+//
+// Query heads sit on the N side (padded to 16; spare columns are ignored).
+// The probabilities are rounded to 16 bits for the second MMA as a sum of two
+// terms, p = hi + lo (columns [0, NPV/2) and [NPV/2, NPV) of P^T), so the
+// product keeps ~16 significant bits of p at no extra tensor-core passes.
+//
+// Persistent, warp-specialised CTA (one per SM, ~215 KB shared memory):
+//   warp 0     producer: claims (sequence, split, KV head) items, follows the
+//              block table, and loads each page's K and V tile (two 64-column
+//              halves each) plus the Q tile with 2-D TMA (128-byte swizzle)
+//              into a 3-stage ring; completion by mbarrier transaction count.
+//   warp 1     allocates TMEM and issues the MMAs (one elected lane); S^T and
+//              O^T accumulators live in TMEM, double-buffered, so the scores
+//              of chunk c+1 are computed while chunk c's softmax runs.
+//   warps 2-5  softmax and correction: thread r owns token r of a chunk for
+//              the softmax (tcgen05.ld of its S^T row), and output column d = r
+//              for the correction O += alpha * O_chunk; partial results of
+//              split items go to the workspace for the merge kernel.
+// No load uses cluster multicast; every wait is bounded (see pa_common.cuh).
+#include <cudaTypedefs.h>
+
+#include <mutex>
+#include <type_traits>
+
 #include "pa_common.cuh"
 #include "pa_internal.h"
 
 namespace pa {
-bool tc_supported(int, int, int) { return false; }
-cudaError_t tc_num_ctas(int, int, int*) { return cudaErrorInvalidValue; }
-cudaError_t launch_decode_tc(const DecodeParams&, int, cudaStream_t) { return cudaErrorInvalidValue; }
+
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+constexpr int kFirst = 1, kLast = 2, kEnd = 4;
+constexpr int kChunk = 128;   // tokens per stage (= MMA M)
+constexpr int kD = 128;       // head_dim
+constexpr int kNst = 3;       // pipeline stages
+constexpr int kHalf = kChunk * 128;           // one 64-column half: 128 rows x 128 B
+constexpr int kQHalf = 16 * 128;              // Q half: 16 rows x 128 B
+constexpr int kStage = 4 * kHalf + 2 * kQHalf;  // K (2 halves), V (2 halves), Q (2 halves)
+constexpr int kThreads = 192;
+
+struct __align__(16) ChunkMeta {
+  int32_t seq, kvh, split_raw, t0, valid, flags, pad0, pad1;
+};
+
+template <int NPV>
+struct TcLayout {
+  static constexpr int GQ = NPV / 2;                 // max query heads
+  static constexpr int PBUF = (NPV / 8) * 2048;      // P^T buffer bytes
+  static constexpr size_t OFF_P = static_cast<size_t>(kNst) * kStage;
+  static constexpr size_t OFF_BAR = OFF_P + 2 * PBUF;
+  // barriers: full[3], empty[3], s_full[2], s_free[2], p_full[2], o_full[2],
+  // o_free[2], grp, drain
+  static constexpr int NBAR = 2 * kNst + 10 + 2;
+  static constexpr size_t OFF_META = OFF_BAR + NBAR * 8;
+  static constexpr size_t OFF_RED = OFF_META + kNst * sizeof(ChunkMeta);
+  static constexpr size_t OFF_LRED = OFF_RED + 2 * 4 * 16 * 4;
+  static constexpr size_t OFF_MISC = OFF_LRED + 4 * 16 * 4;
+  static constexpr size_t SMEM_USED = OFF_MISC + 16;
+  static constexpr size_t SMEM = SMEM_USED + 1024;   // slack to align the base to 1 KB
+  static constexpr uint32_t TMEM_COLS = (32 + 2 * NPV) <= 64 ? 64 : 128;
+};
+
+// ---------------------------------------------------------------------------
+// tcgen05 wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor (sm_100 format): start address, leading and
+// stride byte offsets (16-byte units), version 1, layout type in bits 61-63.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo,
+                                              uint32_t layout) {
+  return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) |
+         (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) |
+         (static_cast<uint64_t>(layout) << 61);
+}
+constexpr uint32_t kSw128 = 2, kSwNone = 0;
+
+// Instruction descriptor, kind::f16 with fp32 accumulation.
+__host__ __device__ constexpr uint32_t instr_desc(uint32_t fmt, bool a_mn, bool b_mn, int M, int N) {
+  return (1u << 4) | (fmt << 7) | (fmt << 10) | ((a_mn ? 1u : 0u) << 15) |
+         ((b_mn ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* f) {
+  uint32_t v[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) f[i] = __uint_as_float(v[i]);
+}
+
+// Round p to 16 bits (hi) and the remainder p - hi to 16 bits (lo): raw bits.
+template <typename T>
+__device__ __forceinline__ void split16(float p, uint16_t& hi, uint16_t& lo) {
+  if constexpr (sizeof(T) == 2 && std::is_same<T, __nv_bfloat16>::value) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(p);
+    const __nv_bfloat16 l = __float2bfloat16_rn(p - __bfloat162float(h));
+    hi = *reinterpret_cast<const uint16_t*>(&h);
+    lo = *reinterpret_cast<const uint16_t*>(&l);
+  } else {
+    const __half h = __float2half_rn(p);
+    const __half l = __float2half_rn(p - __half2float(h));
+    hi = *reinterpret_cast<const uint16_t*>(&h);
+    lo = *reinterpret_cast<const uint16_t*>(&l);
+  }
+}
+
+__device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t& phase, volatile int* abrt,
+                                           int* status) {
+  mbar_arrive(bar);
+  const bool ok = mbar_wait(bar, phase, abrt, status);
+  phase ^= 1u;
+  return ok;
+}
+
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const unsigned long long t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > kWaitLimitNs) break;
+  }
+}
+
+template <typename T, int NPV>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v,
+                     const __grid_constant__ CUtensorMap tm_q) {
+  using Ly = TcLayout<NPV>;
+  constexpr int GQ = Ly::GQ;
+  extern __shared__ uint8_t smem_raw[];
+  // 1 KB alignment for the 128-byte-swizzled tiles
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* pbuf = smem + Ly::OFF_P;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Ly::OFF_BAR);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kNst;
+  uint64_t* s_full = bars + 2 * kNst;
+  uint64_t* s_free = s_full + 2;
+  uint64_t* p_full = s_free + 2;
+  uint64_t* o_full = p_full + 2;
+  uint64_t* o_free = o_full + 2;
+  uint64_t* grp = o_free + 2;
+  uint64_t* drain = grp + 1;
+  ChunkMeta* meta = reinterpret_cast<ChunkMeta*>(smem + Ly::OFF_META);
+  float* red = reinterpret_cast<float*>(smem + Ly::OFF_RED);    // [2][4][16]
+  float* lred = reinterpret_cast<float*>(smem + Ly::OFF_LRED);  // [4][16]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Ly::OFF_MISC);
+  volatile int* abrt = reinterpret_cast<volatile int*>(smem + Ly::OFF_MISC + 4);
+
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(p.ws);
+  int* status = &hdr->status;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kNst; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_free[b], 128);
+      mbar_init(&p_full[b], 128);
+      mbar_init(&o_full[b], 1);
+      mbar_init(&o_free[b], 128);
+    }
+    mbar_init(grp, 128);
+    mbar_init(drain, 1);
+    *abrt = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_holder)),
+                 "r"(Ly::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  const int num_items = hdr->num_items;
+  const int Hkv = p.num_kv_heads, BS = p.block_size;
+  const int G = p.num_q_heads / Hkv;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      prefetch_tmap(&tm_q);
+    }
+    const WorkPair* pairs = reinterpret_cast<const WorkPair*>(p.ws + p.pairs_off);
+    uint32_t c = 0;
+    bool ok = true;
+    int kraw = 0;
+    if (lane == 0) kraw = atomicAdd(&hdr->work_counter, 1);
+    int k = __shfl_sync(kFull, kraw, 0);
+    while (k < num_items) {
+      const int pi = k / Hkv, kvh = k - pi * Hkv;
+      const WorkPair wp = pairs[pi];
+      if (lane == 0) kraw = atomicAdd(&hdr->work_counter, 1);
+      const int32_t* bt_row = p.block_tables + static_cast<size_t>(wp.seq) * p.bt_stride;
+      const int q_row = wp.seq * p.num_q_heads + kvh * G;
+      for (int cs = wp.t_begin; cs < wp.t_end; cs += kChunk) {
+        const int valid = min(kChunk, wp.t_end - cs);
+        const int npg = (valid + BS - 1) / BS;
+        int blk = 0;
+        if (lane < npg) {
+          blk = bt_row[cs / BS + lane];
+          if (blk < 0 || blk >= p.num_blocks) {
+            atomicCAS(status, 0, 1 /* PA_ERR_INVALID_ARG */);
+            blk = 0;
+          }
+        }
+        const int stage = c % kNst;
+        if (!mbar_wait(&empty[stage], ((c / kNst) & 1u) ^ 1u, abrt, status)) {
+          ok = false;
+          break;
+        }
+        uint8_t* st = smem + static_cast<size_t>(stage) * kStage;
+        if (lane == 0) {
+          ChunkMeta m;
+          m.seq = wp.seq;
+          m.kvh = kvh;
+          m.split_raw = wp.split;
+          m.t0 = cs;
+          m.valid = valid;
+          m.flags = (cs == wp.t_begin ? kFirst : 0) | (cs + kChunk >= wp.t_end ? kLast : 0);
+          m.pad0 = m.pad1 = 0;
+          meta[stage] = m;
+          mbar_arrive_expect_tx(&full[stage],
+                                static_cast<uint32_t>(npg * BS * 512 + 2 * kQHalf));
+          tma_load_2d(st + 4 * kHalf, &tm_q, 0, q_row, &full[stage]);
+          tma_load_2d(st + 4 * kHalf + kQHalf, &tm_q, 64, q_row, &full[stage]);
+        }
+        __syncwarp();
+        if (lane < npg) {
+          const int row = (blk * Hkv + kvh) * BS;
+          const int off = lane * BS * 128;
+          tma_load_2d(st + off, &tm_k, 0, row, &full[stage]);
+          tma_load_2d(st + kHalf + off, &tm_k, 64, row, &full[stage]);
+          tma_load_2d(st + 2 * kHalf + off, &tm_v, 0, row, &full[stage]);
+          tma_load_2d(st + 3 * kHalf + off, &tm_v, 64, row, &full[stage]);
+        }
+        ++c;
+      }
+      if (!ok) break;
+      k = __shfl_sync(kFull, kraw, 0);
+    }
+    if (ok) {
+      const int stage = c % kNst;
+      if (mbar_wait(&empty[stage], ((c / kNst) & 1u) ^ 1u, abrt, status)) {
+        if (lane == 0) {
+          meta[stage].flags = kEnd;
+          mbar_arrive(&full[stage]);
+        }
+      } else {
+        ok = false;
+      }
+    }
+    if (!ok && lane == 0) {
+      for (uint32_t cc = c > kNst ? c - kNst : 0; cc < c; ++cc)
+        drain_wait(&full[cc % kNst], (cc / kNst) & 1u);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t fmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
+      const uint32_t idesc_s = instr_desc(fmt, false, false, 128, 16);
+      const uint32_t idesc_pv = instr_desc(fmt, true, true, 128, NPV);
+      const uint32_t sbase = smem_u32(smem);
+      const uint32_t pbase = smem_u32(pbuf);
+
+      auto issue_s = [&](uint32_t cc) {
+        const uint32_t st = sbase + (cc % kNst) * kStage;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t half = kk >> 2, koff = (kk & 3) * 32;
+          const uint64_t a = smem_desc(st + half * kHalf + koff, 16, 1024, kSw128);
+          const uint64_t b = smem_desc(st + 4 * kHalf + half * kQHalf + koff, 16, 1024, kSw128);
+          mma_f16(tmem + 16 * (cc & 1), a, b, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&s_full[cc & 1]);
+      };
+      auto issue_pv = [&](uint32_t cc, int valid) {
+        const uint32_t st = sbase + (cc % kNst) * kStage;
+        const uint32_t pb = pbase + (cc & 1) * Ly::PBUF;
+        const int nks = (valid + 15) >> 4;
+        for (int ks = 0; ks < nks; ++ks) {
+          const uint64_t a = smem_desc(st + 2 * kHalf + ks * 2048, kHalf, 1024, kSw128);
+          const uint64_t b = smem_desc(pb + ks * 256, 128, 2048, kSwNone);
+          mma_f16(tmem + 32 + NPV * (cc & 1), a, b, idesc_pv, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(&o_full[cc & 1]);
+        mma_commit(&empty[cc % kNst]);
+      };
+
+      uint32_t c = 0;
+      bool ok = mbar_wait(&full[0], 0, abrt, status);
+      ChunkMeta cur = meta[0];
+      if (ok && !(cur.flags & kEnd)) {
+        tc_fence_after();
+        issue_s(0);
+      }
+      while (ok && !(cur.flags & kEnd)) {
+        const uint32_t c1 = c + 1;
+        if (!mbar_wait(&full[c1 % kNst], (c1 / kNst) & 1u, abrt, status)) break;
+        const ChunkMeta nxt = meta[c1 % kNst];
+        if (!(nxt.flags & kEnd)) {
+          if (!mbar_wait(&s_free[c1 & 1], ((c1 >> 1) & 1u) ^ 1u, abrt, status)) break;
+          tc_fence_after();
+          issue_s(c1);
+        }
+        if (!mbar_wait(&p_full[c & 1], (c >> 1) & 1u, abrt, status)) break;
+        if (!mbar_wait(&o_free[c & 1], ((c >> 1) & 1u) ^ 1u, abrt, status)) break;
+        tc_fence_after();
+        issue_pv(c, cur.valid);
+        c = c1;
+        cur = nxt;
+      }
+      // all MMAs this thread issued have completed before TMEM is released
+      mma_commit(drain);
+      drain_wait(drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax / correction
+    const int r = 32 * (warp & 3) + lane;   // TMEM lane: token (softmax) / column d (output)
+    const int wq = warp - 2;                 // 0..3 among the softmax warps
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+    const float sl2 = p.scale_log2;
+    float m_run[GQ], l_thr[GQ], o[GQ], a_prev[GQ];
+    uint32_t c = 0, gphase = 0;
+    bool have_prev = false;
+    uint32_t c_prev = 0;
+    float2* ml = reinterpret_cast<float2*>(p.ws + p.ml_off);
+    float* po = reinterpret_cast<float*>(p.ws + p.o_off);
+
+    auto correct = [&](uint32_t cc, const float* alpha) -> bool {
+      const int ob = cc & 1;
+      if (!mbar_wait(&o_full[ob], (cc >> 1) & 1u, abrt, status)) return false;
+      tc_fence_after();
+      float ov[NPV];
+      tmem_ld16(lane_addr + 32 + NPV * ob, ov);
+      if constexpr (NPV == 32) tmem_ld16(lane_addr + 32 + NPV * ob + 16, ov + 16);
+      tc_fence_before();
+      mbar_arrive(&o_free[ob]);
+#pragma unroll
+      for (int g = 0; g < GQ; ++g) o[g] = fmaf(o[g], alpha[g], ov[g] + ov[GQ + g]);
+      return true;
+    };
+
+    while (true) {
+      const int stage = c % kNst;
+      if (!mbar_wait(&full[stage], (c / kNst) & 1u, abrt, status)) break;
+      const ChunkMeta mt = meta[stage];
+      if (mt.flags & kEnd) break;
+      if (mt.flags & kFirst) {
+#pragma unroll
+        for (int g = 0; g < GQ; ++g) {
+          m_run[g] = -INFINITY;
+          l_thr[g] = 0.f;
+          o[g] = 0.f;
+        }
+        have_prev = false;
+      }
+      // ---- scores of token r
+      const int sb = c & 1;
+      if (!mbar_wait(&s_full[sb], (c >> 1) & 1u, abrt, status)) break;
+      tc_fence_after();
+      float sv[16];
+      tmem_ld16(lane_addr + 16 * sb, sv);
+      tc_fence_before();
+      mbar_arrive(&s_free[sb]);
+      const bool tok_ok = r < mt.valid;
+      float s2[GQ];
+#pragma unroll
+      for (int g = 0; g < GQ; ++g)
+        s2[g] = (tok_ok && g < G) ? sv[g < 16 ? g : 15] * sl2 : -INFINITY;
+      // ---- chunk max per head across the 128 tokens
+      float* rb = red + (c & 1) * 64;
+#pragma unroll
+      for (int g = 0; g < GQ; ++g) {
+        float mx = s2[g];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
+        if (lane == 0) rb[wq * 16 + g] = mx;
+      }
+      if (!group_sync(grp, gphase, abrt, status)) break;
+      float alpha[GQ];
+      uint32_t col[NPV];   // P^T row r: column g = hi(p_g), column GQ + g = lo(p_g)
+#pragma unroll
+      for (int g = 0; g < GQ; ++g) {
+        const float cm = fmaxf(fmaxf(rb[g], rb[16 + g]), fmaxf(rb[32 + g], rb[48 + g]));
+        const float mn = fmaxf(m_run[g], cm);
+        // heads g >= G never see a finite score; keep them inert (alpha 0, p 0)
+        alpha[g] = (mn == -INFINITY) ? 0.f : exp2f(m_run[g] - mn);
+        const float pr = (mn == -INFINITY) ? 0.f : exp2f(s2[g] - mn);
+        m_run[g] = mn;
+        l_thr[g] = fmaf(l_thr[g], alpha[g], pr);
+        uint16_t hi, lo;
+        split16<T>(pr, hi, lo);
+        col[g] = hi;
+        col[GQ + g] = lo;
+      }
+      uint32_t packed[NPV / 2];
+#pragma unroll
+      for (int w = 0; w < NPV / 2; ++w) packed[w] = col[2 * w] | (col[2 * w + 1] << 16);
+      // ---- store P^T row r: 8 columns (16 B) per core-matrix group
+      uint8_t* pdst = pbuf + (c & 1) * Ly::PBUF + r * 16;
+#pragma unroll
+      for (int ng = 0; ng < NPV / 8; ++ng)
+        *reinterpret_cast<uint4*>(pdst + ng * 2048) =
+            make_uint4(packed[ng * 4 + 0], packed[ng * 4 + 1], packed[ng * 4 + 2],
+                       packed[ng * 4 + 3]);
+      if (!tok_ok) {
+        // rows past the chunk's valid tokens: make V finite (zero) for the MMA
+        uint8_t* vrow = smem + static_cast<size_t>(stage) * kStage + 2 * kHalf + r * 128;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          reinterpret_cast<uint4*>(vrow)[i] = make_uint4(0, 0, 0, 0);
+          reinterpret_cast<uint4*>(vrow + kHalf)[i] = make_uint4(0, 0, 0, 0);
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&p_full[c & 1]);
+      // ---- deferred correction of the previous chunk of this item
+      if (have_prev) {
+        if (!correct(c_prev, a_prev)) break;
+      }
+#pragma unroll
+      for (int g = 0; g < GQ; ++g) a_prev[g] = alpha[g];
+      have_prev = true;
+      c_prev = c;
+
+      if (mt.flags & kLast) {
+        if (!correct(c, a_prev)) break;
+        have_prev = false;
+        // sum of l over the 128 tokens
+#pragma unroll
+        for (int g = 0; g < GQ; ++g) {
+          float lg = l_thr[g];
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) lg += __shfl_xor_sync(kFull, lg, off);
+          if (lane == 0) lred[wq * 16 + g] = lg;
+        }
+        if (!group_sync(grp, gphase, abrt, status)) break;
+        const bool single = (mt.split_raw & kSingleFlag) != 0;
+        const int split = mt.split_raw & ~kSingleFlag;
+#pragma unroll
+        for (int g = 0; g < GQ; ++g) {
+          if (g >= G) break;
+          const float L = lred[g] + lred[16 + g] + lred[32 + g] + lred[48 + g];
+          const size_t row = static_cast<size_t>(mt.seq) * p.num_q_heads + mt.kvh * G + g;
+          if (single) {
+            p.out[row * kD + r] = o[g] / L;
+          } else {
+            const size_t pr_ = row * p.max_splits + split;
+            po[pr_ * kD + r] = o[g];
+            if (r == 0) ml[pr_] = make_float2(m_run[g], L);
+          }
+        }
+      }
+      ++c;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(Ly::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host: tensor maps and launch
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// 2-D map over a [rows, 128] 16-bit matrix, box = 64 columns x box_rows rows,
+// 128-byte swizzle; out-of-range rows read as zero.
+cudaError_t make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows,
+                     bool bf16) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD) * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                  const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <typename T, int NPV>
+cudaError_t launch_t(const DecodeParams& p, int num_ctas, cudaStream_t stream) {
+  using Ly = TcLayout<NPV>;
+  const bool bf16 = std::is_same<T, __nv_bfloat16>::value;
+  CUtensorMap mk, mv, mq;
+  const uint64_t pool_rows =
+      static_cast<uint64_t>(p.num_blocks) * p.num_kv_heads * p.block_size;
+  cudaError_t e = make_map(&mk, p.k_cache, pool_rows, p.block_size, bf16);
+  if (e == cudaSuccess) e = make_map(&mv, p.v_cache, pool_rows, p.block_size, bf16);
+  if (e == cudaSuccess)
+    e = make_map(&mq, p.q, static_cast<uint64_t>(p.num_seqs) * p.num_q_heads, 16, bf16);
+  if (e != cudaSuccess) return e;
+  auto kern = tc_decode_kernel<T, NPV>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(Ly::SMEM));
+  if (e != cudaSuccess) return e;
+  kern<<<num_ctas, kThreads, Ly::SMEM, stream>>>(p, mk, mv, mq);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_supported(int dtype, int head_dim, int group) {
+  return (dtype == 1 || dtype == 2) && head_dim == kD && group >= 4 && group <= 16 &&
+         encode_fn() != nullptr;
+}
+
+cudaError_t tc_num_ctas(int dtype, int group, int* num_ctas) {
+  (void)dtype;
+  (void)group;
+  *num_ctas = num_sms();   // one CTA per SM (shared memory and TMEM sized for it)
+  return cudaSuccess;
+}
+
+cudaError_t launch_decode_tc(const DecodeParams& p, int num_ctas, cudaStream_t stream) {
+  const int group = p.num_q_heads / p.num_kv_heads;
+  if (!tc_supported(p.dtype, p.head_dim, group)) return cudaErrorInvalidValue;
+  if (p.dtype == 2) {
+    return group <= 8 ? launch_t<__nv_bfloat16, 16>(p, num_ctas, stream)
+                      : launch_t<__nv_bfloat16, 32>(p, num_ctas, stream);
+  }
+  return group <= 8 ? launch_t<__half, 16>(p, num_ctas, stream)
+                    : launch_t<__half, 32>(p, num_ctas, stream);
+}
+
 }  // namespace pa

@@ -252,7 +252,7 @@ def test_bad_table_entry_and_length_are_flagged_not_faulted():
     b.block_tables[0, 1] = b.num_blocks + 1000
     ws = ops.decode_workspace(3, 4, 128, 64, 16)
     out = torch.empty(3, 4, 128, device="cuda")
-    ops.pa_decode(out, b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, 64, b.scale, ws)
+    ops.pa_decode(out, b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, 48, b.scale, ws)
     torch.cuda.synchronize()
     assert ops.pa_decode_status(ws) == ops.PA_ERR_INVALID_ARG
     b2 = _custom_batch([40, 80, 40], Hq=4, Hkv=4)
