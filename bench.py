@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--pool-blocks", type=int, default=0,
+                    help="mha only: pool size in blocks (0 = the workload's 16384)")
     return ap.parse_args()
 
 
@@ -80,25 +82,46 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Max of a per-rank time over all ranks (control path only)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int) -> float:
+    """Sum of a per-rank count over all ranks (control path only)."""
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def weak_scaling_value(units_all_ranks: float, ms_max: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest
+    rank's time."""
+    return units_all_ranks / (ms_max * 1e-3)
 
 
 # ---------------------------------------------------------------------------
 # workload
 # ---------------------------------------------------------------------------
 
-def make_batch(name, device, rank, block_size):
+def make_batch(name, device, rank, block_size, pool_blocks=0):
     from paged_kv_cache_339_b200 import workloads as W
     fn = W.FULL[name]
     seed = {"tiny": 1001, "mha": 1002, "gqa": 1003, "prefix_cow": 1004, "long": 1005}[name]
     kw = {"seed": seed + 100 * rank}
     if block_size and name in ("mha", "gqa", "long"):
         kw["block_size"] = block_size
+    if pool_blocks and name == "mha":
+        kw["num_blocks"] = pool_blocks
     return fn(device, **kw)
 
 
@@ -281,10 +304,12 @@ def time_e2e(b, ops, ws, split, path, stream, K, W):
 
 
 def kernel_source_hash():
+    """Hash of the decode kernels' sources (the traffic figure is only reported
+    while it was measured on these exact sources)."""
     h = hashlib.sha256()
-    for f in sorted((ROOT / "paged_kv_cache_339_b200" / "csrc").glob("*")):
-        if f.suffix in (".cu", ".cuh", ".h"):
-            h.update(f.read_bytes())
+    csrc = ROOT / "paged_kv_cache_339_b200" / "csrc"
+    for name in ("pa_common.cuh", "pa_decode_simt.cu", "pa_decode_tc.cu", "pa_plan_reduce.cu"):
+        h.update((csrc / name).read_bytes())
     return h.hexdigest()[:16]
 
 
@@ -353,7 +378,7 @@ def run_ours(args, rank, world, local):
     pa_build.build()
     from paged_kv_cache_339_b200 import ops
     path = {"auto": ops.PA_PATH_AUTO, "simt": ops.PA_PATH_SIMT, "tc": ops.PA_PATH_TCGEN05}[args.path]
-    b = make_batch(args.workload, "cuda", rank, args.block_size)
+    b = make_batch(args.workload, "cuda", rank, args.block_size, args.pool_blocks)
     kv_bytes = b.kv_bytes_logical()
     B, Hq, D = b.q.shape
     ws = ops.decode_workspace(B, Hq, D, b.max_context_len, b.block_size, args.split)
@@ -372,7 +397,9 @@ def run_ours(args, rank, world, local):
     e2e_ms = max_over_ranks(e2e_ms, world)
 
     peak, peak_kind = measured_peak()
-    gbps = kv_bytes * world / (ms * 1e-3) / 1e9
+    kv_bytes_all = sum_over_ranks(kv_bytes, world)
+    seqs_all = sum_over_ranks(B, world)
+    gbps = weak_scaling_value(kv_bytes_all, ms) / 1e9
     dec_gbps = kv_bytes / (dec_ms * 1e-3) / 1e9
     khash = kernel_source_hash()
     res = {
@@ -383,7 +410,7 @@ def run_ours(args, rank, world, local):
         "data": "synthetic (seeded N(0,1) K/V/Q, shuffled block placement)",
         "config": config_of(b, args.workload,
                             f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of KV read per step"),
-        "seq_steps_per_s": round(B * world / (ms * 1e-3), 1),
+        "seq_steps_per_s": round(weak_scaling_value(seqs_all, ms), 1),
         "pct_of_peak": round(100.0 * gbps / world / peak, 2),
         "pct_of_nominal_8tbs": round(100.0 * gbps / world / 8000.0, 2),
         "decode_status": int(status),
@@ -397,7 +424,7 @@ def run_ours(args, rank, world, local):
             "traffic": traffic_from_profile(b.name, khash),
             "kernel_source_hash": khash,
         },
-        "e2e": {"value": round(kv_bytes * world / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+        "e2e": {"value": round(weak_scaling_value(kv_bytes_all, e2e_ms) / 1e9, 1), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h)},
         "clocks": clk.summary(),
