@@ -178,6 +178,34 @@ pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
                     size_t workspace_bytes, pa_stream_t stream);
 
 /*
+ * pa_decode_noalloc - pa_decode for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart to this call. It exists for callers that
+ * cannot obtain a workspace: a process that gives nearly all of HBM to its
+ * KV-cache pool up front has no room left for a second allocation, and code on
+ * a latency-critical path cannot afford cudaMalloc's implicit synchronisation.
+ *
+ * Arguments and result are those of pa_decode without the workspace. The
+ * scratch is a fixed 32 MiB device array inside this library; every GPU that
+ * loads the library holds it until the process exits. Shapes whose
+ * pa_decode_workspace_size(...) exceeds 32 MiB are rejected with
+ * PA_ERR_WORKSPACE_TOO_SMALL before anything is enqueued. The call allocates
+ * nothing.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents;
+ *     each call re-initialises everything it reads, so nothing has to be
+ *     cleared by the caller. Calls that overlap on the GPU (other streams, or
+ *     other threads) race on the array and must not overlap.
+ */
+pa_status pa_decode_noalloc(const pa_kv_cache* cache, float* out, const void* q,
+                            const int32_t* block_tables, int32_t bt_stride,
+                            const int32_t* context_lens, int32_t num_seqs,
+                            int32_t num_q_heads, int32_t max_context_len,
+                            float scale, const pa_decode_options* opts,
+                            pa_stream_t stream);
+
+/*
  * pa_decode_status - read back (synchronously, on `stream`) the device status
  * word the last pa_decode using `workspace` left: PA_OK, or
  * PA_ERR_DEVICE_TIMEOUT if one of its kernels stopped waiting on a barrier

@@ -76,6 +76,11 @@ constexpr int kItemsPerCta = 12;
 
 }  // namespace
 
+void record_cuda_error(cudaError_t e) {
+  std::snprintf(g_cuda_error, sizeof(g_cuda_error), "%s: %s", cudaGetErrorName(e),
+                cudaGetErrorString(e));
+}
+
 int num_sms() {
   static int cached[64] = {};
   int dev = 0;

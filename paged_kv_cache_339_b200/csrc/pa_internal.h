@@ -73,4 +73,7 @@ cudaError_t launch_copy_blocks(void* k_cache, void* v_cache,
 
 int num_sms();
 
+// Store a CUDA error for pa_last_cuda_error() on this thread.
+void record_cuda_error(cudaError_t e);
+
 }  // namespace pa

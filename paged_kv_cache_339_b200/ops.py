@@ -46,7 +46,8 @@ class PagedAttnError(RuntimeError):
 _lib = None
 
 EXPORTS = ("pa_write_kv", "pa_copy_blocks", "pa_decode_workspace_size", "pa_decode",
-           "pa_decode_status", "pa_status_string", "pa_last_cuda_error", "pa_version")
+           "pa_decode_noalloc", "pa_decode_status", "pa_status_string", "pa_last_cuda_error",
+           "pa_version")
 
 
 def _load():
@@ -69,6 +70,9 @@ def _load():
                               ctypes.c_float, ctypes.POINTER(PaDecodeOptions), vp,
                               ctypes.c_size_t, vp]
     lib.pa_decode.restype = ctypes.c_int
+    lib.pa_decode_noalloc.argtypes = [ctypes.POINTER(PaKvCache), vp, vp, vp, i32, vp, i32, i32,
+                                      i32, ctypes.c_float, ctypes.POINTER(PaDecodeOptions), vp]
+    lib.pa_decode_noalloc.restype = ctypes.c_int
     lib.pa_decode_status.argtypes = [vp, vp]
     lib.pa_decode_status.restype = ctypes.c_int
     lib.pa_status_string.argtypes = [ctypes.c_int]
@@ -182,6 +186,29 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_
         int(max_context_len), float(scale), ctypes.byref(opts),
         _dev_tensor(workspace, "workspace", torch.uint8), workspace.numel(), _stream(stream))
     _check("pa_decode", st)
+    return out
+
+
+def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len,
+                      scale, split_tokens=0, path=PA_PATH_AUTO, stream=None) -> torch.Tensor:
+    """pa_decode with the library's fixed 32 MiB device scratch instead of a
+    workspace, for callers that cannot allocate device memory (see
+    include/pa.h). Calls must not overlap on the GPU."""
+    desc = kv_cache_desc(k_cache, v_cache)
+    B, Hq, D = q.shape
+    if out.shape != (B, Hq, D) or out.dtype != torch.float32:
+        raise ValueError("out must be fp32 [num_seqs, num_q_heads, head_dim]")
+    if D != k_cache.shape[3] or block_tables.dim() != 2 or block_tables.shape[0] != B:
+        raise ValueError("shape mismatch between q, caches and block_tables")
+    if context_lens.shape != (B,):
+        raise ValueError("context_lens must be [num_seqs]")
+    opts = PaDecodeOptions(int(split_tokens), int(path))
+    st = _load().pa_decode_noalloc(
+        ctypes.byref(desc), _dev_tensor(out, "out", torch.float32),
+        _dev_tensor(q, "q", k_cache.dtype), _dev_tensor(block_tables, "block_tables", torch.int32),
+        int(block_tables.shape[1]), _dev_tensor(context_lens, "context_lens", torch.int32), B, Hq,
+        int(max_context_len), float(scale), ctypes.byref(opts), _stream(stream))
+    _check("pa_decode_noalloc", st)
     return out
 
 
