@@ -5,7 +5,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/pa.h"
+#include "pa.h"
 #include "pa_internal.h"
 
 namespace pa {
@@ -250,6 +250,7 @@ pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
   mp.max_splits = lay.max_splits;
   e = launch_merge(mp, s);
   if (e != cudaSuccess) return cuda_fail(e);
+
   return PA_OK;
 }
 

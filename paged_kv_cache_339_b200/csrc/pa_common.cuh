@@ -202,12 +202,21 @@ __device__ __forceinline__ void unpack16(const uint4& v, float* f) {
 // the KV-head index is folded into the claimed item number.
 struct __align__(16) WorkPair {
   int32_t seq;
-  int32_t split;
+  int32_t split_n;  // split index (low 16 bits) | number of splits of the sequence << 16
   int32_t t_begin;  // first token of the range
-  int32_t t_end;    // one past the last token; the sequence has one split
-                    // iff split == 0 and t_end == context length (flag below)
+  int32_t t_end;    // one past the last token
 };
-constexpr int32_t kSingleFlag = 1 << 30;  // set in `split` when the item is the
-                                          // whole sequence (output written directly)
+__device__ __forceinline__ int item_split(int32_t split_n) { return split_n & 0xffff; }
+__device__ __forceinline__ int item_nsplit(int32_t split_n) { return split_n >> 16; }
+
+// Programmatic dependent launch: let the next kernel in the stream start its
+// prologue now / wait until the previous kernel has completed and its writes
+// are visible. Both are no-ops for kernels launched without the attribute.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
 
 }  // namespace pa

@@ -128,6 +128,8 @@ __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
     fence_barrier_init();
   }
   __syncthreads();
+  pdl_wait();   // the plan (and the KV write before it) are complete from here on
+  pdl_launch_dependents();   // the merge kernel may get resident; it waits for us
 
   const int num_items = hdr->num_items;
   const int Hkv = p.num_kv_heads, BS = p.block_size;
@@ -165,7 +167,7 @@ __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
           ChunkMeta m;
           m.seq = wp.seq;
           m.kvh = kvh;
-          m.split_raw = wp.split;
+          m.split_raw = wp.split_n;
           m.t0 = cs;
           m.valid = valid;
           m.flags = (cs == wp.t_begin ? kFirst : 0) | (cs + CHUNK >= wp.t_end ? kLast : 0);
@@ -340,8 +342,9 @@ __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
         }
         if (!group_sync(&gbar[0], gphase, abrt, status)) break;
         const int tid = threadIdx.x - 32;
-        const bool single = (mt.split_raw & kSingleFlag) != 0;
-        const int split = mt.split_raw & ~kSingleFlag;
+        const int nsp = item_nsplit(mt.split_raw);
+        const bool single = nsp == 1;
+        const int split = item_split(mt.split_raw);
         float2* ml = reinterpret_cast<float2*>(p.ws + p.ml_off);
         float* po = reinterpret_cast<float*>(p.ws + p.o_off);
         for (int idx = tid; idx < G * D; idx += Tr::NCW * 32) {
@@ -380,8 +383,8 @@ cudaError_t launch_t(const DecodeParams& p, int num_ctas, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(Tr::SMEM));
   if (e != cudaSuccess) return e;
-  kern<<<num_ctas, Tr::NTHREADS, Tr::SMEM, stream>>>(p);
-  return cudaGetLastError();
+  e = launch_pdl(kern, dim3(num_ctas), dim3(Tr::NTHREADS), Tr::SMEM, stream, p);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <typename T, int D, int GPW>

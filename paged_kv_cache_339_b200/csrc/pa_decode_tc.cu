@@ -219,6 +219,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  pdl_wait();   // the plan (and the KV write before it) are complete from here on
+  pdl_launch_dependents();   // the merge kernel may get resident; it waits for us
 
   const int num_items = hdr->num_items;
   const int Hkv = p.num_kv_heads, BS = p.block_size;
@@ -264,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ChunkMeta m;
           m.seq = wp.seq;
           m.kvh = kvh;
-          m.split_raw = wp.split;
+          m.split_raw = wp.split_n;
           m.t0 = cs;
           m.valid = valid;
           m.flags = (cs == wp.t_begin ? kFirst : 0) | (cs + kChunk >= wp.t_end ? kLast : 0);
@@ -487,8 +489,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) lred[wq * 16 + g] = lg;
         }
         if (!group_sync(grp, gphase, abrt, status)) break;
-        const bool single = (mt.split_raw & kSingleFlag) != 0;
-        const int split = mt.split_raw & ~kSingleFlag;
+        const int nsp = item_nsplit(mt.split_raw);
+        const bool single = nsp == 1;
+        const int split = item_split(mt.split_raw);
 #pragma unroll
         for (int g = 0; g < GQ; ++g) {
           if (g >= G) break;
@@ -566,8 +569,8 @@ cudaError_t launch_t(const DecodeParams& p, int num_ctas, cudaStream_t stream) {
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(Ly::SMEM));
   if (e != cudaSuccess) return e;
-  kern<<<num_ctas, kThreads, Ly::SMEM, stream>>>(p, mk, mv, mq);
-  return cudaGetLastError();
+  e = launch_pdl(kern, dim3(num_ctas), dim3(kThreads), Ly::SMEM, stream, p, mk, mv, mq);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace

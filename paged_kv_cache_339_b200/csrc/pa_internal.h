@@ -23,13 +23,6 @@ struct PlanParams {
   int32_t items_per_cta;  // target work items per CTA (automatic split)
 };
 
-struct MergeParams {
-  float* out;
-  const uint8_t* ws;
-  size_t nsplit_off, ml_off, o_off;
-  int32_t num_seqs, num_q_heads, num_kv_heads, head_dim, max_splits;
-};
-
 // Everything a decode main kernel needs; filled by the C-ABI shim.
 struct DecodeParams {
   const void* k_cache;
@@ -45,6 +38,15 @@ struct DecodeParams {
   int32_t dtype;     // pa_dtype
 };
 
+struct MergeParams {
+  float* out;
+  const uint8_t* ws;
+  size_t nsplit_off, ml_off, o_off;
+  int32_t num_seqs, num_q_heads, num_kv_heads, head_dim, max_splits;
+};
+
+// Both launch with programmatic stream serialisation (PDL): the kernel may be
+// scheduled while its predecessor in the stream finishes.
 cudaError_t launch_plan(const PlanParams& p, cudaStream_t stream);
 cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream);
 
@@ -72,6 +74,25 @@ cudaError_t launch_copy_blocks(void* k_cache, void* v_cache,
                                cudaStream_t stream);
 
 int num_sms();
+
+// Launch with programmatic stream serialisation: the kernel may be scheduled
+// while its predecessor in the stream is still running; it must execute
+// griddepcontrol.wait (pdl_wait) before touching anything that kernel writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
 
 // Store a CUDA error for pa_last_cuda_error() on this thread.
 void record_cuda_error(cudaError_t e);

@@ -9,7 +9,7 @@
 // then obtain a workspace for pa_decode.
 #include <mutex>
 
-#include "../../include/pa.h"
+#include "pa.h"
 #include "pa_internal.h"
 
 namespace pa {

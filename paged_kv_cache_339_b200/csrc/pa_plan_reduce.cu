@@ -11,6 +11,11 @@
 //   M = max_p m_p,  L = sum_p l_p 2^(m_p - M),  o = sum_p a_p 2^(m_p - M) / L.
 // This regrouping is exact algebra on the softmax sums; the pages do not
 // discuss splitting a context.
+//
+// Launched with programmatic stream serialisation: it may start while the KV
+// write before it is still running (it reads only the lengths), and waits for
+// that kernel before it exits, so the decode kernel that waits on the plan
+// also sees the new tokens.
 #include "pa_common.cuh"
 #include "pa_internal.h"
 
@@ -18,7 +23,7 @@ namespace pa {
 
 namespace {
 
-constexpr int kPlanThreads = 1024;
+constexpr int kPlanMaxThreads = 1024;
 
 __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
 #pragma unroll
@@ -29,15 +34,15 @@ __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
   return v;
 }
 
-// Exclusive scan of one int per thread over the CTA; returns the prefix and
-// writes the total to *total (all threads).
+// Exclusive scan of one int per thread over the CTA; the total goes to *total.
 __device__ int block_excl_scan(int v, int* scratch, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
   int inc = warp_incl_scan(v, lane);
   if (lane == 31) scratch[warp] = inc;
   __syncthreads();
   if (warp == 0) {
-    int w = lane < (kPlanThreads / 32) ? scratch[lane] : 0;
+    int w = lane < nwarps ? scratch[lane] : 0;
     int wi = warp_incl_scan(w, lane);
     scratch[32 + lane] = wi - w;
     if (lane == 31) scratch[64] = wi;
@@ -49,8 +54,8 @@ __device__ int block_excl_scan(int v, int* scratch, int* total) {
   return res;
 }
 
-__global__ void __launch_bounds__(kPlanThreads, 1)
-    plan_kernel(PlanParams p) {
+__global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) {
+  pdl_launch_dependents();
   __shared__ long long s_sum[32];
   __shared__ int s_max[32];
   __shared__ int s_bad[32];
@@ -62,12 +67,13 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
   WorkPair* pairs = reinterpret_cast<WorkPair*>(p.ws + p.pairs_off);
   int32_t* nsplit = reinterpret_cast<int32_t*>(p.ws + p.nsplit_off);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nthreads = blockDim.x, nwarps = nthreads >> 5;
   const int64_t cap = static_cast<int64_t>(p.bt_stride) * p.block_size;
 
   // 1. validate lengths, total and maximum
   long long tot = 0;
   int mx = 0, bad = 0;
-  for (int i = tid; i < p.num_seqs; i += kPlanThreads) {
+  for (int i = tid; i < p.num_seqs; i += nthreads) {
     const int L = p.context_lens[i];
     if (L < 0 || L > p.max_context_len || L > cap) {
       bad = 1;
@@ -91,7 +97,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
   if (tid == 0) {
     long long t = 0;
     int m = 0, b = 0;
-    for (int w = 0; w < kPlanThreads / 32; ++w) {
+    for (int w = 0; w < nwarps; ++w) {
       t += s_sum[w];
       m = max(m, s_max[w]);
       b |= s_bad[w];
@@ -117,7 +123,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
   const int maxn = min(s_maxn, p.max_splits);
 
   // 2. splits per sequence; sequences with nothing to attend to get zero rows
-  for (int i = tid; i < p.num_seqs; i += kPlanThreads) {
+  for (int i = tid; i < p.num_seqs; i += nthreads) {
     const int L = p.context_lens[i];
     const bool ok = !(L < 0 || L > p.max_context_len || L > cap);
     const int n = (ok && L > 0) ? (L + S - 1) / S : 0;
@@ -134,7 +140,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
   // 3. split-major pair list
   int base = 0;
   for (int s = 0; s < maxn; ++s) {
-    for (int i0 = 0; i0 < p.num_seqs; i0 += kPlanThreads) {
+    for (int i0 = 0; i0 < p.num_seqs; i0 += nthreads) {
       const int i = i0 + tid;
       int n = 0, L = 0;
       if (i < p.num_seqs) {
@@ -147,7 +153,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
       if (f) {
         WorkPair w;
         w.seq = i;
-        w.split = s | (n == 1 ? kSingleFlag : 0);
+        w.split_n = s | (n << 16);
         w.t_begin = s * S;
         w.t_end = min(L, (s + 1) * S);
         pairs[base + rank] = w;
@@ -160,12 +166,14 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
     hdr->num_items = base * p.num_kv_heads;
     hdr->work_counter = 0;
   }
+  // complete only after the kernel before this one (the KV write) has
+  pdl_wait();
 }
 
 constexpr int kMergeThreads = 256;
 
-__global__ void __launch_bounds__(kMergeThreads)
-    merge_kernel(MergeParams p) {
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(MergeParams p) {
+  pdl_wait();   // every partial of the decode kernel is written and visible
   extern __shared__ float s_w[];  // [G][max_splits] normalised weights
   const int seq = blockIdx.x / p.num_kv_heads;
   const int kvh = blockIdx.x % p.num_kv_heads;
@@ -199,6 +207,7 @@ __global__ void __launch_bounds__(kMergeThreads)
     const float* src = po + row * p.max_splits * D + d;
     const float* w = s_w + g * p.max_splits;
     float acc = 0.f;
+#pragma unroll 4
     for (int s = 0; s < n; ++s) acc = fmaf(w[s], src[static_cast<size_t>(s) * D], acc);
     p.out[row * D + d] = acc;
   }
@@ -206,23 +215,33 @@ __global__ void __launch_bounds__(kMergeThreads)
 
 }  // namespace
 
-cudaError_t launch_plan(const PlanParams& p, cudaStream_t stream) {
-  plan_kernel<<<1, kPlanThreads, 0, stream>>>(p);
-  return cudaGetLastError();
-}
-
 cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream) {
   if (p.max_splits <= 1 || p.num_seqs == 0) return cudaSuccess;
   const int G = p.num_q_heads / p.num_kv_heads;
   const size_t smem = static_cast<size_t>(G) * p.max_splits * sizeof(float);
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(
-        merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-        static_cast<int>(smem));
+    cudaError_t e = cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  merge_kernel<<<p.num_seqs * p.num_kv_heads, kMergeThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(merge_kernel, dim3(p.num_seqs * p.num_kv_heads), dim3(kMergeThreads), smem,
+                    stream, p);
+}
+
+cudaError_t launch_plan(const PlanParams& p, cudaStream_t stream) {
+  int threads = (p.num_seqs + 31) / 32 * 32;
+  threads = threads < 64 ? 64 : (threads > kPlanMaxThreads ? kPlanMaxThreads : threads);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, plan_kernel, p);
 }
 
 }  // namespace pa

@@ -28,6 +28,7 @@ __global__ void __launch_bounds__(kCopyThreads)
                     const int64_t* __restrict__ slots, int32_t num_tokens,
                     int32_t num_kv_heads, int32_t block_size,
                     int32_t row_vecs, int64_t num_slots) {
+  pdl_launch_dependents();   // the decode plan may start; it waits for us before it ends
   const int64_t per_token = static_cast<int64_t>(num_kv_heads) * row_vecs;
   const int64_t total = per_token * num_tokens;
   for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
@@ -50,6 +51,7 @@ __global__ void __launch_bounds__(kCopyThreads)
     copy_blocks_kernel(uint4* __restrict__ kc, uint4* __restrict__ vc,
                        const int64_t* __restrict__ pairs, int32_t num_pairs,
                        int64_t block_vecs, int32_t num_blocks) {
+  pdl_launch_dependents();
   const int64_t total = block_vecs * num_pairs;
   for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
        idx < total; idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
