@@ -209,7 +209,8 @@ pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
   pp.split_tokens = split;
   pp.min_split = split > 0 ? split : auto_min_split(max_context_len);
   pp.max_splits = lay.max_splits;
-  pp.num_ctas = ctas;
+  // the tensor-core kernel runs two independent item streams per CTA
+  pp.num_ctas = use_tc ? 2 * ctas : ctas;
   pp.items_per_cta = kItemsPerCta;
   e = launch_plan(pp, s);
   if (e != cudaSuccess) return cuda_fail(e);

@@ -58,6 +58,9 @@ struct SimtTraits {
   static constexpr size_t OFF_ABORT = OFF_CMB + NCW * CMB * 4;
   static constexpr size_t SMEM = OFF_ABORT + 16;
   static_assert(NV >= 1, "row must be at least 128 bytes");
+  static_assert(OFF_BAR % 16 == 0 && OFF_META % 16 == 0 && OFF_PSCR % 16 == 0 &&
+                    OFF_CMB % 16 == 0 && OFF_ABORT % 16 == 0,
+                "16-byte aligned shared regions");
   static_assert(EPL == 2 || EPL == 4, "head_dim 64 or 128");
 };
 

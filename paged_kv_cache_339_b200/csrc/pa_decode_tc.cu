@@ -12,18 +12,26 @@
 // terms, p = hi + lo (columns [0, NPV/2) and [NPV/2, NPV) of P^T), so the
 // product keeps ~16 significant bits of p at no extra tensor-core passes.
 //
-// Persistent, warp-specialised CTA (one per SM, ~215 KB shared memory):
-//   warp 0     producer: claims (sequence, split, KV head) items, follows the
-//              block table, and loads each page's K and V tile (two 64-column
-//              halves each) plus the Q tile with 2-D TMA (128-byte swizzle)
-//              into a 3-stage ring; completion by mbarrier transaction count.
-//   warp 1     allocates TMEM and issues the MMAs (one elected lane); S^T and
-//              O^T accumulators live in TMEM, double-buffered, so the scores
-//              of chunk c+1 are computed while chunk c's softmax runs.
-//   warps 2-5  softmax and correction: thread r owns token r of a chunk for
-//              the softmax (tcgen05.ld of its S^T row), and output column d = r
-//              for the correction O += alpha * O_chunk; partial results of
-//              split items go to the workspace for the merge kernel.
+// Persistent, warp-specialised CTA (one per SM, ~220 KB shared memory) that
+// runs two independent item streams, so one stream's serial steps (the MMA
+// round trips, the end-of-item reduction and stores) overlap the other's:
+//   warp 0      producer: claims (sequence, split, KV head) items for the two
+//               streams and emits their 128-token chunks alternately (chunk
+//               position c belongs to stream c & 1); for each chunk it follows
+//               the block table and loads each page's K and V tile (two
+//               64-column halves each) plus the Q tile with 2-D TMA (128-byte
+//               swizzle) into a 3-stage ring; completion by mbarrier
+//               transaction count. When a stream runs out of items its
+//               positions carry END, then empty "bubble" slots, and finally a
+//               STOP for each stream.
+//   warps 1, 2  MMA issuers (one elected lane each), one per stream: S^T into
+//               the stream's TMEM columns, then O^T once its softmax group has
+//               published P; warp 1 also allocates and frees TMEM.
+//   warps 3-6,  softmax and correction groups, one per stream: thread r owns
+//   7-10        token r of a chunk for the softmax (tcgen05.ld of its S^T row)
+//               and output column d = r for the correction O = alpha O + O_c;
+//               partial results of split items go to the workspace for the
+//               merge kernel.
 // No load uses cluster multicast; every wait is bounded (see pa_common.cuh).
 #include <cudaTypedefs.h>
 
@@ -38,35 +46,41 @@ namespace pa {
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
-constexpr int kFirst = 1, kLast = 2, kEnd = 4;
+constexpr int kFirst = 1, kLast = 2, kEnd = 4, kBubble = 8, kStop = 16;
 constexpr int kChunk = 128;   // tokens per stage (= MMA M)
 constexpr int kD = 128;       // head_dim
 constexpr int kNst = 3;       // pipeline stages
 constexpr int kHalf = kChunk * 128;           // one 64-column half: 128 rows x 128 B
 constexpr int kQHalf = 16 * 128;              // Q half: 16 rows x 128 B
 constexpr int kStage = 4 * kHalf + 2 * kQHalf;  // K (2 halves), V (2 halves), Q (2 halves)
-constexpr int kThreads = 192;
+constexpr int kThreads = 352;  // producer, 2 MMA issuers, 2 softmax groups of 4 warps
 
 struct __align__(16) ChunkMeta {
   int32_t seq, kvh, split_raw, t0, valid, flags, pad0, pad1;
 };
 
-template <int NPV>
+template <int GT>
 struct TcLayout {
-  static constexpr int GQ = NPV / 2;                 // max query heads
-  static constexpr int PBUF = (NPV / 8) * 2048;      // P^T buffer bytes
+  static constexpr int NPV = GT * 2 < 16 ? 16 : GT * 2;  // P^T columns: hi, lo (M=128 needs N%16==0)
+  static constexpr int PBUF = (NPV / 8) * 2048;      // P^T buffer bytes (one per group)
   static constexpr size_t OFF_P = static_cast<size_t>(kNst) * kStage;
   static constexpr size_t OFF_BAR = OFF_P + 2 * PBUF;
-  // barriers: full[3], empty[3], s_full[2], s_free[2], p_full[2], o_full[2],
-  // o_free[2], grp, drain
-  static constexpr int NBAR = 2 * kNst + 10 + 2;
-  static constexpr size_t OFF_META = OFF_BAR + NBAR * 8;
-  static constexpr size_t OFF_RED = OFF_META + kNst * sizeof(ChunkMeta);
-  static constexpr size_t OFF_LRED = OFF_RED + 2 * 4 * 16 * 4;
-  static constexpr size_t OFF_MISC = OFF_LRED + 4 * 16 * 4;
+  // barriers: full[3][2], empty[3]; per group: s_full, s_free, p_full,
+  // o_full, o_free, group barrier, MMA drain
+  static constexpr int NBAR = 3 * kNst + 14;
+  static constexpr size_t OFF_META = (OFF_BAR + NBAR * 8 + 15) / 16 * 16;  // 16-B vector stores
+  static constexpr size_t OFF_RED = (OFF_META + kNst * sizeof(ChunkMeta) + 15) / 16 * 16;
+  static constexpr size_t OFF_LRED = OFF_RED + 2 * 2 * 4 * 16 * 4;
+  static constexpr size_t OFF_MISC = OFF_LRED + 2 * 4 * 16 * 4;
   static constexpr size_t SMEM_USED = OFF_MISC + 16;
   static constexpr size_t SMEM = SMEM_USED + 1024;   // slack to align the base to 1 KB
   static constexpr uint32_t TMEM_COLS = (32 + 2 * NPV) <= 64 ? 64 : 128;
+  static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(kStage % 1024 == 0 && OFF_P % 1024 == 0, "swizzled tiles need 1 KB alignment");
+  static_assert(OFF_BAR % 8 == 0, "mbarriers need 8-byte alignment");
+  static_assert(OFF_META % 16 == 0 && OFF_RED % 16 == 0 && OFF_LRED % 16 == 0 &&
+                    OFF_MISC % 16 == 0,
+                "16-byte aligned shared regions");
 };
 
 // ---------------------------------------------------------------------------
@@ -159,31 +173,34 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-template <typename T, int NPV>
+template <typename T, int GT>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v,
                      const __grid_constant__ CUtensorMap tm_q) {
-  using Ly = TcLayout<NPV>;
-  constexpr int GQ = Ly::GQ;
+  using Ly = TcLayout<GT>;
+  constexpr int NPV = Ly::NPV;
   extern __shared__ uint8_t smem_raw[];
   // 1 KB alignment for the 128-byte-swizzled tiles
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* pbuf = smem + Ly::OFF_P;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Ly::OFF_BAR);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + kNst;
-  uint64_t* s_full = bars + 2 * kNst;
+  // full[2 * stage + group]: one barrier per (stage, stream) so a stream's
+  // consumers see every phase of the barriers they wait on (the two streams
+  // alternate over an odd number of stages)
+  uint64_t* full = bars;                 // [kNst][2]
+  uint64_t* empty = bars + 2 * kNst;     // [kNst]
+  uint64_t* s_full = bars + 3 * kNst;    // [2] per group
   uint64_t* s_free = s_full + 2;
   uint64_t* p_full = s_free + 2;
   uint64_t* o_full = p_full + 2;
   uint64_t* o_free = o_full + 2;
-  uint64_t* grp = o_free + 2;
-  uint64_t* drain = grp + 1;
+  uint64_t* grp = o_free + 2;            // [2] group barriers
+  uint64_t* drain = grp + 2;             // [2] MMA drain
   ChunkMeta* meta = reinterpret_cast<ChunkMeta*>(smem + Ly::OFF_META);
-  float* red = reinterpret_cast<float*>(smem + Ly::OFF_RED);    // [2][4][16]
-  float* lred = reinterpret_cast<float*>(smem + Ly::OFF_LRED);  // [4][16]
+  float* red = reinterpret_cast<float*>(smem + Ly::OFF_RED);    // [2 grp][2][4][16]
+  float* lred = reinterpret_cast<float*>(smem + Ly::OFF_LRED);  // [2 grp][4][16]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Ly::OFF_MISC);
   volatile int* abrt = reinterpret_cast<volatile int*>(smem + Ly::OFF_MISC + 4);
 
@@ -193,7 +210,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNst; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[2 * s], 1);
+      mbar_init(&full[2 * s + 1], 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -202,9 +220,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&p_full[b], 128);
       mbar_init(&o_full[b], 1);
       mbar_init(&o_free[b], 128);
+      mbar_init(&grp[b], 128);
+      mbar_init(&drain[b], 1);
     }
-    mbar_init(grp, 128);
-    mbar_init(drain, 1);
     *abrt = 0;
     fence_barrier_init();
   }
@@ -228,213 +246,239 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // Two item streams; chunk position c belongs to stream (group) c & 1.
     if (lane == 0) {
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
       prefetch_tmap(&tm_q);
     }
     const WorkPair* pairs = reinterpret_cast<const WorkPair*>(p.ws + p.pairs_off);
+    int kraw0 = 0, kraw1 = 0;
+    if (lane == 0) {
+      kraw0 = atomicAdd(&hdr->work_counter, 1);
+      kraw1 = atomicAdd(&hdr->work_counter, 1);
+    }
+    // per-stream state (warp-uniform); two named copies so every access is a
+    // register select, not an indexed local array
+    struct Stream {
+      int seq, kvh, split_n, tb, te, cs;
+      bool ended;
+    };
+    Stream st0 = {0, 0, 0, 0, 0, 0, false}, st1 = st0;
+    int stops = 0;
     uint32_t c = 0;
     bool ok = true;
-    int kraw = 0;
-    if (lane == 0) kraw = atomicAdd(&hdr->work_counter, 1);
-    int k = __shfl_sync(kFull, kraw, 0);
-    while (k < num_items) {
-      const int pi = k / Hkv, kvh = k - pi * Hkv;
-      const WorkPair wp = pairs[pi];
-      if (lane == 0) kraw = atomicAdd(&hdr->work_counter, 1);
-      const int32_t* bt_row = p.block_tables + static_cast<size_t>(wp.seq) * p.bt_stride;
-      const int q_row = wp.seq * p.num_q_heads + kvh * G;
-      for (int cs = wp.t_begin; cs < wp.t_end; cs += kChunk) {
-        const int valid = min(kChunk, wp.t_end - cs);
-        const int npg = (valid + BS - 1) / BS;
-        int blk = 0;
+    while (true) {
+      const int t = c & 1;
+      Stream cur = t ? st1 : st0;
+      const bool other_ended = t ? st0.ended : st1.ended;
+      int kind = 0;   // 0 data, 1 end, 2 bubble, 3 stop
+      if (!cur.ended && cur.cs >= cur.te) {
+        const int k = __shfl_sync(kFull, t == 0 ? kraw0 : kraw1, 0);
+        if (k < num_items) {
+          const int pi = k / Hkv;
+          const WorkPair wp = pairs[pi];
+          if (lane == 0) {
+            if (t == 0) kraw0 = atomicAdd(&hdr->work_counter, 1);   // next claim in flight
+            else kraw1 = atomicAdd(&hdr->work_counter, 1);
+          }
+          cur.seq = wp.seq;
+          cur.kvh = k - pi * Hkv;
+          cur.split_n = wp.split_n;
+          cur.tb = wp.t_begin;
+          cur.te = wp.t_end;
+          cur.cs = wp.t_begin;
+        } else {
+          cur.ended = true;
+          kind = 1;
+        }
+      } else if (cur.ended) {
+        kind = other_ended ? 3 : 2;
+      }
+      int valid = 0, npg = 0, blk = 0;
+      if (kind == 0) {
+        valid = min(kChunk, cur.te - cur.cs);
+        npg = (valid + BS - 1) / BS;
         if (lane < npg) {
-          blk = bt_row[cs / BS + lane];
+          blk = p.block_tables[static_cast<size_t>(cur.seq) * p.bt_stride + cur.cs / BS + lane];
           if (blk < 0 || blk >= p.num_blocks) {
             atomicCAS(status, 0, 1 /* PA_ERR_INVALID_ARG */);
             blk = 0;
           }
         }
-        const int stage = c % kNst;
-        if (!mbar_wait(&empty[stage], ((c / kNst) & 1u) ^ 1u, abrt, status)) {
-          ok = false;
-          break;
-        }
-        uint8_t* st = smem + static_cast<size_t>(stage) * kStage;
+      }
+      const int stage = c % kNst;
+      if (!mbar_wait(&empty[stage], ((c / kNst) & 1u) ^ 1u, abrt, status)) {
+        ok = false;
+        break;
+      }
+      uint8_t* st = smem + static_cast<size_t>(stage) * kStage;
+      uint64_t* fb = &full[2 * stage + t];
+      if (kind == 0) {
         if (lane == 0) {
           ChunkMeta m;
-          m.seq = wp.seq;
-          m.kvh = kvh;
-          m.split_raw = wp.split_n;
-          m.t0 = cs;
+          m.seq = cur.seq;
+          m.kvh = cur.kvh;
+          m.split_raw = cur.split_n;
+          m.t0 = cur.cs;
           m.valid = valid;
-          m.flags = (cs == wp.t_begin ? kFirst : 0) | (cs + kChunk >= wp.t_end ? kLast : 0);
+          m.flags = (cur.cs == cur.tb ? kFirst : 0) | (cur.cs + kChunk >= cur.te ? kLast : 0);
           m.pad0 = m.pad1 = 0;
           meta[stage] = m;
-          mbar_arrive_expect_tx(&full[stage],
-                                static_cast<uint32_t>(npg * BS * 512 + 2 * kQHalf));
-          tma_load_2d(st + 4 * kHalf, &tm_q, 0, q_row, &full[stage]);
-          tma_load_2d(st + 4 * kHalf + kQHalf, &tm_q, 64, q_row, &full[stage]);
+          mbar_arrive_expect_tx(fb, static_cast<uint32_t>(npg * BS * 512 + 2 * kQHalf));
+          const int q_row = cur.seq * p.num_q_heads + cur.kvh * G;
+          tma_load_2d(st + 4 * kHalf, &tm_q, 0, q_row, fb);
+          tma_load_2d(st + 4 * kHalf + kQHalf, &tm_q, 64, q_row, fb);
         }
         __syncwarp();
         if (lane < npg) {
-          const int row = (blk * Hkv + kvh) * BS;
+          const int row = (blk * Hkv + cur.kvh) * BS;
           const int off = lane * BS * 128;
-          tma_load_2d(st + off, &tm_k, 0, row, &full[stage]);
-          tma_load_2d(st + kHalf + off, &tm_k, 64, row, &full[stage]);
-          tma_load_2d(st + 2 * kHalf + off, &tm_v, 0, row, &full[stage]);
-          tma_load_2d(st + 3 * kHalf + off, &tm_v, 64, row, &full[stage]);
+          tma_load_2d(st + off, &tm_k, 0, row, fb);
+          tma_load_2d(st + kHalf + off, &tm_k, 64, row, fb);
+          tma_load_2d(st + 2 * kHalf + off, &tm_v, 0, row, fb);
+          tma_load_2d(st + 3 * kHalf + off, &tm_v, 64, row, fb);
         }
-        ++c;
-      }
-      if (!ok) break;
-      k = __shfl_sync(kFull, kraw, 0);
-    }
-    if (ok) {
-      const int stage = c % kNst;
-      if (mbar_wait(&empty[stage], ((c / kNst) & 1u) ^ 1u, abrt, status)) {
-        if (lane == 0) {
-          meta[stage].flags = kEnd;
-          mbar_arrive(&full[stage]);
-        }
+        cur.cs += kChunk;
       } else {
-        ok = false;
+        if (lane == 0) {
+          meta[stage].flags = kind == 1 ? kEnd : (kind == 2 ? kBubble : kStop);
+          mbar_arrive(fb);
+        }
+        __syncwarp();
       }
+      if (t) st1 = cur;
+      else st0 = cur;
+      ++c;
+      if (kind == 3 && ++stops == 2) break;
     }
     if (!ok && lane == 0) {
+      // copies may still be landing in the last kNst stages: let them finish
       for (uint32_t cc = c > kNst ? c - kNst : 0; cc < c; ++cc)
-        drain_wait(&full[cc % kNst], (cc / kNst) & 1u);
+        drain_wait(&full[2 * (cc % kNst) + (cc & 1)], (cc / (2 * kNst)) & 1u);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------ MMA issuers
+    const int t = warp - 1;   // group served
     if (lane == 0) {
       const uint32_t fmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
       const uint32_t idesc_s = instr_desc(fmt, false, false, 128, 16);
       const uint32_t idesc_pv = instr_desc(fmt, true, true, 128, NPV);
       const uint32_t sbase = smem_u32(smem);
-      const uint32_t pbase = smem_u32(pbuf);
-
-      auto issue_s = [&](uint32_t cc) {
-        const uint32_t st = sbase + (cc % kNst) * kStage;
+      const uint32_t pb = smem_u32(pbuf) + t * Ly::PBUF;
+      const uint32_t s_tm = tmem + 16 * t;
+      const uint32_t o_tm = tmem + 32 + NPV * t;
+      uint32_t n = 0;   // data chunks of this group so far
+      for (uint32_t c = t;; c += 2) {
+        const int stage = c % kNst;
+        if (!mbar_wait(&full[2 * stage + t], (c / (2 * kNst)) & 1u, abrt, status)) break;
+        const ChunkMeta mt = meta[stage];
+        if (mt.flags & kStop) break;
+        const uint32_t par = n & 1u;
+        if (mt.flags & kEnd) {
+          // release only after the softmax group has seen END (it acknowledges
+          // on p_full); a slot refilled earlier could complete the next phase of
+          // full[] before the group observed this one
+          if (!mbar_wait(&p_full[t], par, abrt, status)) break;
+          mbar_arrive(&empty[stage]);
+          continue;
+        }
+        if (mt.flags & kBubble) {   // only this warp looks at bubbles
+          mbar_arrive(&empty[stage]);
+          continue;
+        }
+        // S^T = K . Q^T
+        if (!mbar_wait(&s_free[t], par ^ 1u, abrt, status)) break;
+        tc_fence_after();
+        const uint32_t stg = sbase + stage * kStage;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t half = kk >> 2, koff = (kk & 3) * 32;
-          const uint64_t a = smem_desc(st + half * kHalf + koff, 16, 1024, kSw128);
-          const uint64_t b = smem_desc(st + 4 * kHalf + half * kQHalf + koff, 16, 1024, kSw128);
-          mma_f16(tmem + 16 * (cc & 1), a, b, idesc_s, kk > 0 ? 1u : 0u);
+          const uint64_t a = smem_desc(stg + half * kHalf + koff, 16, 1024, kSw128);
+          const uint64_t b = smem_desc(stg + 4 * kHalf + half * kQHalf + koff, 16, 1024, kSw128);
+          mma_f16(s_tm, a, b, idesc_s, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&s_full[cc & 1]);
-      };
-      auto issue_pv = [&](uint32_t cc, int valid) {
-        const uint32_t st = sbase + (cc % kNst) * kStage;
-        const uint32_t pb = pbase + (cc & 1) * Ly::PBUF;
-        const int nks = (valid + 15) >> 4;
+        mma_commit(&s_full[t]);
+        // O^T = V^T . P^T once the softmax group has written P
+        if (!mbar_wait(&p_full[t], par, abrt, status)) break;
+        if (!mbar_wait(&o_free[t], par ^ 1u, abrt, status)) break;
+        tc_fence_after();
+        const int nks = (mt.valid + 15) >> 4;
         for (int ks = 0; ks < nks; ++ks) {
-          const uint64_t a = smem_desc(st + 2 * kHalf + ks * 2048, kHalf, 1024, kSw128);
+          const uint64_t a = smem_desc(stg + 2 * kHalf + ks * 2048, kHalf, 1024, kSw128);
           const uint64_t b = smem_desc(pb + ks * 256, 128, 2048, kSwNone);
-          mma_f16(tmem + 32 + NPV * (cc & 1), a, b, idesc_pv, ks > 0 ? 1u : 0u);
+          mma_f16(o_tm, a, b, idesc_pv, ks > 0 ? 1u : 0u);
         }
-        mma_commit(&o_full[cc & 1]);
-        mma_commit(&empty[cc % kNst]);
-      };
-
-      uint32_t c = 0;
-      bool ok = mbar_wait(&full[0], 0, abrt, status);
-      ChunkMeta cur = meta[0];
-      if (ok && !(cur.flags & kEnd)) {
-        tc_fence_after();
-        issue_s(0);
-      }
-      while (ok && !(cur.flags & kEnd)) {
-        const uint32_t c1 = c + 1;
-        if (!mbar_wait(&full[c1 % kNst], (c1 / kNst) & 1u, abrt, status)) break;
-        const ChunkMeta nxt = meta[c1 % kNst];
-        if (!(nxt.flags & kEnd)) {
-          if (!mbar_wait(&s_free[c1 & 1], ((c1 >> 1) & 1u) ^ 1u, abrt, status)) break;
-          tc_fence_after();
-          issue_s(c1);
-        }
-        if (!mbar_wait(&p_full[c & 1], (c >> 1) & 1u, abrt, status)) break;
-        if (!mbar_wait(&o_free[c & 1], ((c >> 1) & 1u) ^ 1u, abrt, status)) break;
-        tc_fence_after();
-        issue_pv(c, cur.valid);
-        c = c1;
-        cur = nxt;
+        mma_commit(&o_full[t]);
+        mma_commit(&empty[stage]);
+        ++n;
       }
       // all MMAs this thread issued have completed before TMEM is released
-      mma_commit(drain);
-      drain_wait(drain, 0);
+      mma_commit(&drain[t]);
+      drain_wait(&drain[t], 0);
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax / correction
-    const int r = 32 * (warp & 3) + lane;   // TMEM lane: token (softmax) / column d (output)
-    const int wq = warp - 2;                 // 0..3 among the softmax warps
+    const int t = (warp - 3) >> 2;          // group 0: warps 3-6, group 1: warps 7-10
+    const int wq = (warp - 3) & 3;           // 0..3 within the group
+    const int r = 32 * (warp & 3) + lane;    // TMEM lane: token (softmax) / column d (output)
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+    const uint32_t s_col = 16 * t, o_col = 32 + NPV * t;
     const float sl2 = p.scale_log2;
-    float m_run[GQ], l_thr[GQ], o[GQ], a_prev[GQ];
-    uint32_t c = 0, gphase = 0;
-    bool have_prev = false;
-    uint32_t c_prev = 0;
+    uint8_t* pdst_base = pbuf + t * Ly::PBUF + r * 16;
+    float* red_t = red + t * 128;
+    float* lred_t = lred + t * 64;
+    uint64_t* gbar = &grp[t];
+    float m_run[GT], l_thr[GT], o[GT];
+    uint32_t gphase = 0, n = 0;
     float2* ml = reinterpret_cast<float2*>(p.ws + p.ml_off);
     float* po = reinterpret_cast<float*>(p.ws + p.o_off);
 
-    auto correct = [&](uint32_t cc, const float* alpha) -> bool {
-      const int ob = cc & 1;
-      if (!mbar_wait(&o_full[ob], (cc >> 1) & 1u, abrt, status)) return false;
-      tc_fence_after();
-      float ov[NPV];
-      tmem_ld16(lane_addr + 32 + NPV * ob, ov);
-      if constexpr (NPV == 32) tmem_ld16(lane_addr + 32 + NPV * ob + 16, ov + 16);
-      tc_fence_before();
-      mbar_arrive(&o_free[ob]);
-#pragma unroll
-      for (int g = 0; g < GQ; ++g) o[g] = fmaf(o[g], alpha[g], ov[g] + ov[GQ + g]);
-      return true;
-    };
-
-    while (true) {
+    for (uint32_t c = t;; c += 2) {
       const int stage = c % kNst;
-      if (!mbar_wait(&full[stage], (c / kNst) & 1u, abrt, status)) break;
+      if (!mbar_wait(&full[2 * stage + t], (c / (2 * kNst)) & 1u, abrt, status)) break;
       const ChunkMeta mt = meta[stage];
-      if (mt.flags & kEnd) break;
+      if (mt.flags & kEnd) {
+        mbar_arrive(&p_full[t]);   // acknowledge END so the slot can be released
+        break;
+      }
       if (mt.flags & kFirst) {
 #pragma unroll
-        for (int g = 0; g < GQ; ++g) {
+        for (int g = 0; g < GT; ++g) {
           m_run[g] = -INFINITY;
           l_thr[g] = 0.f;
           o[g] = 0.f;
         }
-        have_prev = false;
       }
+      const uint32_t par = n & 1u;
       // ---- scores of token r
-      const int sb = c & 1;
-      if (!mbar_wait(&s_full[sb], (c >> 1) & 1u, abrt, status)) break;
+      if (!mbar_wait(&s_full[t], par, abrt, status)) break;
       tc_fence_after();
       float sv[16];
-      tmem_ld16(lane_addr + 16 * sb, sv);
+      tmem_ld16(lane_addr + s_col, sv);
       tc_fence_before();
-      mbar_arrive(&s_free[sb]);
+      mbar_arrive(&s_free[t]);
       const bool tok_ok = r < mt.valid;
-      float s2[GQ];
+      float s2[GT];
 #pragma unroll
-      for (int g = 0; g < GQ; ++g)
-        s2[g] = (tok_ok && g < G) ? sv[g < 16 ? g : 15] * sl2 : -INFINITY;
-      // ---- chunk max per head across the 128 tokens
-      float* rb = red + (c & 1) * 64;
+      for (int g = 0; g < GT; ++g) s2[g] = (tok_ok && g < G) ? sv[g] * sl2 : -INFINITY;
+      // ---- chunk max per head across the group's 128 threads
+      float* rb = red_t + par * 64;
 #pragma unroll
-      for (int g = 0; g < GQ; ++g) {
+      for (int g = 0; g < GT; ++g) {
         float mx = s2[g];
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
         if (lane == 0) rb[wq * 16 + g] = mx;
       }
-      if (!group_sync(grp, gphase, abrt, status)) break;
-      float alpha[GQ];
-      uint32_t col[NPV];   // P^T row r: column g = hi(p_g), column GQ + g = lo(p_g)
+      if (!group_sync(gbar, gphase, abrt, status)) break;
+      float alpha[GT];
+      uint32_t col[NPV];   // P^T row r: column g = hi(p_g), column GT + g = lo(p_g)
 #pragma unroll
-      for (int g = 0; g < GQ; ++g) {
+      for (int i = 0; i < NPV; ++i) col[i] = 0;
+#pragma unroll
+      for (int g = 0; g < GT; ++g) {
         const float cm = fmaxf(fmaxf(rb[g], rb[16 + g]), fmaxf(rb[32 + g], rb[48 + g]));
         const float mn = fmaxf(m_run[g], cm);
         // heads g >= G never see a finite score; keep them inert (alpha 0, p 0)
@@ -445,18 +489,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint16_t hi, lo;
         split16<T>(pr, hi, lo);
         col[g] = hi;
-        col[GQ + g] = lo;
+        col[GT + g] = lo;
       }
-      uint32_t packed[NPV / 2];
-#pragma unroll
-      for (int w = 0; w < NPV / 2; ++w) packed[w] = col[2 * w] | (col[2 * w + 1] << 16);
-      // ---- store P^T row r: 8 columns (16 B) per core-matrix group
-      uint8_t* pdst = pbuf + (c & 1) * Ly::PBUF + r * 16;
 #pragma unroll
       for (int ng = 0; ng < NPV / 8; ++ng)
-        *reinterpret_cast<uint4*>(pdst + ng * 2048) =
-            make_uint4(packed[ng * 4 + 0], packed[ng * 4 + 1], packed[ng * 4 + 2],
-                       packed[ng * 4 + 3]);
+        *reinterpret_cast<uint4*>(pdst_base + ng * 2048) =
+            make_uint4(col[8 * ng + 0] | (col[8 * ng + 1] << 16),
+                       col[8 * ng + 2] | (col[8 * ng + 3] << 16),
+                       col[8 * ng + 4] | (col[8 * ng + 5] << 16),
+                       col[8 * ng + 6] | (col[8 * ng + 7] << 16));
       if (!tok_ok) {
         // rows past the chunk's valid tokens: make V finite (zero) for the MMA
         uint8_t* vrow = smem + static_cast<size_t>(stage) * kStage + 2 * kHalf + r * 128;
@@ -467,37 +508,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       fence_proxy_async_smem();
-      mbar_arrive(&p_full[c & 1]);
-      // ---- deferred correction of the previous chunk of this item
-      if (have_prev) {
-        if (!correct(c_prev, a_prev)) break;
-      }
+      mbar_arrive(&p_full[t]);
+      // ---- correction: O = alpha * O + O_chunk (thread r owns column d = r)
+      if (!mbar_wait(&o_full[t], par, abrt, status)) break;
+      tc_fence_after();
+      float ov[NPV];
+      tmem_ld16(lane_addr + o_col, ov);
+      if constexpr (NPV == 32) tmem_ld16(lane_addr + o_col + 16, ov + 16);
+      tc_fence_before();
+      mbar_arrive(&o_free[t]);
 #pragma unroll
-      for (int g = 0; g < GQ; ++g) a_prev[g] = alpha[g];
-      have_prev = true;
-      c_prev = c;
+      for (int g = 0; g < GT; ++g) o[g] = fmaf(o[g], alpha[g], ov[g] + ov[GT + g]);
+      ++n;
 
       if (mt.flags & kLast) {
-        if (!correct(c, a_prev)) break;
-        have_prev = false;
-        // sum of l over the 128 tokens
+        // sum of l over the group's 128 tokens
 #pragma unroll
-        for (int g = 0; g < GQ; ++g) {
+        for (int g = 0; g < GT; ++g) {
           float lg = l_thr[g];
 #pragma unroll
           for (int off = 16; off > 0; off >>= 1) lg += __shfl_xor_sync(kFull, lg, off);
-          if (lane == 0) lred[wq * 16 + g] = lg;
+          if (lane == 0) lred_t[wq * 16 + g] = lg;
         }
-        if (!group_sync(grp, gphase, abrt, status)) break;
+        if (!group_sync(gbar, gphase, abrt, status)) break;
         const int nsp = item_nsplit(mt.split_raw);
-        const bool single = nsp == 1;
         const int split = item_split(mt.split_raw);
 #pragma unroll
-        for (int g = 0; g < GQ; ++g) {
+        for (int g = 0; g < GT; ++g) {
           if (g >= G) break;
-          const float L = lred[g] + lred[16 + g] + lred[32 + g] + lred[48 + g];
+          const float L = lred_t[g] + lred_t[16 + g] + lred_t[32 + g] + lred_t[48 + g];
           const size_t row = static_cast<size_t>(mt.seq) * p.num_q_heads + mt.kvh * G + g;
-          if (single) {
+          if (nsp == 1) {
             p.out[row * kD + r] = o[g] / L;
           } else {
             const size_t pr_ = row * p.max_splits + split;
@@ -506,7 +547,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      ++c;
     }
   }
   tc_fence_before();
@@ -553,9 +593,9 @@ cudaError_t make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t b
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <typename T, int NPV>
+template <typename T, int GT>
 cudaError_t launch_t(const DecodeParams& p, int num_ctas, cudaStream_t stream) {
-  using Ly = TcLayout<NPV>;
+  using Ly = TcLayout<GT>;
   const bool bf16 = std::is_same<T, __nv_bfloat16>::value;
   CUtensorMap mk, mv, mq;
   const uint64_t pool_rows =
@@ -565,7 +605,7 @@ cudaError_t launch_t(const DecodeParams& p, int num_ctas, cudaStream_t stream) {
   if (e == cudaSuccess)
     e = make_map(&mq, p.q, static_cast<uint64_t>(p.num_seqs) * p.num_q_heads, 16, bf16);
   if (e != cudaSuccess) return e;
-  auto kern = tc_decode_kernel<T, NPV>;
+  auto kern = tc_decode_kernel<T, GT>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(Ly::SMEM));
   if (e != cudaSuccess) return e;
@@ -591,11 +631,13 @@ cudaError_t launch_decode_tc(const DecodeParams& p, int num_ctas, cudaStream_t s
   const int group = p.num_q_heads / p.num_kv_heads;
   if (!tc_supported(p.dtype, p.head_dim, group)) return cudaErrorInvalidValue;
   if (p.dtype == 2) {
-    return group <= 8 ? launch_t<__nv_bfloat16, 16>(p, num_ctas, stream)
-                      : launch_t<__nv_bfloat16, 32>(p, num_ctas, stream);
+    if (group <= 4) return launch_t<__nv_bfloat16, 4>(p, num_ctas, stream);
+    if (group <= 8) return launch_t<__nv_bfloat16, 8>(p, num_ctas, stream);
+    return launch_t<__nv_bfloat16, 16>(p, num_ctas, stream);
   }
-  return group <= 8 ? launch_t<__half, 16>(p, num_ctas, stream)
-                    : launch_t<__half, 32>(p, num_ctas, stream);
+  if (group <= 4) return launch_t<__half, 4>(p, num_ctas, stream);
+  if (group <= 8) return launch_t<__half, 8>(p, num_ctas, stream);
+  return launch_t<__half, 16>(p, num_ctas, stream);
 }
 
 }  // namespace pa
