@@ -253,18 +253,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tm_q);
     }
     const WorkPair* pairs = reinterpret_cast<const WorkPair*>(p.ws + p.pairs_off);
-    int kraw0 = 0, kraw1 = 0;
-    if (lane == 0) {
-      kraw0 = atomicAdd(&hdr->work_counter, 1);
-      kraw1 = atomicAdd(&hdr->work_counter, 1);
-    }
-    // per-stream state (warp-uniform); two named copies so every access is a
-    // register select, not an indexed local array
+    // Per-stream state (warp-uniform), plus a window of block-table entries:
+    // lane j holds entries wbase + j and wbase + 32 + j of the current item.
+    // The next item of each stream is prefetched one step per emission
+    // (claim -> work pair -> first table window), so item switches and table
+    // reads rarely stall the chunk issue. Two named copies keep every access a
+    // register select.
     struct Stream {
-      int seq, kvh, split_n, tb, te, cs;
+      int seq, kvh, split_n, tb, te, cs;   // current item, next chunk start
+      int wbase, w0, w1;                   // table window of the current item
+      int nst;                             // next item: 0 none, 1 claimed, 2 pair, 3 window, 4 no more
+      int nkraw;                           // claim result (lane 0)
+      int nseq, nkvh, nsplit_n, ntb, nte;  // next item's work pair
+      int nw0, nw1;                        // next item's first window
       bool ended;
     };
-    Stream st0 = {0, 0, 0, 0, 0, 0, false}, st1 = st0;
+    Stream st0 = {};
+    st0.ended = false;
+    Stream st1 = st0;
+    auto load_window = [&](int sq, int first_page, int& a, int& b) {
+      const int32_t* row = p.block_tables + static_cast<size_t>(sq) * p.bt_stride;
+      const int i0 = first_page + lane, i1 = first_page + 32 + lane;
+      a = i0 < p.bt_stride ? row[i0] : 0;
+      b = i1 < p.bt_stride ? row[i1] : 0;
+    };
+    // one prefetch step for the next item of stream `cur`
+    auto prefetch_step = [&](Stream& cur) {
+      if (cur.nst == 0) {
+        int kr = 0;
+        if (lane == 0) kr = atomicAdd(&hdr->work_counter, 1);
+        cur.nkraw = kr;
+        cur.nst = 1;
+      } else if (cur.nst == 1) {
+        const int k = __shfl_sync(kFull, cur.nkraw, 0);
+        if (k < num_items) {
+          const int pi = k / Hkv;
+          const WorkPair wp = pairs[pi];
+          cur.nseq = wp.seq;
+          cur.nkvh = k - pi * Hkv;
+          cur.nsplit_n = wp.split_n;
+          cur.ntb = wp.t_begin;
+          cur.nte = wp.t_end;
+          cur.nst = 2;
+        } else {
+          cur.nst = 4;
+        }
+      } else if (cur.nst == 2) {
+        load_window(cur.nseq, cur.ntb / BS, cur.nw0, cur.nw1);
+        cur.nst = 3;
+      }
+    };
     int stops = 0;
     uint32_t c = 0;
     bool ok = true;
@@ -274,23 +312,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool other_ended = t ? st0.ended : st1.ended;
       int kind = 0;   // 0 data, 1 end, 2 bubble, 3 stop
       if (!cur.ended && cur.cs >= cur.te) {
-        const int k = __shfl_sync(kFull, t == 0 ? kraw0 : kraw1, 0);
-        if (k < num_items) {
-          const int pi = k / Hkv;
-          const WorkPair wp = pairs[pi];
-          if (lane == 0) {
-            if (t == 0) kraw0 = atomicAdd(&hdr->work_counter, 1);   // next claim in flight
-            else kraw1 = atomicAdd(&hdr->work_counter, 1);
-          }
-          cur.seq = wp.seq;
-          cur.kvh = k - pi * Hkv;
-          cur.split_n = wp.split_n;
-          cur.tb = wp.t_begin;
-          cur.te = wp.t_end;
-          cur.cs = wp.t_begin;
-        } else {
+        // current item done: finish the prefetch of the next one, then switch
+        while (cur.nst < 3) prefetch_step(cur);
+        if (cur.nst == 4) {
           cur.ended = true;
           kind = 1;
+        } else {
+          cur.seq = cur.nseq;
+          cur.kvh = cur.nkvh;
+          cur.split_n = cur.nsplit_n;
+          cur.tb = cur.ntb;
+          cur.te = cur.nte;
+          cur.cs = cur.ntb;
+          cur.wbase = cur.ntb / BS;
+          cur.w0 = cur.nw0;
+          cur.w1 = cur.nw1;
+          cur.nst = 0;
         }
       } else if (cur.ended) {
         kind = other_ended ? 3 : 2;
@@ -299,13 +336,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (kind == 0) {
         valid = min(kChunk, cur.te - cur.cs);
         npg = (valid + BS - 1) / BS;
-        if (lane < npg) {
-          blk = p.block_tables[static_cast<size_t>(cur.seq) * p.bt_stride + cur.cs / BS + lane];
-          if (blk < 0 || blk >= p.num_blocks) {
-            atomicCAS(status, 0, 1 /* PA_ERR_INVALID_ARG */);
-            blk = 0;
-          }
+        const int p0 = cur.cs / BS;
+        if (p0 + npg > cur.wbase + 64) {   // chunk runs past the window: next window
+          cur.wbase = p0;
+          load_window(cur.seq, p0, cur.w0, cur.w1);
         }
+        const int j = p0 - cur.wbase + lane;   // window index of this lane's page
+        const int e0 = __shfl_sync(kFull, cur.w0, j & 31);
+        const int e1 = __shfl_sync(kFull, cur.w1, j & 31);
+        blk = j < 32 ? e0 : e1;
+        if (lane < npg && (blk < 0 || blk >= p.num_blocks)) {
+          atomicCAS(status, 0, 1 /* PA_ERR_INVALID_ARG */);
+          blk = 0;
+        }
+        prefetch_step(cur);   // advance the next item's prefetch by one step
       }
       const int stage = c % kNst;
       if (!mbar_wait(&empty[stage], ((c / kNst) & 1u) ^ 1u, abrt, status)) {

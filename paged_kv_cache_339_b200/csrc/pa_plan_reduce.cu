@@ -34,34 +34,15 @@ __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
   return v;
 }
 
-// Exclusive scan of one int per thread over the CTA; the total goes to *total.
-__device__ int block_excl_scan(int v, int* scratch, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nwarps = blockDim.x >> 5;
-  int inc = warp_incl_scan(v, lane);
-  if (lane == 31) scratch[warp] = inc;
-  __syncthreads();
-  if (warp == 0) {
-    int w = lane < nwarps ? scratch[lane] : 0;
-    int wi = warp_incl_scan(w, lane);
-    scratch[32 + lane] = wi - w;
-    if (lane == 31) scratch[64] = wi;
-  }
-  __syncthreads();
-  int res = scratch[32 + warp] + inc - v;
-  *total = scratch[64];
-  __syncthreads();
-  return res;
-}
-
 __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) {
   pdl_launch_dependents();
   __shared__ long long s_sum[32];
   __shared__ int s_max[32];
   __shared__ int s_bad[32];
-  __shared__ int s_scan[96];
   __shared__ int s_split;
   __shared__ int s_maxn;
+  __shared__ int s_total;
+  extern __shared__ int cell_cnt[];   // [levels][32-sequence groups]
 
   WsHeader* hdr = reinterpret_cast<WsHeader*>(p.ws);
   WorkPair* pairs = reinterpret_cast<WorkPair*>(p.ws + p.pairs_off);
@@ -137,30 +118,53 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
   }
   __syncthreads();
 
-  // 3. split-major pair list
-  int base = 0;
-  for (int s = 0; s < maxn; ++s) {
-    for (int i0 = 0; i0 < p.num_seqs; i0 += nthreads) {
-      const int i = i0 + tid;
-      int n = 0, L = 0;
-      if (i < p.num_seqs) {
-        n = nsplit[i];
-        L = p.context_lens[i];
-      }
-      const int f = (n > s) ? 1 : 0;
-      int count;
-      const int rank = block_excl_scan(f, s_scan, &count);
-      if (f) {
-        WorkPair w;
-        w.seq = i;
-        w.split_n = s | (n << 16);
-        w.t_begin = s * S;
-        w.t_end = min(L, (s + 1) * S);
-        pairs[base + rank] = w;
-      }
-      base += count;
+  // 3. split-major pair list: position of (i, s) = base_s + rank_s(i), with
+  // base_s = number of pairs at levels < s and rank_s(i) = number of
+  // sequences j < i with more than s splits. Per 32-sequence group and level,
+  // a ballot gives the group's count and each lane's rank inside the group;
+  // one scan over the (level, group) counts gives every group's base.
+  const int ngroups = (p.num_seqs + 31) / 32;
+  const int ncells = maxn * ngroups;   // (level, group) cells, level-major
+  for (int cell = warp; cell < ncells; cell += nwarps) {
+    const int s = cell / ngroups, g = cell - s * ngroups;
+    const int i = g * 32 + lane;
+    const int n = i < p.num_seqs ? nsplit[i] : 0;
+    const unsigned m = __ballot_sync(0xffffffffu, n > s);
+    if (lane == 0) cell_cnt[cell] = __popc(m);
+  }
+  __syncthreads();
+  // exclusive scan of cell_cnt (level-major) by warp 0
+  if (warp == 0) {
+    int carry = 0;
+    for (int c0 = 0; c0 < ncells; c0 += 32) {
+      const int c = c0 + lane;
+      const int v = c < ncells ? cell_cnt[c] : 0;
+      const int inc = warp_incl_scan(v, lane);
+      if (c < ncells) cell_cnt[c] = carry + inc - v;
+      carry += __shfl_sync(0xffffffffu, inc, 31);
+    }
+    if (lane == 0) s_total = carry;
+  }
+  __syncthreads();
+  for (int cell = warp; cell < ncells; cell += nwarps) {
+    const int s = cell / ngroups, g = cell - s * ngroups;
+    const int i = g * 32 + lane;
+    int n = 0, L = 0;
+    if (i < p.num_seqs) {
+      n = nsplit[i];
+      L = p.context_lens[i];
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, n > s);
+    if (n > s) {
+      WorkPair w;
+      w.seq = i;
+      w.split_n = s | (n << 16);
+      w.t_begin = s * S;
+      w.t_end = min(L, (s + 1) * S);
+      pairs[cell_cnt[cell] + __popc(m & ((1u << lane) - 1u))] = w;
     }
   }
+  const int base = s_total;
   if (tid == 0) {
     hdr->num_pairs = base;
     hdr->num_items = base * p.num_kv_heads;
@@ -231,10 +235,18 @@ cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream) {
 cudaError_t launch_plan(const PlanParams& p, cudaStream_t stream) {
   int threads = (p.num_seqs + 31) / 32 * 32;
   threads = threads < 64 ? 64 : (threads > kPlanMaxThreads ? kPlanMaxThreads : threads);
+  const size_t cells = static_cast<size_t>(p.max_splits) * ((p.num_seqs + 31) / 32);
+  const size_t smem = cells * sizeof(int);
+  if (smem > 227 * 1024) return cudaErrorInvalidValue;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(1);
   cfg.blockDim = dim3(threads);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
