@@ -355,8 +355,8 @@ def oracle_sample(b, seconds):
         L = int(b.context_lens[i])
         nb = (L + BS - 1) // BS
         rows = b.block_tables[i, :nb].long()
-        kc = b.k_cache[rows].to(torch.float32).cpu().numpy().astype(np.float64)
-        vc = b.v_cache[rows].to(torch.float32).cpu().numpy().astype(np.float64)
+        kc = ORACLE.logical_pool(b.k_cache[rows].to(torch.float32).cpu().numpy().astype(np.float64))
+        vc = ORACLE.logical_pool(b.v_cache[rows].to(torch.float32).cpu().numpy().astype(np.float64))
         q = b.q[i].to(torch.float32).cpu().numpy().astype(np.float64)
         t0 = time.perf_counter()
         tab = np.arange(nb)

@@ -17,6 +17,15 @@ Pages: "Paged Attention: Virtual Memory for the KV Cache" (P1),
   borrowed from operating systems"; P2, "Virtual Memory as the Blueprint").
   Layout reading: two pools ``k_cache`` / ``v_cache`` of shape
   ``[num_blocks, num_kv_heads, block_size, head_dim]``.
+* In-block storage order. Each (block, KV head) tile of block_size x head_dim
+  elements is stored contiguously, its rows cut into 64-element halves and
+  grouped 16 tokens at a time: element (t, d) sits at
+  ((t // SH) * NH + d // 64) * SH * 64 + (t % SH) * 64 + d % 64 with
+  SH = min(block_size, 16) and NH = head_dim // 64 (plain row-major when
+  head_dim is 64). ``logical_pool`` / ``physical_pool`` convert between this
+  order and the logical ``[num_blocks, num_kv_heads, block_size, head_dim]``
+  view every other function here works on. The pages leave the inside of a
+  block open; this order lets one copy of a tile feed the tensor cores.
 * Block table. Each sequence keeps an ordered list of the physical blocks that
   hold it; logical token ``j`` lives in block ``table[j // block_size]`` at
   offset ``j % block_size`` (P1, "The fix borrowed from operating systems").
@@ -53,6 +62,30 @@ import numpy as np
 class PagedAttentionOracle:
     """fp64 reference. Methods are overridable so the pin suite can plant
     mistakes in a subclass and check that some pin catches each one."""
+
+    # ------------------------------------------------------------------
+    # In-block storage order (a reading: the pages leave it open)
+    # ------------------------------------------------------------------
+    def tile_offset(self, t: int, d: int, block_size: int, head_dim: int) -> int:
+        """Element offset of (token t, column d) inside one (block, head) tile."""
+        sh = min(block_size, 16)
+        nh = head_dim // 64
+        return ((t // sh) * nh + d // 64) * sh * 64 + (t % sh) * 64 + d % 64
+
+    def logical_pool(self, pool: np.ndarray) -> np.ndarray:
+        """Stored pool [NB, Hkv, BS, D] (tiles in storage order) -> logical
+        [NB, Hkv, BS, D] with element [b, h, t, d] = K/V of token t, column d."""
+        NB, H, BS, D = pool.shape
+        sh, nh = min(BS, 16), D // 64
+        return (pool.reshape(NB, H, BS // sh, nh, sh, 64)
+                .transpose(0, 1, 2, 4, 3, 5).reshape(NB, H, BS, D))
+
+    def physical_pool(self, pool: np.ndarray) -> np.ndarray:
+        """Inverse of logical_pool."""
+        NB, H, BS, D = pool.shape
+        sh, nh = min(BS, 16), D // 64
+        return (pool.reshape(NB, H, BS // sh, sh, nh, 64)
+                .transpose(0, 1, 2, 4, 3, 5).reshape(NB, H, BS, D))
 
     # ------------------------------------------------------------------
     # Block addressing (P1, "The fix borrowed from operating systems")
@@ -172,6 +205,9 @@ class PagedAttentionOracle:
 ORACLE = PagedAttentionOracle()
 
 # Module-level names for the common calls.
+logical_pool = ORACLE.logical_pool
+physical_pool = ORACLE.physical_pool
+tile_offset = ORACLE.tile_offset
 gather = ORACLE.gather
 attend = ORACLE.attend
 decode = ORACLE.decode

@@ -72,7 +72,8 @@ cudaError_t cached_ctas(bool tc, int dtype, int head_dim, int group, int* out) {
   return cudaSuccess;
 }
 
-constexpr int kItemsPerCta = 12;
+constexpr int kItemsPerCta = 12;      // CUDA-core kernel: per persistent CTA
+constexpr int kItemsPerStreamTc = 8;  // tensor-core kernel: per item stream
 
 }  // namespace
 
@@ -113,7 +114,8 @@ pa_status pa_write_kv(const pa_kv_cache* cache, const void* key, const void* val
   const int64_t num_slots = static_cast<int64_t>(cache->num_blocks) * cache->block_size;
   cudaError_t e = launch_write_kv(cache->k_cache, cache->v_cache, key, value, slot_mapping,
                                   num_tokens, cache->num_kv_heads, cache->block_size, row_bytes,
-                                  num_slots, static_cast<cudaStream_t>(stream));
+                                  elem_bytes(cache->dtype), num_slots,
+                                  static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PA_OK : cuda_fail(e);
 }
 
@@ -215,7 +217,7 @@ pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
   pp.max_splits = lay.max_splits;
   // the tensor-core kernel runs two independent item streams per CTA
   pp.num_ctas = use_tc ? 2 * ctas : ctas;
-  pp.items_per_cta = kItemsPerCta;
+  pp.items_per_cta = use_tc ? kItemsPerStreamTc : kItemsPerCta;
   e = launch_plan(pp, s);
   if (e != cudaSuccess) return cuda_fail(e);
 

@@ -198,6 +198,22 @@ __device__ __forceinline__ void unpack16(const uint4& v, float* f) {
   }
 }
 
+// In-block storage order of one (block, KV head) tile of block_size x
+// head_dim elements: rows cut into 64-element halves and grouped 16 tokens at
+// a time, so element (t, d) sits at
+//   ((t / SH) * NH + d / 64) * SH * 64 + (t % SH) * 64 + d % 64,
+// SH = min(block_size, 16), NH = head_dim / 64 (row-major when head_dim = 64).
+// A whole tile is one contiguous range, and each 16-token group of one half
+// is a run of 128-byte (16-bit) rows that a single 2-D TMA box and the tensor
+// cores consume directly.
+__host__ __device__ __forceinline__ int tile_sub_height(int block_size) {
+  return block_size < 16 ? block_size : 16;
+}
+__host__ __device__ __forceinline__ int tile_offset(int t, int d, int block_size, int head_dim) {
+  const int sh = tile_sub_height(block_size), nh = head_dim >> 6;
+  return ((t / sh) * nh + (d >> 6)) * sh * 64 + (t % sh) * 64 + (d & 63);
+}
+
 // Work-item record written by the planning kernel: one per (sequence, split);
 // the KV-head index is folded into the claimed item number.
 struct __align__(16) WorkPair {

@@ -16,6 +16,8 @@
 //               output columns; at the end of an item the warps' partial
 //               (max, sum, acc) are merged and written as the final row or as a
 //               split partial.
+// Tiles are kept in the in-block storage order (pa_common.cuh) in shared
+// memory too; rows are addressed through it.
 // The block table is followed page by page, so the sequence is read in its
 // logical order although its blocks sit anywhere in the pool ("Paged
 // Attention: Virtual Memory for the KV Cache", "The fix borrowed from
@@ -50,6 +52,8 @@ struct SimtTraits {
   static constexpr int EPL = D / 32;           // output columns per lane
   static constexpr int PVB = ROW / 32;         // bytes per lane per V row
   static constexpr int SUB = 16;               // tokens per softmax sub-block
+  static constexpr int NH = D / 64;            // 64-element halves per row
+  static constexpr int HALF = 64 * E;          // bytes of one half-row
   static constexpr int CMB = GPW * D + 2 * GPW;  // floats per warp in the merge area
   static constexpr size_t OFF_BAR = static_cast<size_t>(NST) * STAGE;
   static constexpr size_t OFF_META = OFF_BAR + (2 * NST + 2) * 8;
@@ -180,12 +184,28 @@ __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
         }
         __syncwarp();
         if (lane < npg) {
+          // one copy per tile; a partly used last tile copies only its valid
+          // rows, one 16-token half-row segment at a time
           const int rows = min(BS, valid - lane * BS);
           const size_t src = (static_cast<size_t>(blk) * Hkv + kvh) * BS * ROW;
+          const uint8_t* gk = static_cast<const uint8_t*>(p.k_cache) + src;
+          const uint8_t* gv = static_cast<const uint8_t*>(p.v_cache) + src;
           uint8_t* dk = stages + static_cast<size_t>(stage) * Tr::STAGE + lane * BS * ROW;
-          bulk_g2s(dk, static_cast<const uint8_t*>(p.k_cache) + src, rows * ROW, &full[stage]);
-          bulk_g2s(dk + CHUNK * ROW, static_cast<const uint8_t*>(p.v_cache) + src, rows * ROW,
-                   &full[stage]);
+          if (rows == BS || Tr::NH == 1) {
+            bulk_g2s(dk, gk, rows * ROW, &full[stage]);
+            bulk_g2s(dk + CHUNK * ROW, gv, rows * ROW, &full[stage]);
+          } else {
+            const int sh = tile_sub_height(BS);
+            for (int sp = 0; sp * sh < rows; ++sp) {
+              const uint32_t nb = static_cast<uint32_t>(min(sh, rows - sp * sh)) * Tr::HALF;
+#pragma unroll
+              for (int h = 0; h < Tr::NH; ++h) {
+                const int seg = (sp * Tr::NH + h) * sh * Tr::HALF;
+                bulk_g2s(dk + seg, gk + seg, nb, &full[stage]);
+                bulk_g2s(dk + CHUNK * ROW + seg, gv + seg, nb, &full[stage]);
+              }
+            }
+          }
         }
         ++c;
       }
@@ -220,6 +240,26 @@ __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
     const int TPW = CHUNK / WPG;
     const int gi = lane >> 3, j = lane & 7;
     float* ps_w = pscr + cw * Tr::SUB * 4;
+    // in-block storage order: byte offset of token t's first half-row inside
+    // a stage region (pages packed in table order); half h adds h * seg
+    const int bs_shift = __ffs(BS) - 1;
+    const int sh = tile_sub_height(BS), sh_shift = __ffs(sh) - 1;
+    const int seg = sh * Tr::HALF;
+    auto row_off = [&](int t) -> int {
+      const int r = t & (BS - 1);
+      return (t >> bs_shift) * BS * ROW + (r >> sh_shift) * Tr::NH * seg + (r & (sh - 1)) * Tr::HALF;
+    };
+    // Rows of consecutive groups of sh tokens are sh * ROW bytes apart (pages
+    // are packed), so inside a 16-token sub-block (which starts on a multiple of
+    // 16) token tb + i is at row_off(tb) + (i / sh) * sh * ROW + (i % sh) * HALF.
+    const int grp_stride = sh * ROW;
+    // score loads: vector j + 8v of a row lies in half v * EPV / 8
+    int kofs[Tr::NV];
+#pragma unroll
+    for (int v = 0; v < Tr::NV; ++v)
+      kofs[v] = ((v * Tr::EPV) >> 3) * seg + ((j + 8 * v) * 16) % Tr::HALF;
+    // PV: this lane's columns d = lane * EPL .. lie in half (lane * EPL) / 64
+    const int pv_off = ((lane * Tr::EPL) >> 6) * seg + (lane * Tr::PVB) % Tr::HALF;
     float q[GPW][Tr::QPL];
     float m[GPW], l[GPW], o[GPW][Tr::EPL];
     uint32_t c = 0, gphase = 0;
@@ -255,19 +295,23 @@ __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
         const int tw0 = wg * TPW;
         const int tend = min(tw0 + TPW, mt.valid);
         for (int tb = tw0; tb < tend; tb += Tr::SUB) {
+          const int sb_off = row_off(tb);
+          auto tok_off = [&](int i) {   // token tb + i, 0 <= i < 16
+            return sb_off + (i >> sh_shift) * grp_stride + (i & (sh - 1)) * Tr::HALF;
+          };
           // scores of tokens tb .. tb+15 (lane group gi takes every 4th)
           float s[4][GPW];
 #pragma unroll
           for (int pp = 0; pp < 4; ++pp) {
             const int t = tb + pp * 4 + gi;
-            const uint8_t* krow = Kst + t * ROW;
+            const uint8_t* krow = Kst + tok_off(pp * 4 + gi);
             float acc[GPW];
 #pragma unroll
             for (int g = 0; g < GPW; ++g) acc[g] = 0.f;
 #pragma unroll
             for (int v = 0; v < Tr::NV; ++v) {
               float f[Tr::EPV];
-              unpack16<T>(*reinterpret_cast<const uint4*>(krow + (j + 8 * v) * 16), f);
+              unpack16<T>(*reinterpret_cast<const uint4*>(krow + kofs[v]), f);
 #pragma unroll
               for (int g = 0; g < GPW; ++g)
 #pragma unroll
@@ -316,7 +360,7 @@ __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
             const float4 pw = *reinterpret_cast<const float4*>(ps_w + tt * 4);
             const float pv[4] = {pw.x, pw.y, pw.z, pw.w};
             float vf[Tr::EPL];
-            load_row_slice<T, Tr::PVB>(Vst + (tb + tt) * ROW + lane * Tr::PVB, vf);
+            load_row_slice<T, Tr::PVB>(Vst + tok_off(tt) + pv_off, vf);
 #pragma unroll
             for (int g = 0; g < GPW; ++g)
 #pragma unroll

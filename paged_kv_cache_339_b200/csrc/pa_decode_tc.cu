@@ -50,9 +50,9 @@ constexpr int kFirst = 1, kLast = 2, kEnd = 4, kBubble = 8, kStop = 16;
 constexpr int kChunk = 128;   // tokens per stage (= MMA M)
 constexpr int kD = 128;       // head_dim
 constexpr int kNst = 3;       // pipeline stages
-constexpr int kHalf = kChunk * 128;           // one 64-column half: 128 rows x 128 B
-constexpr int kQHalf = 16 * 128;              // Q half: 16 rows x 128 B
-constexpr int kStage = 4 * kHalf + 2 * kQHalf;  // K (2 halves), V (2 halves), Q (2 halves)
+constexpr int kTile = kChunk * 256;           // K (or V) of 128 tokens: 256 half-rows x 128 B
+constexpr int kQReg = 32 * 128;               // Q' region: up to 32 half-rows x 128 B
+constexpr int kStage = 2 * kTile + kQReg;     // K, V, Q' of one chunk
 constexpr int kThreads = 352;  // producer, 2 MMA issuers, 2 softmax groups of 4 warps
 
 struct __align__(16) ChunkMeta {
@@ -74,7 +74,10 @@ struct TcLayout {
   static constexpr size_t OFF_MISC = OFF_LRED + 2 * 4 * 16 * 4;
   static constexpr size_t SMEM_USED = OFF_MISC + 16;
   static constexpr size_t SMEM = SMEM_USED + 1024;   // slack to align the base to 1 KB
-  static constexpr uint32_t TMEM_COLS = (32 + 2 * NPV) <= 64 ? 64 : 128;
+  static constexpr int NS = GT <= 8 ? 16 : 32;       // score MMA N: two halves x heads
+  // per stream: two score accumulators (NS columns each) and the O^T accumulator
+  static constexpr int COLS_PER_STREAM = 2 * NS + NPV;
+  static constexpr uint32_t TMEM_COLS = 2 * COLS_PER_STREAM <= 128 ? 128 : 256;
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(kStage % 1024 == 0 && OFF_P % 1024 == 0, "swizzled tiles need 1 KB alignment");
   static_assert(OFF_BAR % 8 == 0, "mbarriers need 8-byte alignment");
@@ -369,19 +372,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           m.flags = (cur.cs == cur.tb ? kFirst : 0) | (cur.cs + kChunk >= cur.te ? kLast : 0);
           m.pad0 = m.pad1 = 0;
           meta[stage] = m;
-          mbar_arrive_expect_tx(fb, static_cast<uint32_t>(npg * BS * 512 + 2 * kQHalf));
+          // K and V: one box of 2*BS half-rows per page; Q': the group's query
+          // rows, first halves then second halves (NS/2 rows each)
+          mbar_arrive_expect_tx(fb, static_cast<uint32_t>(npg * BS * 512 + Ly::NS * 128));
           const int q_row = cur.seq * p.num_q_heads + cur.kvh * G;
-          tma_load_2d(st + 4 * kHalf, &tm_q, 0, q_row, fb);
-          tma_load_2d(st + 4 * kHalf + kQHalf, &tm_q, 64, q_row, fb);
+          tma_load_2d(st + 2 * kTile, &tm_q, 0, q_row, fb);
+          tma_load_2d(st + 2 * kTile + (Ly::NS / 2) * 128, &tm_q, 64, q_row, fb);
         }
         __syncwarp();
         if (lane < npg) {
-          const int row = (blk * Hkv + cur.kvh) * BS;
-          const int off = lane * BS * 128;
+          const int row = (blk * Hkv + cur.kvh) * BS * 2;   // first half-row of the tile
+          const int off = lane * BS * 256;
           tma_load_2d(st + off, &tm_k, 0, row, fb);
-          tma_load_2d(st + kHalf + off, &tm_k, 64, row, fb);
-          tma_load_2d(st + 2 * kHalf + off, &tm_v, 0, row, fb);
-          tma_load_2d(st + 3 * kHalf + off, &tm_v, 64, row, fb);
+          tma_load_2d(st + kTile + off, &tm_v, 0, row, fb);
         }
         cur.cs += kChunk;
       } else {
@@ -406,12 +409,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int t = warp - 1;   // group served
     if (lane == 0) {
       const uint32_t fmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
-      const uint32_t idesc_s = instr_desc(fmt, false, false, 128, 16);
+      const uint32_t idesc_s = instr_desc(fmt, false, false, 128, Ly::NS);
+      const uint32_t sh = static_cast<uint32_t>(tile_sub_height(BS));
+      const uint32_t v_sbo = sh == 16 ? 1024u : 2048u;   // 8-token groups
       const uint32_t idesc_pv = instr_desc(fmt, true, true, 128, NPV);
       const uint32_t sbase = smem_u32(smem);
       const uint32_t pb = smem_u32(pbuf) + t * Ly::PBUF;
-      const uint32_t s_tm = tmem + 16 * t;
-      const uint32_t o_tm = tmem + 32 + NPV * t;
+      const uint32_t s_tm = tmem + t * Ly::COLS_PER_STREAM;   // two NS-column score tiles
+      const uint32_t o_tm = s_tm + 2 * Ly::NS;
       uint32_t n = 0;   // data chunks of this group so far
       for (uint32_t c = t;; c += 2) {
         const int stage = c % kNst;
@@ -431,16 +436,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(&empty[stage]);
           continue;
         }
-        // S^T = K . Q^T
+        // Half-row scores: the K region holds 256 half-rows (token, half) of
+        // 128 B; Q' holds the query rows' first halves then their second
+        // halves. S'[(t, h), (h', g)] = K_h[t] . Q_h'[g]; the softmax group
+        // adds the two h == h' terms of each token.
         if (!mbar_wait(&s_free[t], par ^ 1u, abrt, status)) break;
         tc_fence_after();
         const uint32_t stg = sbase + stage * kStage;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t half = kk >> 2, koff = (kk & 3) * 32;
-          const uint64_t a = smem_desc(stg + half * kHalf + koff, 16, 1024, kSw128);
-          const uint64_t b = smem_desc(stg + 4 * kHalf + half * kQHalf + koff, 16, 1024, kSw128);
-          mma_f16(s_tm, a, b, idesc_s, kk > 0 ? 1u : 0u);
+        for (int m = 0; m < 2; ++m) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t a = smem_desc(stg + m * 16384 + kk * 32, 16, 1024, kSw128);
+            const uint64_t b = smem_desc(stg + 2 * kTile + kk * 32, 16, 1024, kSw128);
+            mma_f16(s_tm + m * Ly::NS, a, b, idesc_s, kk > 0 ? 1u : 0u);
+          }
         }
         mma_commit(&s_full[t]);
         // O^T = V^T . P^T once the softmax group has written P
@@ -449,7 +459,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const int nks = (mt.valid + 15) >> 4;
         for (int ks = 0; ks < nks; ++ks) {
-          const uint64_t a = smem_desc(stg + 2 * kHalf + ks * 2048, kHalf, 1024, kSw128);
+          // V^T for tokens 16ks..16ks+15: 4 KB of half-rows; M atoms (column
+          // halves) sh * 128 B apart, 8-token groups v_sbo apart
+          const uint64_t a = smem_desc(stg + kTile + ks * 4096, sh * 128, v_sbo, kSw128);
           const uint64_t b = smem_desc(pb + ks * 256, 128, 2048, kSwNone);
           mma_f16(o_tm, a, b, idesc_pv, ks > 0 ? 1u : 0u);
         }
@@ -466,11 +478,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ softmax / correction
     const int t = (warp - 3) >> 2;          // group 0: warps 3-6, group 1: warps 7-10
     const int wq = (warp - 3) & 3;           // 0..3 within the group
-    const int r = 32 * (warp & 3) + lane;    // TMEM lane: token (softmax) / column d (output)
+    const int r = 32 * (warp & 3) + lane;    // TMEM lane: score half-row / output column d
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
-    const uint32_t s_col = 16 * t, o_col = 32 + NPV * t;
+    const uint32_t s_col = t * Ly::COLS_PER_STREAM, o_col = s_col + 2 * Ly::NS;
     const float sl2 = p.scale_log2;
-    uint8_t* pdst_base = pbuf + t * Ly::PBUF + r * 16;
+    // Half-row r of score tile m is (token tk0 + 64 m, half hh); its partner
+    // half-row (same token, other half) is lane r ^ sh of the same warp.
+    const int sh = tile_sub_height(BS);
+    const int hh = (r / sh) & 1;
+    const int tk0 = (r / (2 * sh)) * sh + r % sh;
+    const int own_t = hh ? tk0 + 64 : tk0;   // the token whose P row / V row this thread writes
+    uint8_t* pdst_base = pbuf + t * Ly::PBUF + own_t * 16;
+    // own token's V half-rows in the stage: (t / sh) * sh * 256 + (t % sh) * 128, + sh * 128
+    const int vrow_off = kTile + (own_t / sh) * sh * 256 + (own_t % sh) * 128;
     float* red_t = red + t * 128;
     float* lred_t = lred + t * 64;
     uint64_t* gbar = &grp[t];
@@ -496,29 +516,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       const uint32_t par = n & 1u;
-      // ---- scores of token r
+      // ---- scores of tokens tk0 and tk0 + 64 (both halves summed)
       if (!mbar_wait(&s_full[t], par, abrt, status)) break;
       tc_fence_after();
-      float sv[16];
-      tmem_ld16(lane_addr + s_col, sv);
+      float sv0[Ly::NS], sv1[Ly::NS];
+      tmem_ld16(lane_addr + s_col, sv0);
+      tmem_ld16(lane_addr + s_col + Ly::NS, sv1);
+      if constexpr (Ly::NS == 32) {
+        tmem_ld16(lane_addr + s_col + 16, sv0 + 16);
+        tmem_ld16(lane_addr + s_col + Ly::NS + 16, sv1 + 16);
+      }
       tc_fence_before();
       mbar_arrive(&s_free[t]);
-      const bool tok_ok = r < mt.valid;
-      float s2[GT];
+      const bool ok0 = tk0 < mt.valid, ok1 = tk0 + 64 < mt.valid;
+      float sa[GT], sb[GT];
 #pragma unroll
-      for (int g = 0; g < GT; ++g) s2[g] = (tok_ok && g < G) ? sv[g] * sl2 : -INFINITY;
+      for (int g = 0; g < GT; ++g) {
+        float a = hh ? sv0[Ly::NS / 2 + g] : sv0[g];
+        float b = hh ? sv1[Ly::NS / 2 + g] : sv1[g];
+        a += __shfl_xor_sync(kFull, a, sh);
+        b += __shfl_xor_sync(kFull, b, sh);
+        sa[g] = (ok0 && g < G) ? a * sl2 : -INFINITY;
+        sb[g] = (ok1 && g < G) ? b * sl2 : -INFINITY;
+      }
       // ---- chunk max per head across the group's 128 threads
       float* rb = red_t + par * 64;
 #pragma unroll
       for (int g = 0; g < GT; ++g) {
-        float mx = s2[g];
+        float mx = fmaxf(sa[g], sb[g]);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
         if (lane == 0) rb[wq * 16 + g] = mx;
       }
       if (!group_sync(gbar, gphase, abrt, status)) break;
       float alpha[GT];
-      uint32_t col[NPV];   // P^T row r: column g = hi(p_g), column GT + g = lo(p_g)
+      uint32_t col[NPV];   // P^T row own_t: column g = hi(p_g), column GT + g = lo(p_g)
 #pragma unroll
       for (int i = 0; i < NPV; ++i) col[i] = 0;
 #pragma unroll
@@ -527,7 +559,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float mn = fmaxf(m_run[g], cm);
         // heads g >= G never see a finite score; keep them inert (alpha 0, p 0)
         alpha[g] = (mn == -INFINITY) ? 0.f : exp2f(m_run[g] - mn);
-        const float pr = (mn == -INFINITY) ? 0.f : exp2f(s2[g] - mn);
+        const float own_s = hh ? sb[g] : sa[g];
+        const float pr = (mn == -INFINITY) ? 0.f : exp2f(own_s - mn);
         m_run[g] = mn;
         l_thr[g] = fmaf(l_thr[g], alpha[g], pr);
         uint16_t hi, lo;
@@ -542,13 +575,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                        col[8 * ng + 2] | (col[8 * ng + 3] << 16),
                        col[8 * ng + 4] | (col[8 * ng + 5] << 16),
                        col[8 * ng + 6] | (col[8 * ng + 7] << 16));
-      if (!tok_ok) {
-        // rows past the chunk's valid tokens: make V finite (zero) for the MMA
-        uint8_t* vrow = smem + static_cast<size_t>(stage) * kStage + 2 * kHalf + r * 128;
+      if (own_t >= mt.valid) {
+        // past the chunk's valid tokens: make V finite (zero) for the MMA
+        uint8_t* vrow = smem + static_cast<size_t>(stage) * kStage + vrow_off;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           reinterpret_cast<uint4*>(vrow)[i] = make_uint4(0, 0, 0, 0);
-          reinterpret_cast<uint4*>(vrow + kHalf)[i] = make_uint4(0, 0, 0, 0);
+          reinterpret_cast<uint4*>(vrow + sh * 128)[i] = make_uint4(0, 0, 0, 0);
         }
       }
       fence_proxy_async_smem();
@@ -620,14 +653,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D map over a [rows, 128] 16-bit matrix, box = 64 columns x box_rows rows,
-// 128-byte swizzle; out-of-range rows read as zero.
-cudaError_t make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows,
-                     bool bf16) {
+// 2-D map over a [rows, cols] 16-bit matrix with the given row pitch, box =
+// 64 columns x box_rows rows, 128-byte swizzle; out-of-range rows read as zero.
+cudaError_t make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
+                     uint64_t row_bytes, uint32_t box_rows, bool bf16) {
   auto fn = encode_fn();
   if (fn == nullptr) return cudaErrorNotSupported;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD) * 2};
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
   cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
@@ -642,12 +675,16 @@ cudaError_t launch_t(const DecodeParams& p, int num_ctas, cudaStream_t stream) {
   using Ly = TcLayout<GT>;
   const bool bf16 = std::is_same<T, __nv_bfloat16>::value;
   CUtensorMap mk, mv, mq;
-  const uint64_t pool_rows =
-      static_cast<uint64_t>(p.num_blocks) * p.num_kv_heads * p.block_size;
-  cudaError_t e = make_map(&mk, p.k_cache, pool_rows, p.block_size, bf16);
-  if (e == cudaSuccess) e = make_map(&mv, p.v_cache, pool_rows, p.block_size, bf16);
+  // pools as [half-rows, 64]: a (block, head) tile is 2 * block_size
+  // consecutive 128-byte half-rows in its storage order, loaded as one box
+  const uint64_t half_rows =
+      static_cast<uint64_t>(p.num_blocks) * p.num_kv_heads * p.block_size * 2;
+  cudaError_t e = make_map(&mk, p.k_cache, 64, half_rows, 128, 2 * p.block_size, bf16);
+  if (e == cudaSuccess) e = make_map(&mv, p.v_cache, 64, half_rows, 128, 2 * p.block_size, bf16);
+  // q as [rows, 128]: one box per column half, NS/2 query rows
   if (e == cudaSuccess)
-    e = make_map(&mq, p.q, static_cast<uint64_t>(p.num_seqs) * p.num_q_heads, 16, bf16);
+    e = make_map(&mq, p.q, kD, static_cast<uint64_t>(p.num_seqs) * p.num_q_heads, kD * 2,
+                 Ly::NS / 2, bf16);
   if (e != cudaSuccess) return e;
   auto kern = tc_decode_kernel<T, GT>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,

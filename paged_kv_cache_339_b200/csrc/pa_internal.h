@@ -66,7 +66,7 @@ cudaError_t launch_decode_tc(const DecodeParams& p, int num_ctas,
 cudaError_t launch_write_kv(void* k_cache, void* v_cache, const void* key,
                             const void* value, const int64_t* slots,
                             int32_t num_tokens, int32_t num_kv_heads,
-                            int32_t block_size, int32_t row_bytes,
+                            int32_t block_size, int32_t row_bytes, int32_t elem_bytes,
                             int64_t num_slots, cudaStream_t stream);
 cudaError_t launch_copy_blocks(void* k_cache, void* v_cache,
                                const int64_t* pairs, int32_t num_pairs,

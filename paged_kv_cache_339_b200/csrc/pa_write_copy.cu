@@ -2,6 +2,7 @@
 //
 // write: each new token's K/V row of one KV head (head_dim elements) goes to
 //   pool[slot / BS][head][slot % BS][:]   (slot < 0: padding, skipped)
+// at the positions the in-block storage order gives (pa_common.cuh).
 // "Paged Attention: Virtual Memory for the KV Cache", "The fix borrowed from
 // operating systems": a request fills its current block, then asks for more.
 //
@@ -27,7 +28,7 @@ __global__ void __launch_bounds__(kCopyThreads)
                     const uint4* __restrict__ value,
                     const int64_t* __restrict__ slots, int32_t num_tokens,
                     int32_t num_kv_heads, int32_t block_size,
-                    int32_t row_vecs, int64_t num_slots) {
+                    int32_t row_vecs, int32_t head_dim, int64_t num_slots) {
   pdl_launch_dependents();   // the decode plan may start; it waits for us before it ends
   const int64_t per_token = static_cast<int64_t>(num_kv_heads) * row_vecs;
   const int64_t total = per_token * num_tokens;
@@ -41,7 +42,12 @@ __global__ void __launch_bounds__(kCopyThreads)
     const int64_t off = slot - blk * block_size;
     const int64_t h = r / row_vecs;
     const int64_t v = r - h * row_vecs;
-    const int64_t dst = ((blk * num_kv_heads + h) * block_size + off) * row_vecs + v;
+    // a 16-byte vector never straddles a 64-element half of the row
+    const int vec_elems = head_dim / row_vecs;
+    const int64_t in_tile =
+        tile_offset(static_cast<int>(off), static_cast<int>(v) * vec_elems, block_size, head_dim) /
+        vec_elems;
+    const int64_t dst = (blk * num_kv_heads + h) * block_size * row_vecs + in_tile;
     kc[dst] = key[idx];
     vc[dst] = value[idx];
   }
@@ -75,14 +81,14 @@ int grid_for(int64_t work) {
 cudaError_t launch_write_kv(void* k_cache, void* v_cache, const void* key,
                             const void* value, const int64_t* slots,
                             int32_t num_tokens, int32_t num_kv_heads,
-                            int32_t block_size, int32_t row_bytes,
+                            int32_t block_size, int32_t row_bytes, int32_t elem_bytes,
                             int64_t num_slots, cudaStream_t stream) {
   const int32_t row_vecs = row_bytes / 16;
   const int64_t work = static_cast<int64_t>(num_tokens) * num_kv_heads * row_vecs;
   write_kv_kernel<<<grid_for(work), kCopyThreads, 0, stream>>>(
       static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
       static_cast<const uint4*>(key), static_cast<const uint4*>(value), slots,
-      num_tokens, num_kv_heads, block_size, row_vecs, num_slots);
+      num_tokens, num_kv_heads, block_size, row_vecs, row_vecs * 16 / elem_bytes, num_slots);
   return cudaGetLastError();
 }
 

@@ -23,6 +23,16 @@ def bits(t: torch.Tensor) -> np.ndarray:
     return t.detach().contiguous().view(RAW[t.dtype]).cpu().numpy()
 
 
+def pool_f64(t: torch.Tensor) -> np.ndarray:
+    """A stored KV pool, as the oracle's logical [NB, Hkv, BS, D] fp64 view."""
+    return ORACLE.logical_pool(f64(t))
+
+
+def pool_bits(t: torch.Tensor) -> np.ndarray:
+    """A stored KV pool's bit patterns in the logical [NB, Hkv, BS, D] view."""
+    return ORACLE.logical_pool(bits(t))
+
+
 def run_step(batch, split_tokens=0, path=ops.PA_PATH_AUTO, workspace=None, write=True):
     """copy-on-write copies, new-token write, decode - the whole hot path."""
     if write:
@@ -45,7 +55,7 @@ def run_step(batch, split_tokens=0, path=ops.PA_PATH_AUTO, workspace=None, write
 
 def oracle_step(batch_cpu):
     """The same step on the CPU oracle, from host copies of the inputs."""
-    kc, vc = f64(batch_cpu.k_cache), f64(batch_cpu.v_cache)
+    kc, vc = pool_f64(batch_cpu.k_cache), pool_f64(batch_cpu.v_cache)
     if batch_cpu.cow_pairs.numel():
         kc, vc = ORACLE.copy_blocks(kc, vc, batch_cpu.cow_pairs.numpy())
     kc, vc = ORACLE.write_kv(kc, vc, f64(batch_cpu.key), f64(batch_cpu.value),
@@ -69,7 +79,7 @@ def sampled_reference(batch, seq, h):
     G = batch.num_q_heads // batch.num_kv_heads
     kv = h // G
     rows = batch.block_tables[seq, :nb].long()
-    ksub = f64(batch.k_cache[rows][:, kv:kv + 1])      # [nb, 1, BS, D]
-    vsub = f64(batch.v_cache[rows][:, kv:kv + 1])
+    ksub = pool_f64(batch.k_cache[rows][:, kv:kv + 1])      # [nb, 1, BS, D]
+    vsub = pool_f64(batch.v_cache[rows][:, kv:kv + 1])
     return ORACLE.decode_one(f64(batch.q[seq, h]), ksub, vsub, np.arange(nb), L, 0, 1,
                              float(np.float32(batch.scale)))

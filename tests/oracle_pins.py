@@ -356,6 +356,28 @@ def check_merge_partition(orc):
         assert np.allclose(orc.merge(parts), full, rtol=0, atol=1e-13), cuts
 
 
+def check_tile_layout(orc):
+    """The stored order of a (block, head) tile: every element of the logical
+    view sits at the offset the storage formula gives, the conversion is a
+    bijection, and head_dim 64 is plain row-major."""
+    r = _rng(17)
+    for BS, D in ((8, 128), (16, 128), (32, 128), (16, 64), (32, 64)):
+        NB, H = 3, 2
+        phys = r.integers(0, 1 << 30, size=(NB, H, BS, D))
+        log = orc.logical_pool(phys)
+        flat = phys.reshape(NB, H, BS * D)
+        for (b, h, t, d) in ((0, 0, 0, 0), (2, 1, BS - 1, D - 1), (1, 0, BS // 2, 63),
+                             (1, 1, min(BS - 1, 17), D // 2), (0, 1, 7, 64 % D)):
+            assert log[b, h, t, d] == flat[b, h, orc.tile_offset(t, d, BS, D)]
+        assert np.array_equal(orc.physical_pool(log), phys)
+        assert len(np.unique(log)) == len(np.unique(phys))
+    row_major = r.integers(0, 100, size=(2, 2, 16, 64))
+    assert np.array_equal(orc.logical_pool(row_major), row_major)
+    # BS 16, D 128: column 64 of token 0 is the first element of the second half
+    assert orc.tile_offset(0, 64, 16, 128) == 16 * 64
+    assert orc.tile_offset(16, 0, 32, 128) == 2 * 16 * 64
+
+
 ALL_CHECKS = [
     check_single_token, check_zero_query_mean, check_equal_keys_mean,
     check_two_token_logistic, check_golden_rational, check_argmax_limit,
@@ -363,5 +385,5 @@ ALL_CHECKS = [
     check_identity_table_is_contiguous, check_permutation_invariance,
     check_gqa_is_repeated_mha, check_context_len_bounds, check_prefix_sharing,
     check_copy_on_write, check_write_layout, check_write_then_gather,
-    check_copy_blocks, check_merge_partition,
+    check_copy_blocks, check_merge_partition, check_tile_layout,
 ]

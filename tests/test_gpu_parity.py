@@ -14,8 +14,8 @@ from oracle import ORACLE
 from paged_kv_cache_339_b200 import build as pa_build
 from paged_kv_cache_339_b200 import ops
 from paged_kv_cache_339_b200 import workloads as W
-from tests.gpu_helpers import (TOL, bits, f64, max_abs_err, oracle_step, run_step,
-                               sampled_reference)
+from tests.gpu_helpers import (TOL, bits, f64, max_abs_err, oracle_step, pool_bits,
+                               pool_f64, run_step, sampled_reference)
 
 pytestmark = pytest.mark.gpu
 
@@ -60,17 +60,17 @@ SMALL_NAMES = list(W.SMALL)
 @pytest.mark.parametrize("name", SMALL_NAMES)
 def test_write_and_copy_bit_exact(name):
     b = W.SMALL[name]("cuda")
-    kb, vb = bits(b.k_cache), bits(b.v_cache)
+    kb, vb = pool_bits(b.k_cache), pool_bits(b.v_cache)
     if b.cow_pairs.numel():
         ops.pa_copy_blocks(b.k_cache, b.v_cache, b.cow_pairs)
         kb, vb = ORACLE.copy_blocks(kb, vb, b.cow_pairs.cpu().numpy())
         torch.cuda.synchronize()
-        assert np.array_equal(bits(b.k_cache), kb) and np.array_equal(bits(b.v_cache), vb)
+        assert np.array_equal(pool_bits(b.k_cache), kb) and np.array_equal(pool_bits(b.v_cache), vb)
     ops.pa_write_kv(b.k_cache, b.v_cache, b.key, b.value, b.slot_mapping)
     torch.cuda.synchronize()
     kb, vb = ORACLE.write_kv(kb, vb, bits(b.key), bits(b.value), b.slot_mapping.cpu().numpy())
-    assert np.array_equal(bits(b.k_cache), kb)
-    assert np.array_equal(bits(b.v_cache), vb)
+    assert np.array_equal(pool_bits(b.k_cache), kb)
+    assert np.array_equal(pool_bits(b.v_cache), vb)
 
 
 def test_write_many_tokens_skips_padding_and_out_of_pool():
@@ -86,13 +86,13 @@ def test_write_many_tokens_skips_padding_and_out_of_pool():
     slots[5] = NB * BS + 3                      # outside the pool: skipped
     key = torch.randn(T, H, D, generator=g).to(torch.bfloat16)
     val = torch.randn(T, H, D, generator=g).to(torch.bfloat16)
-    kb, vb = bits(kc), bits(vc)
+    kb, vb = pool_bits(kc), pool_bits(vc)
     ops.pa_write_kv(kc, vc, key.cuda(), val.cuda(), slots.cuda())
     torch.cuda.synchronize()
     ok = slots.clone()
     ok[5] = -1
     kb, vb = ORACLE.write_kv(kb, vb, bits(key), bits(val), ok.numpy())
-    assert np.array_equal(bits(kc), kb) and np.array_equal(bits(vc), vb)
+    assert np.array_equal(pool_bits(kc), kb) and np.array_equal(pool_bits(vc), vb)
 
 
 # ---------------------------------------------------------------------------
@@ -162,7 +162,8 @@ def test_nan_in_unread_slots_does_not_leak():
         for i, L in enumerate(lens):
             for j in range(L):
                 used[bt[i, j // b.block_size], j % b.block_size] = True
-        mask = (~used).cuda()[:, None, :, None].expand_as(b.k_cache)
+        logical = (~used)[:, None, :, None].expand(b.k_cache.shape).numpy()
+        mask = torch.from_numpy(ORACLE.physical_pool(np.ascontiguousarray(logical))).cuda()
         b.k_cache[mask] = float("nan")
         b.v_cache[mask] = float("nan")
         bc = b.to("cpu")
@@ -225,8 +226,9 @@ def test_deterministic_and_split_consistent():
     o2 = run_step(b, write=False)
     assert torch.equal(o1, o2)
     bc = b.to("cpu")
-    ref = ORACLE.decode(f64(bc.q), f64(bc.k_cache), f64(bc.v_cache), bc.block_tables.numpy(),
-                        bc.context_lens.numpy(), float(np.float32(bc.scale)))
+    ref = ORACLE.decode(f64(bc.q), pool_f64(bc.k_cache), pool_f64(bc.v_cache),
+                        bc.block_tables.numpy(), bc.context_lens.numpy(),
+                        float(np.float32(bc.scale)))
     for st in (32, 256, 4096):
         assert max_abs_err(run_step(b, split_tokens=st, write=False), ref) <= 2e-3
 
@@ -294,5 +296,7 @@ def test_full_size_sampled(name):
     BS = b.block_size
     for i in seqs:
         s = int(b.slot_mapping[i])
-        assert torch.equal(b.k_cache[s // BS, :, s % BS], b.key[i])
-        assert torch.equal(b.v_cache[s // BS, :, s % BS], b.value[i])
+        kblk = pool_bits(b.k_cache[s // BS:s // BS + 1])[0]
+        vblk = pool_bits(b.v_cache[s // BS:s // BS + 1])[0]
+        assert np.array_equal(kblk[:, s % BS], bits(b.key[i]))
+        assert np.array_equal(vblk[:, s % BS], bits(b.value[i]))

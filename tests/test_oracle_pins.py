@@ -116,7 +116,21 @@ class EmptyContextNotZero(PagedAttentionOracle):
                                   max(context_len, 1), h, num_q_heads, scale)
 
 
-MUTANTS = [NoScale, NegatedScores, KeysValuesSwapped, GqaModulo,
+class TileHalvesSwapped(PagedAttentionOracle):
+    def logical_pool(self, pool):
+        NB, H, BS, D = pool.shape
+        sh, nh = min(BS, 16), D // 64
+        return (pool.reshape(NB, H, BS // sh, sh, nh, 64)
+                .transpose(0, 1, 2, 3, 4, 5).reshape(NB, H, BS, D))
+
+
+class TileGroupOf8(PagedAttentionOracle):
+    def tile_offset(self, t, d, block_size, head_dim):
+        sh, nh = min(block_size, 8), head_dim // 64
+        return ((t // sh) * nh + d // 64) * sh * 64 + (t % sh) * 64 + d % 64
+
+
+MUTANTS = [TileHalvesSwapped, TileGroupOf8, NoScale, NegatedScores, KeysValuesSwapped, GqaModulo,
            GatherIndexSwap, GatherWrongOffset, ContextOffByOne,
            NoMaxSubtraction, NoNormalisation, WriteSlotSwap, WriteKeyIntoBoth,
            WriteNegativeSlotWraps, CopyReversed, MergeWithoutRescale,
