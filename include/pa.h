@@ -63,11 +63,19 @@ typedef enum {
 } pa_status;
 
 /*
- * The two pools of one layer's cache. Both have shape
- *   [num_blocks, num_kv_heads, block_size, head_dim]
- * and element type `dtype`: slot s (token) of the pool lives in block
- * s / block_size at offset s % block_size; inside a block, each KV head's
- * block_size x head_dim tile is contiguous.
+ * The two pools of one layer's cache, each num_blocks x num_kv_heads tiles of
+ * block_size x head_dim elements of type `dtype` (the byte size of a
+ * [num_blocks, num_kv_heads, block_size, head_dim] array). Slot s (a token)
+ * lives in block s / block_size at offset s % block_size. Each (block, KV
+ * head) tile is contiguous, tile (b, h) starting at element
+ * (b * num_kv_heads + h) * block_size * head_dim. Inside a tile, rows are cut
+ * into 64-element halves and grouped 16 tokens at a time: element (t, d) of
+ * the tile sits at
+ *   ((t / SH) * NH + d / 64) * SH * 64 + (t % SH) * 64 + d % 64,
+ *   SH = min(block_size, 16), NH = head_dim / 64
+ * (plain row-major when head_dim is 64). The pages leave the inside of a block
+ * open; this order lets one copy of a tile feed the tensor cores. Write and
+ * read the pools through pa_write_kv / pa_copy_blocks / pa_decode.
  * Supported: dtype F32/F16/BF16, head_dim 64/128, block_size 8/16/32
  * (the block sizes the pages call typical: "Paged Attention as a Memory
  * Manager", "Virtual Memory as the Blueprint").

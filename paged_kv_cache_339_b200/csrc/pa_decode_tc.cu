@@ -260,8 +260,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // lane j holds entries wbase + j and wbase + 32 + j of the current item.
     // The next item of each stream is prefetched one step per emission
     // (claim -> work pair -> first table window), so item switches and table
-    // reads rarely stall the chunk issue. Two named copies keep every access a
-    // register select.
+    // reads rarely stall the chunk issue. The loop below is unrolled over the
+    // two streams so each stream's state sits in its own registers and a
+    // prefetched value is only waited for when it is used.
     struct Stream {
       int seq, kvh, split_n, tb, te, cs;   // current item, next chunk start
       int wbase, w0, w1;                   // table window of the current item
@@ -271,21 +272,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       int nw0, nw1;                        // next item's first window
       bool ended;
     };
-    Stream st0 = {};
-    st0.ended = false;
-    Stream st1 = st0;
     auto load_window = [&](int sq, int first_page, int& a, int& b) {
       const int32_t* row = p.block_tables + static_cast<size_t>(sq) * p.bt_stride;
       const int i0 = first_page + lane, i1 = first_page + 32 + lane;
       a = i0 < p.bt_stride ? row[i0] : 0;
       b = i1 < p.bt_stride ? row[i1] : 0;
     };
+    auto claim = [&]() {
+      int kr = 0;
+      if (lane == 0) kr = atomicAdd(&hdr->work_counter, 1);
+      return kr;
+    };
     // one prefetch step for the next item of stream `cur`
     auto prefetch_step = [&](Stream& cur) {
       if (cur.nst == 0) {
-        int kr = 0;
-        if (lane == 0) kr = atomicAdd(&hdr->work_counter, 1);
-        cur.nkraw = kr;
+        cur.nkraw = claim();
         cur.nst = 1;
       } else if (cur.nst == 1) {
         const int k = __shfl_sync(kFull, cur.nkraw, 0);
@@ -306,13 +307,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         cur.nst = 3;
       }
     };
+    Stream st0 = {};
+    st0.nkraw = claim();   // both streams' first claims in flight at once
+    st0.nst = 1;
+    Stream st1 = {};
+    st1.nkraw = claim();
+    st1.nst = 1;
     int stops = 0;
     uint32_t c = 0;
     bool ok = true;
-    while (true) {
-      const int t = c & 1;
-      Stream cur = t ? st1 : st0;
-      const bool other_ended = t ? st0.ended : st1.ended;
+    // emit the chunk (or END / bubble / STOP marker) at position c for stream t;
+    // returns false when the producer should stop
+    auto emit = [&](Stream& cur, const Stream& other, const int t) -> bool {
       int kind = 0;   // 0 data, 1 end, 2 bubble, 3 stop
       if (!cur.ended && cur.cs >= cur.te) {
         // current item done: finish the prefetch of the next one, then switch
@@ -333,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           cur.nst = 0;
         }
       } else if (cur.ended) {
-        kind = other_ended ? 3 : 2;
+        kind = other.ended ? 3 : 2;
       }
       int valid = 0, npg = 0, blk = 0;
       if (kind == 0) {
@@ -357,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int stage = c % kNst;
       if (!mbar_wait(&empty[stage], ((c / kNst) & 1u) ^ 1u, abrt, status)) {
         ok = false;
-        break;
+        return false;
       }
       uint8_t* st = smem + static_cast<size_t>(stage) * kStage;
       uint64_t* fb = &full[2 * stage + t];
@@ -394,10 +400,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
       }
-      if (t) st1 = cur;
-      else st0 = cur;
       ++c;
-      if (kind == 3 && ++stops == 2) break;
+      return !(kind == 3 && ++stops == 2);
+    };
+    while (emit(st0, st1, 0) && emit(st1, st0, 1)) {
     }
     if (!ok && lane == 0) {
       // copies may still be landing in the last kNst stages: let them finish
