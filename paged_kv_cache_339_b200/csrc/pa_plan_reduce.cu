@@ -42,7 +42,11 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
   __shared__ int s_split;
   __shared__ int s_maxn;
   __shared__ int s_total;
-  extern __shared__ int cell_cnt[];   // [levels][32-sequence groups]
+  // dynamic: lengths [num_seqs], splits [num_seqs], cell counts [levels][32-sequence groups]
+  extern __shared__ int s_dyn[];
+  int* s_len = s_dyn;
+  int* s_n = s_dyn + p.num_seqs;
+  int* cell_cnt = s_dyn + 2 * p.num_seqs;
 
   WsHeader* hdr = reinterpret_cast<WsHeader*>(p.ws);
   WorkPair* pairs = reinterpret_cast<WorkPair*>(p.ws + p.pairs_off);
@@ -56,6 +60,7 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
   int mx = 0, bad = 0;
   for (int i = tid; i < p.num_seqs; i += nthreads) {
     const int L = p.context_lens[i];
+    s_len[i] = L;
     if (L < 0 || L > p.max_context_len || L > cap) {
       bad = 1;
     } else {
@@ -105,10 +110,11 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
 
   // 2. splits per sequence; sequences with nothing to attend to get zero rows
   for (int i = tid; i < p.num_seqs; i += nthreads) {
-    const int L = p.context_lens[i];
+    const int L = s_len[i];
     const bool ok = !(L < 0 || L > p.max_context_len || L > cap);
     const int n = (ok && L > 0) ? (L + S - 1) / S : 0;
     nsplit[i] = n;
+    s_n[i] = n;
     if (n == 0) {
       float4* row = reinterpret_cast<float4*>(
           p.out + static_cast<size_t>(i) * p.num_q_heads * p.head_dim);
@@ -128,7 +134,7 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
   for (int cell = warp; cell < ncells; cell += nwarps) {
     const int s = cell / ngroups, g = cell - s * ngroups;
     const int i = g * 32 + lane;
-    const int n = i < p.num_seqs ? nsplit[i] : 0;
+    const int n = i < p.num_seqs ? s_n[i] : 0;
     const unsigned m = __ballot_sync(0xffffffffu, n > s);
     if (lane == 0) cell_cnt[cell] = __popc(m);
   }
@@ -151,8 +157,8 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
     const int i = g * 32 + lane;
     int n = 0, L = 0;
     if (i < p.num_seqs) {
-      n = nsplit[i];
-      L = p.context_lens[i];
+      n = s_n[i];
+      L = s_len[i];
     }
     const unsigned m = __ballot_sync(0xffffffffu, n > s);
     if (n > s) {
@@ -176,67 +182,87 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
 
 constexpr int kMergeThreads = 256;
 
+// One warp per output row (sequence, query head) for head_dim 128, one
+// half-warp per row for head_dim 64: each lane owns 4 consecutive columns.
+// The row's splits are read in batches of 8 independent 16-byte loads, and
+// the per-split weights 2^(m_p - M) / L travel between lanes by shuffle.
+template <int D>
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(MergeParams p) {
+  constexpr int VPR = D / 4;        // float4 columns per row = lanes per row
+  constexpr int RPW = 32 / VPR;     // rows per warp
   pdl_wait();   // every partial of the decode kernel is written and visible
-  extern __shared__ float s_w[];  // [G][max_splits] normalised weights
-  const int seq = blockIdx.x / p.num_kv_heads;
-  const int kvh = blockIdx.x % p.num_kv_heads;
+  const int lane = threadIdx.x & 31;
+  const int cv = lane % VPR, base = lane - cv;
+  const int total_rows = p.num_seqs * p.num_q_heads;
+  const int row = (blockIdx.x * (kMergeThreads / 32) + (threadIdx.x >> 5)) * RPW + lane / VPR;
   const int32_t* nsplit = reinterpret_cast<const int32_t*>(p.ws + p.nsplit_off);
-  const int n = nsplit[seq];
-  if (n <= 1) return;
-  const int G = p.num_q_heads / p.num_kv_heads;
-  const float2* ml = reinterpret_cast<const float2*>(p.ws + p.ml_off);
-  const float* po = reinterpret_cast<const float*>(p.ws + p.o_off);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int n = row < total_rows ? nsplit[row / p.num_q_heads] : 0;
+  int nw = n;   // loop bound shared by the rows of the warp
+#pragma unroll
+  for (int o = VPR; o < 32; o <<= 1) nw = max(nw, __shfl_xor_sync(0xffffffffu, nw, o));
+  if (nw <= 1) return;   // no split row here: the decode kernel wrote the output
 
-  for (int g = warp; g < G; g += kMergeThreads / 32) {
-    const size_t row = static_cast<size_t>(seq) * p.num_q_heads + kvh * G + g;
-    const float2* r = ml + row * p.max_splits;
-    float M = -INFINITY;
-    for (int s = lane; s < n; s += 32) M = fmaxf(M, r[s].x);
+  const size_t r = row < total_rows ? static_cast<size_t>(row) : 0;
+  const float2* ml = reinterpret_cast<const float2*>(p.ws + p.ml_off) + r * p.max_splits;
+  const float4* src = reinterpret_cast<const float4*>(p.ws + p.o_off) + r * p.max_splits * VPR + cv;
+
+  float M = -INFINITY;
+  for (int s = cv; s < nw; s += VPR)
+    if (s < n) M = fmaxf(M, ml[s].x);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float L = 0.f;
-    for (int s = lane; s < n; s += 32) L += r[s].y * exp2f(r[s].x - M);
+  for (int o = VPR / 2; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float L = 0.f;
+  for (int s = cv; s < nw; s += VPR)
+    if (s < n) {
+      const float2 e = ml[s];
+      L += e.y * exp2f(e.x - M);
+    }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    const float inv = 1.0f / L;
-    for (int s = lane; s < n; s += 32) s_w[g * p.max_splits + s] = exp2f(r[s].x - M) * inv;
+  for (int o = VPR / 2; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+  const float inv = n > 1 ? 1.0f / L : 0.f;
+
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = 0; s0 < nw; s0 += VPR) {
+    const int sl = s0 + cv;
+    const float wl = sl < n ? exp2f(ml[sl].x - M) * inv : 0.f;
+    const int jn = min(VPR, nw - s0);
+    for (int j0 = 0; j0 < jn; j0 += 8) {
+      float4 v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int sj = s0 + j0 + j;
+        v[j] = sj < n ? __ldg(src + static_cast<size_t>(sj) * VPR) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float w = __shfl_sync(0xffffffffu, wl, base + j0 + j);
+        acc.x = fmaf(w, v[j].x, acc.x);
+        acc.y = fmaf(w, v[j].y, acc.y);
+        acc.z = fmaf(w, v[j].z, acc.z);
+        acc.w = fmaf(w, v[j].w, acc.w);
+      }
+    }
   }
-  __syncthreads();
-  const int D = p.head_dim;
-  for (int idx = threadIdx.x; idx < G * D; idx += kMergeThreads) {
-    const int g = idx / D, d = idx % D;
-    const size_t row = static_cast<size_t>(seq) * p.num_q_heads + kvh * G + g;
-    const float* src = po + row * p.max_splits * D + d;
-    const float* w = s_w + g * p.max_splits;
-    float acc = 0.f;
-#pragma unroll 4
-    for (int s = 0; s < n; ++s) acc = fmaf(w[s], src[static_cast<size_t>(s) * D], acc);
-    p.out[row * D + d] = acc;
-  }
+  if (n > 1) reinterpret_cast<float4*>(p.out)[r * VPR + cv] = acc;
 }
 
 }  // namespace
 
 cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream) {
   if (p.max_splits <= 1 || p.num_seqs == 0) return cudaSuccess;
-  const int G = p.num_q_heads / p.num_kv_heads;
-  const size_t smem = static_cast<size_t>(G) * p.max_splits * sizeof(float);
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-  }
-  return launch_pdl(merge_kernel, dim3(p.num_seqs * p.num_kv_heads), dim3(kMergeThreads), smem,
-                    stream, p);
+  const int rows_per_cta = (kMergeThreads / 32) * (p.head_dim == 64 ? 2 : 1);
+  const int rows = p.num_seqs * p.num_q_heads;
+  const dim3 grid((rows + rows_per_cta - 1) / rows_per_cta);
+  if (p.head_dim == 64) return launch_pdl(merge_kernel<64>, grid, dim3(kMergeThreads), 0, stream, p);
+  if (p.head_dim == 128) return launch_pdl(merge_kernel<128>, grid, dim3(kMergeThreads), 0, stream, p);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_plan(const PlanParams& p, cudaStream_t stream) {
-  int threads = (p.num_seqs + 31) / 32 * 32;
-  threads = threads < 64 ? 64 : (threads > kPlanMaxThreads ? kPlanMaxThreads : threads);
+  // many warps even for small batches: the (level, group) cells are spread over them
+  const int threads = kPlanMaxThreads;
   const size_t cells = static_cast<size_t>(p.max_splits) * ((p.num_seqs + 31) / 32);
-  const size_t smem = cells * sizeof(int);
+  const size_t smem = (cells + 2 * static_cast<size_t>(p.num_seqs)) * sizeof(int);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
