@@ -15,15 +15,17 @@
 // Persistent, warp-specialised CTA (one per SM, ~220 KB shared memory) that
 // runs two independent item streams, so one stream's serial steps (the MMA
 // round trips, the end-of-item reduction and stores) overlap the other's:
-//   warp 0      producer: claims (sequence, split, KV head) items for the two
-//               streams and emits their 128-token chunks alternately (chunk
-//               position c belongs to stream c & 1); for each chunk it follows
-//               the block table and loads each page's K and V tile (two
-//               64-column halves each) plus the Q tile with 2-D TMA (128-byte
-//               swizzle) into a 3-stage ring; completion by mbarrier
-//               transaction count. When a stream runs out of items its
-//               positions carry END, then empty "bubble" slots, and finally a
-//               STOP for each stream.
+//   warp 11     scheduler: claims (sequence, split, KV head) items for the two
+//               streams and describes their 128-token chunks alternately (ring
+//               position c belongs to stream c & 1): metadata, query row and
+//               the physical blocks read from the block table. It runs up to
+//               8 positions ahead through a shared-memory descriptor queue.
+//               When a stream runs out of items its positions carry END, then
+//               empty "bubble" slots, and finally a STOP for each stream.
+//   warp 0      producer: for each descriptor, waits for the stage and loads
+//               each page's K and V tile (two 64-column halves each) plus the
+//               Q tile with 2-D TMA (128-byte swizzle) into a 3-stage ring;
+//               completion by mbarrier transaction count.
 //   warps 1, 2  MMA issuers (one elected lane each), one per stream: S^T into
 //               the stream's TMEM columns, then O^T once its softmax group has
 //               published P; warp 1 also allocates and frees TMEM.
@@ -53,10 +55,21 @@ constexpr int kNst = 3;       // pipeline stages
 constexpr int kTile = kChunk * 256;           // K (or V) of 128 tokens: 256 half-rows x 128 B
 constexpr int kQReg = 32 * 128;               // Q' region: up to 32 half-rows x 128 B
 constexpr int kStage = 2 * kTile + kQReg;     // K, V, Q' of one chunk
-constexpr int kThreads = 352;  // producer, 2 MMA issuers, 2 softmax groups of 4 warps
+constexpr int kQd = 8;        // chunk descriptors the scheduler may run ahead
+constexpr int kMaxPages = kChunk / 8;          // pages per chunk at the smallest block size
+constexpr int kSchedWarp = 11;
+constexpr int kThreads = 384;  // producer, 2 MMA issuers, 2 softmax groups of 4 warps, scheduler
 
 struct __align__(16) ChunkMeta {
   int32_t seq, kvh, split_raw, t0, valid, flags, pad0, pad1;
+};
+
+// One ring position as the scheduler hands it to the producer: what the
+// consumers will read (meta), the query row and the chunk's physical blocks.
+struct __align__(16) ChunkDesc {
+  ChunkMeta meta;
+  int32_t q_row, npg, pad0, pad1;
+  int32_t blk[kMaxPages];
 };
 
 template <int GT>
@@ -66,10 +79,11 @@ struct TcLayout {
   static constexpr size_t OFF_P = static_cast<size_t>(kNst) * kStage;
   static constexpr size_t OFF_BAR = OFF_P + 2 * PBUF;
   // barriers: full[3][2], empty[3]; per group: s_full, s_free, p_full,
-  // o_full, o_free, group barrier, MMA drain
-  static constexpr int NBAR = 3 * kNst + 14;
+  // o_full, o_free, group barrier, MMA drain; descriptor queue full/empty
+  static constexpr int NBAR = 3 * kNst + 14 + 2 * kQd;
   static constexpr size_t OFF_META = (OFF_BAR + NBAR * 8 + 15) / 16 * 16;  // 16-B vector stores
-  static constexpr size_t OFF_RED = (OFF_META + kNst * sizeof(ChunkMeta) + 15) / 16 * 16;
+  static constexpr size_t OFF_DESC = (OFF_META + kNst * sizeof(ChunkMeta) + 15) / 16 * 16;
+  static constexpr size_t OFF_RED = OFF_DESC + kQd * sizeof(ChunkDesc);
   static constexpr size_t OFF_LRED = OFF_RED + 2 * 2 * 4 * 16 * 4;
   static constexpr size_t OFF_MISC = OFF_LRED + 2 * 4 * 16 * 4;
   static constexpr size_t SMEM_USED = OFF_MISC + 16;
@@ -81,8 +95,8 @@ struct TcLayout {
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(kStage % 1024 == 0 && OFF_P % 1024 == 0, "swizzled tiles need 1 KB alignment");
   static_assert(OFF_BAR % 8 == 0, "mbarriers need 8-byte alignment");
-  static_assert(OFF_META % 16 == 0 && OFF_RED % 16 == 0 && OFF_LRED % 16 == 0 &&
-                    OFF_MISC % 16 == 0,
+  static_assert(OFF_META % 16 == 0 && OFF_DESC % 16 == 0 && OFF_RED % 16 == 0 &&
+                    OFF_LRED % 16 == 0 && OFF_MISC % 16 == 0,
                 "16-byte aligned shared regions");
 };
 
@@ -201,7 +215,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* o_free = o_full + 2;
   uint64_t* grp = o_free + 2;            // [2] group barriers
   uint64_t* drain = grp + 2;             // [2] MMA drain
+  uint64_t* desc_full = drain + 2;       // [kQd]
+  uint64_t* desc_empty = desc_full + kQd;  // [kQd]
   ChunkMeta* meta = reinterpret_cast<ChunkMeta*>(smem + Ly::OFF_META);
+  ChunkDesc* desc = reinterpret_cast<ChunkDesc*>(smem + Ly::OFF_DESC);
   float* red = reinterpret_cast<float*>(smem + Ly::OFF_RED);    // [2 grp][2][4][16]
   float* lred = reinterpret_cast<float*>(smem + Ly::OFF_LRED);  // [2 grp][4][16]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Ly::OFF_MISC);
@@ -226,6 +243,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&grp[b], 128);
       mbar_init(&drain[b], 1);
     }
+    for (int q = 0; q < kQd; ++q) {
+      mbar_init(&desc_full[q], 32);
+      mbar_init(&desc_empty[q], 32);
+    }
     *abrt = 0;
     fence_barrier_init();
   }
@@ -249,20 +270,90 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    // Two item streams; chunk position c belongs to stream (group) c & 1.
+    // Takes ring position c's descriptor from the scheduler, waits for the
+    // stage, and issues the chunk's copies: Q' (two boxes) and one K and one
+    // V box per page; or forwards an END / bubble / STOP marker.
     if (lane == 0) {
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
       prefetch_tmap(&tm_q);
     }
+    int stops = 0;
+    uint32_t c = 0;
+    bool ok = true;
+    for (;; ++c) {
+      const int qd = c % kQd;
+      if (!mbar_wait(&desc_full[qd], (c / kQd) & 1u, abrt, status)) {
+        ok = false;
+        break;
+      }
+      const ChunkDesc& d = desc[qd];
+      const int flags = d.meta.flags;
+      const int kvh = d.meta.kvh;
+      const int npg = d.npg;
+      const int blk = d.blk[lane & (kMaxPages - 1)];
+      uint4 m0 = make_uint4(0, 0, 0, 0), m1 = m0;
+      int q_row = 0;
+      if (lane == 0) {
+        m0 = reinterpret_cast<const uint4*>(&d.meta)[0];
+        m1 = reinterpret_cast<const uint4*>(&d.meta)[1];
+        q_row = d.q_row;
+      }
+      mbar_arrive(&desc_empty[qd]);   // every lane has its copy of the descriptor
+      const int stage = c % kNst;
+      if (!mbar_wait(&empty[stage], ((c / kNst) & 1u) ^ 1u, abrt, status)) {
+        ok = false;
+        break;
+      }
+      uint8_t* st = smem + static_cast<size_t>(stage) * kStage;
+      uint64_t* fb = &full[2 * stage + (c & 1)];
+      if (!(flags & (kEnd | kBubble | kStop))) {
+        if (lane == 0) {
+          reinterpret_cast<uint4*>(&meta[stage])[0] = m0;
+          reinterpret_cast<uint4*>(&meta[stage])[1] = m1;
+          // K and V: one box of 2*BS half-rows per page; Q': the group's query
+          // rows, first halves then second halves (NS/2 rows each)
+          mbar_arrive_expect_tx(fb, static_cast<uint32_t>(npg * BS * 512 + Ly::NS * 128));
+          tma_load_2d(st + 2 * kTile, &tm_q, 0, q_row, fb);
+          tma_load_2d(st + 2 * kTile + (Ly::NS / 2) * 128, &tm_q, 64, q_row, fb);
+        }
+        __syncwarp();
+        if (lane < npg) {
+          const int row = (blk * Hkv + kvh) * BS * 2;   // first half-row of the tile
+          const int off = lane * BS * 256;
+          tma_load_2d(st + off, &tm_k, 0, row, fb);
+          tma_load_2d(st + kTile + off, &tm_v, 0, row, fb);
+        }
+      } else {
+        if (lane == 0) {
+          meta[stage].flags = flags;
+          mbar_arrive(fb);
+        }
+        __syncwarp();
+      }
+      if ((flags & kStop) && ++stops == 2) {
+        ++c;
+        break;
+      }
+    }
+    if (!ok && lane == 0) {
+      // copies may still be landing in the last kNst stages: let them finish
+      for (uint32_t cc = c > kNst ? c - kNst : 0; cc < c; ++cc)
+        drain_wait(&full[2 * (cc % kNst) + (cc & 1)], (cc / (2 * kNst)) & 1u);
+    }
+  } else if (warp == kSchedWarp) {
+    // ------------------------------------------------------------ scheduler
+    // Two item streams; ring position c belongs to stream (group) c & 1. The
+    // scheduler claims (sequence, split, KV head) items, follows the block
+    // table and writes one descriptor per position, up to kQd positions ahead
+    // of the producer, so none of this global-memory latency sits on the copy
+    // issue path.
     const WorkPair* pairs = reinterpret_cast<const WorkPair*>(p.ws + p.pairs_off);
     // Per-stream state (warp-uniform), plus a window of block-table entries:
     // lane j holds entries wbase + j and wbase + 32 + j of the current item.
     // The next item of each stream is prefetched one step per emission
-    // (claim -> work pair -> first table window), so item switches and table
-    // reads rarely stall the chunk issue. The loop below is unrolled over the
-    // two streams so each stream's state sits in its own registers and a
-    // prefetched value is only waited for when it is used.
+    // (claim -> work pair -> first table window). The loop below is unrolled
+    // over the two streams so each stream's state sits in its own registers.
     struct Stream {
       int seq, kvh, split_n, tb, te, cs;   // current item, next chunk start
       int wbase, w0, w1;                   // table window of the current item
@@ -315,10 +406,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     st1.nst = 1;
     int stops = 0;
     uint32_t c = 0;
-    bool ok = true;
-    // emit the chunk (or END / bubble / STOP marker) at position c for stream t;
-    // returns false when the producer should stop
-    auto emit = [&](Stream& cur, const Stream& other, const int t) -> bool {
+    // describe position c for stream `cur` (a chunk, or an END / bubble /
+    // STOP marker); returns false when the scheduler should stop
+    auto emit = [&](Stream& cur, const Stream& other) -> bool {
       int kind = 0;   // 0 data, 1 end, 2 bubble, 3 stop
       if (!cur.ended && cur.cs >= cur.te) {
         // current item done: finish the prefetch of the next one, then switch
@@ -360,13 +450,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         prefetch_step(cur);   // advance the next item's prefetch by one step
       }
-      const int stage = c % kNst;
-      if (!mbar_wait(&empty[stage], ((c / kNst) & 1u) ^ 1u, abrt, status)) {
-        ok = false;
-        return false;
-      }
-      uint8_t* st = smem + static_cast<size_t>(stage) * kStage;
-      uint64_t* fb = &full[2 * stage + t];
+      const int qd = c % kQd;
+      if (!mbar_wait(&desc_empty[qd], ((c / kQd) & 1u) ^ 1u, abrt, status)) return false;
+      ChunkDesc& d = desc[qd];
       if (kind == 0) {
         if (lane == 0) {
           ChunkMeta m;
@@ -377,38 +463,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           m.valid = valid;
           m.flags = (cur.cs == cur.tb ? kFirst : 0) | (cur.cs + kChunk >= cur.te ? kLast : 0);
           m.pad0 = m.pad1 = 0;
-          meta[stage] = m;
-          // K and V: one box of 2*BS half-rows per page; Q': the group's query
-          // rows, first halves then second halves (NS/2 rows each)
-          mbar_arrive_expect_tx(fb, static_cast<uint32_t>(npg * BS * 512 + Ly::NS * 128));
-          const int q_row = cur.seq * p.num_q_heads + cur.kvh * G;
-          tma_load_2d(st + 2 * kTile, &tm_q, 0, q_row, fb);
-          tma_load_2d(st + 2 * kTile + (Ly::NS / 2) * 128, &tm_q, 64, q_row, fb);
+          d.meta = m;
+          d.q_row = cur.seq * p.num_q_heads + cur.kvh * G;
+          d.npg = npg;
         }
-        __syncwarp();
-        if (lane < npg) {
-          const int row = (blk * Hkv + cur.kvh) * BS * 2;   // first half-row of the tile
-          const int off = lane * BS * 256;
-          tma_load_2d(st + off, &tm_k, 0, row, fb);
-          tma_load_2d(st + kTile + off, &tm_v, 0, row, fb);
-        }
+        if (lane < kMaxPages) d.blk[lane] = lane < npg ? blk : 0;
         cur.cs += kChunk;
-      } else {
-        if (lane == 0) {
-          meta[stage].flags = kind == 1 ? kEnd : (kind == 2 ? kBubble : kStop);
-          mbar_arrive(fb);
-        }
-        __syncwarp();
+      } else if (lane == 0) {
+        d.meta.flags = kind == 1 ? kEnd : (kind == 2 ? kBubble : kStop);
       }
+      mbar_arrive(&desc_full[qd]);
       ++c;
       return !(kind == 3 && ++stops == 2);
     };
-    while (emit(st0, st1, 0) && emit(st1, st0, 1)) {
-    }
-    if (!ok && lane == 0) {
-      // copies may still be landing in the last kNst stages: let them finish
-      for (uint32_t cc = c > kNst ? c - kNst : 0; cc < c; ++cc)
-        drain_wait(&full[2 * (cc % kNst) + (cc & 1)], (cc / (2 * kNst)) & 1u);
+    while (emit(st0, st1) && emit(st1, st0)) {
     }
   } else if (warp == 1 || warp == 2) {
     // ------------------------------------------------------------ MMA issuers
