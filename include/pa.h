@@ -177,10 +177,8 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
  *                 time (two calls that overlap on the GPU must not share it).
  * Accumulation and softmax are fp32; the tensor-core path keeps the
  * probabilities at ~16 significant bits (two 16-bit terms).
- * PA_ERR_UNSUPPORTED also when the planning table does not fit one CTA's
- * shared memory: (max_splits * ceil(num_seqs / 32) + 2 * num_seqs) int32
- * above 227 KB, max_splits as in pa_decode_workspace_size (about 28,000
- * sequences when max_splits is 1).
+ * PA_ERR_UNSUPPORTED also for more than 56,320 sequences in one call (the
+ * planning kernel keeps the lengths in one CTA's shared memory).
  */
 pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
                     const int32_t* block_tables, int32_t bt_stride,

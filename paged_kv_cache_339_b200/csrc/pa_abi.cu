@@ -176,11 +176,8 @@ pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
     return PA_ERR_MISALIGNED;
   const WsLayout lay = ws_layout(num_seqs, num_q_heads, cache->head_dim, max_context_len, split);
   if (workspace_bytes < lay.total) return PA_ERR_WORKSPACE_TOO_SMALL;
-  // the planning kernel keeps the lengths, the split counts and one counter
-  // per (split level, 32 sequences) in shared memory
-  if ((static_cast<int64_t>(lay.max_splits) * ((num_seqs + 31) / 32) + 2 * static_cast<int64_t>(num_seqs)) * 4 >
-      227 * 1024)
-    return PA_ERR_UNSUPPORTED;
+  // the planning kernel keeps the lengths in shared memory
+  if (static_cast<int64_t>(num_seqs) * 4 > 220 * 1024) return PA_ERR_UNSUPPORTED;
 
   // the tensor-core kernel loads query tiles of 16 rows: it needs >= 16 query rows
   const bool tc_ok = tc_supported(cache->dtype, cache->head_dim, group) &&

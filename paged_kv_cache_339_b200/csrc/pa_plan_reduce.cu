@@ -1,9 +1,14 @@
 // Work planning and split-context merge for pa_decode.
 //
 // plan_kernel (one CTA) reads the context lengths, checks them, picks the
-// split size, and writes the list of (sequence, split) work pairs in
-// split-major order (every sequence's first split, then every second split,
-// ...), so the persistent decode kernels claim the longest ranges first.
+// split size S and cuts every sequence into pieces (work pairs). It lists
+// the pairs longest first (bucketed by 128-token chunk count), so the
+// persistent decode kernels, which claim pairs in list order, end on short
+// pieces and finish together. Pieces: as many whole S-token pieces as fit,
+// then the rest of the sequence. With an automatic split, when those rests
+// hold too little work to even out the CTAs' finishing times (a few long
+// sequences), each sequence's last few S-token pieces are cut into pieces
+// of about S/4 tokens instead.
 //
 // merge_kernel combines the partial softmax results of sequences that were
 // split: with per-split running max m_p (log2 units), sum l_p and
@@ -24,29 +29,52 @@ namespace pa {
 namespace {
 
 constexpr int kPlanMaxThreads = 1024;
+constexpr int kKeys = 64;   // length buckets: 1..63 chunks of 128 tokens, and >= 64 chunks
 
-__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int n = __shfl_up_sync(0xffffffffu, v, o);
-    if (lane >= o) v += n;
+__device__ __forceinline__ int piece_key(int tokens) {
+  const int k = (tokens + 127) >> 7;
+  return k < kKeys ? k : kKeys;
+}
+
+struct PieceRule {
+  int S;      // whole-piece size
+  int cut;    // 1: the last `e` whole pieces (and the rest) are cut into ~sB-token pieces
+  int e, sB, ms;
+};
+
+// Pieces of one sequence of L tokens: nA whole pieces of S tokens, then the
+// remaining L - nA*S tokens as k pieces of sb tokens (the last one shorter).
+// n = nA + k <= ms always: S >= max_context_len / ms by the workspace sizing.
+__device__ __forceinline__ void seq_pieces(int L, const PieceRule& r, int& nA, int& sb, int& k) {
+  const int nf = L / r.S;
+  if (!r.cut) {
+    nA = nf;
+    sb = L - nf * r.S;
+    k = sb > 0 ? 1 : 0;
+    return;
   }
-  return v;
+  nA = nf - min(r.e, nf);
+  const int rest = L - nA * r.S;
+  if (rest == 0) {
+    sb = 0;
+    k = 0;
+    return;
+  }
+  const int room = r.ms - nA;   // >= 1: nA * S < L <= ms * S
+  const int need = (rest + room - 1) / room;
+  sb = need > r.sB ? (need + 127) / 128 * 128 : r.sB;
+  k = (rest + sb - 1) / sb;
 }
 
 __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) {
   pdl_launch_dependents();
   __shared__ long long s_sum[32];
-  __shared__ int s_max[32];
   __shared__ int s_bad[32];
-  __shared__ int s_split;
-  __shared__ int s_maxn;
+  __shared__ int s_hist[kKeys + 1];
+  __shared__ int s_fill[kKeys + 1];
+  __shared__ PieceRule s_rule;
   __shared__ int s_total;
-  // dynamic: lengths [num_seqs], splits [num_seqs], cell counts [levels][32-sequence groups]
-  extern __shared__ int s_dyn[];
-  int* s_len = s_dyn;
-  int* s_n = s_dyn + p.num_seqs;
-  int* cell_cnt = s_dyn + 2 * p.num_seqs;
+  extern __shared__ int s_len[];   // [num_seqs]
 
   WsHeader* hdr = reinterpret_cast<WsHeader*>(p.ws);
   WorkPair* pairs = reinterpret_cast<WorkPair*>(p.ws + p.pairs_off);
@@ -54,38 +82,39 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nthreads = blockDim.x, nwarps = nthreads >> 5;
   const int64_t cap = static_cast<int64_t>(p.bt_stride) * p.block_size;
+  auto valid_len = [&](int L) { return !(L < 0 || L > p.max_context_len || L > cap); };
 
   // 1. validate lengths, total and maximum
   long long tot = 0;
-  int mx = 0, bad = 0;
+  int bad = 0;
   for (int i = tid; i < p.num_seqs; i += nthreads) {
     const int L = p.context_lens[i];
     s_len[i] = L;
-    if (L < 0 || L > p.max_context_len || L > cap) {
+    if (!valid_len(L)) {
       bad = 1;
     } else {
       tot += L;
-      mx = max(mx, L);
     }
+  }
+  for (int k = tid; k <= kKeys; k += nthreads) {
+    s_hist[k] = 0;
+    s_fill[k] = 0;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     tot += __shfl_xor_sync(0xffffffffu, tot, o);
-    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     bad |= __shfl_xor_sync(0xffffffffu, bad, o);
   }
   if (lane == 0) {
     s_sum[warp] = tot;
-    s_max[warp] = mx;
     s_bad[warp] = bad;
   }
   __syncthreads();
   if (tid == 0) {
     long long t = 0;
-    int m = 0, b = 0;
+    int b = 0;
     for (int w = 0; w < nwarps; ++w) {
       t += s_sum[w];
-      m = max(m, s_max[w]);
       b |= s_bad[w];
     }
     int S = p.split_tokens;
@@ -98,24 +127,58 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
       if (want > (1 << 30)) want = 1 << 30;
       S = static_cast<int>(want);
     }
-    s_split = S;
-    s_maxn = m > 0 ? (m + S - 1) / S : 0;
+    s_rule.S = S;
+    s_rule.cut = 0;
+    s_rule.e = 0;
+    s_rule.sB = S;
+    s_rule.ms = p.max_splits;
     hdr->status = b ? 1 /* PA_ERR_INVALID_ARG */ : 0;
     hdr->split_tokens = S;
     hdr->max_splits = p.max_splits;
   }
   __syncthreads();
-  const int S = s_split;
-  const int maxn = min(s_maxn, p.max_splits);
+  const int S = s_rule.S;
 
-  // 2. splits per sequence; sequences with nothing to attend to get zero rows
+  // 2. work in the rests (the pieces shorter than S), per KV head
+  if (p.split_tokens <= 0) {
+    long long rem = 0;
+    for (int i = tid; i < p.num_seqs; i += nthreads) {
+      const int L = s_len[i];
+      if (valid_len(L)) rem += L % S;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) rem += __shfl_xor_sync(0xffffffffu, rem, o);
+    __syncthreads();
+    if (lane == 0) s_sum[warp] = rem;
+    __syncthreads();
+    if (tid == 0) {
+      long long r = 0;
+      for (int w = 0; w < nwarps; ++w) r += s_sum[w];
+      // When the whole pieces run out, the CTAs are on average half an S-piece
+      // from their end; about that much short-piece work evens them out.
+      const long long target = static_cast<long long>(p.num_ctas) * S / (2 * p.num_kv_heads);
+      if (r < target && p.num_seqs > 0) {
+        const long long per_seq = static_cast<long long>(p.num_seqs) * S;
+        s_rule.cut = 1;
+        s_rule.e = static_cast<int>(min((target - r + per_seq - 1) / per_seq, 1LL << 20));
+        s_rule.sB = max(128, S / 4 / 128 * 128);
+      }
+    }
+    __syncthreads();
+  }
+  const PieceRule rule = s_rule;
+
+  // 3. pieces per sequence and the length histogram; sequences with nothing
+  // to attend to get zero rows
   for (int i = tid; i < p.num_seqs; i += nthreads) {
     const int L = s_len[i];
-    const bool ok = !(L < 0 || L > p.max_context_len || L > cap);
-    const int n = (ok && L > 0) ? (L + S - 1) / S : 0;
-    nsplit[i] = n;
-    s_n[i] = n;
-    if (n == 0) {
+    int nA = 0, sb = 0, k = 0;
+    if (valid_len(L) && L > 0) seq_pieces(L, rule, nA, sb, k);
+    nsplit[i] = nA + k;
+    if (nA > 0) atomicAdd(&s_hist[piece_key(S)], nA);
+    if (k > 1) atomicAdd(&s_hist[piece_key(sb)], k - 1);
+    if (k > 0) atomicAdd(&s_hist[piece_key(L - nA * S - (k - 1) * sb)], 1);
+    if (nA + k == 0) {
       float4* row = reinterpret_cast<float4*>(
           p.out + static_cast<size_t>(i) * p.num_q_heads * p.head_dim);
       const int n4 = p.num_q_heads * p.head_dim / 4;
@@ -123,57 +186,43 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
     }
   }
   __syncthreads();
-
-  // 3. split-major pair list: position of (i, s) = base_s + rank_s(i), with
-  // base_s = number of pairs at levels < s and rank_s(i) = number of
-  // sequences j < i with more than s splits. Per 32-sequence group and level,
-  // a ballot gives the group's count and each lane's rank inside the group;
-  // one scan over the (level, group) counts gives every group's base.
-  const int ngroups = (p.num_seqs + 31) / 32;
-  const int ncells = maxn * ngroups;   // (level, group) cells, level-major
-  for (int cell = warp; cell < ncells; cell += nwarps) {
-    const int s = cell / ngroups, g = cell - s * ngroups;
-    const int i = g * 32 + lane;
-    const int n = i < p.num_seqs ? s_n[i] : 0;
-    const unsigned m = __ballot_sync(0xffffffffu, n > s);
-    if (lane == 0) cell_cnt[cell] = __popc(m);
+  // 4. longest first: bucket bases in descending length order
+  if (tid == 0) {
+    int base = 0;
+    for (int k = kKeys; k >= 1; --k) {
+      s_fill[k] = base;
+      base += s_hist[k];
+    }
+    s_total = base;
   }
   __syncthreads();
-  // exclusive scan of cell_cnt (level-major) by warp 0
-  if (warp == 0) {
-    int carry = 0;
-    for (int c0 = 0; c0 < ncells; c0 += 32) {
-      const int c = c0 + lane;
-      const int v = c < ncells ? cell_cnt[c] : 0;
-      const int inc = warp_incl_scan(v, lane);
-      if (c < ncells) cell_cnt[c] = carry + inc - v;
-      carry += __shfl_sync(0xffffffffu, inc, 31);
-    }
-    if (lane == 0) s_total = carry;
-  }
-  __syncthreads();
-  for (int cell = warp; cell < ncells; cell += nwarps) {
-    const int s = cell / ngroups, g = cell - s * ngroups;
-    const int i = g * 32 + lane;
-    int n = 0, L = 0;
-    if (i < p.num_seqs) {
-      n = s_n[i];
-      L = s_len[i];
-    }
-    const unsigned m = __ballot_sync(0xffffffffu, n > s);
-    if (n > s) {
+  // 5. place every piece: a warp per sequence, a lane per piece. The order
+  // inside a bucket is whatever the atomics give; results do not depend on it
+  // (every piece's split index and token range are fixed by the sequence).
+  for (int i = warp; i < p.num_seqs; i += nwarps) {
+    const int L = s_len[i];
+    if (!valid_len(L) || L == 0) continue;
+    int nA, sb, k;
+    seq_pieces(L, rule, nA, sb, k);
+    const int n = nA + k;
+    for (int j = lane; j < n; j += 32) {
       WorkPair w;
       w.seq = i;
-      w.split_n = s | (n << 16);
-      w.t_begin = s * S;
-      w.t_end = min(L, (s + 1) * S);
-      pairs[cell_cnt[cell] + __popc(m & ((1u << lane) - 1u))] = w;
+      w.split_n = j | (n << 16);
+      if (j < nA) {
+        w.t_begin = j * S;
+        w.t_end = w.t_begin + S;
+      } else {
+        w.t_begin = nA * S + (j - nA) * sb;
+        w.t_end = min(L, w.t_begin + sb);
+      }
+      pairs[atomicAdd(&s_fill[piece_key(w.t_end - w.t_begin)], 1)] = w;
     }
   }
-  const int base = s_total;
+  __syncthreads();
   if (tid == 0) {
-    hdr->num_pairs = base;
-    hdr->num_items = base * p.num_kv_heads;
+    hdr->num_pairs = s_total;
+    hdr->num_items = s_total * p.num_kv_heads;
     hdr->work_counter = 0;
   }
   // complete only after the kernel before this one (the KV write) has
@@ -259,10 +308,9 @@ cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream) {
 }
 
 cudaError_t launch_plan(const PlanParams& p, cudaStream_t stream) {
-  // many warps even for small batches: the (level, group) cells are spread over them
+  // many warps even for small batches: a warp places one sequence's pieces
   const int threads = kPlanMaxThreads;
-  const size_t cells = static_cast<size_t>(p.max_splits) * ((p.num_seqs + 31) / 32);
-  const size_t smem = (cells + 2 * static_cast<size_t>(p.num_seqs)) * sizeof(int);
+  const size_t smem = static_cast<size_t>(p.num_seqs) * sizeof(int);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -1,0 +1,98 @@
+"""The work plan a decode call leaves in its workspace.
+
+The planning kernel cuts every sequence into pieces (work pairs) and lists
+them longest first. Whatever the cut, the pieces of a sequence must tile its
+context exactly once, carry split indices 0..n-1 with n = the recorded split
+count (at most the workspace's split capacity), and the list must be sorted
+by 128-token chunk count, longest first. Checked on the workspace after real
+calls, at full size and with explicit split sizes.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from paged_kv_cache_339_b200 import build as pa_build
+from paged_kv_cache_339_b200 import ops
+from paged_kv_cache_339_b200 import workloads as W
+from tests.gpu_helpers import run_step
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    pa_build.build()
+    ops.library()
+
+
+def _align256(x):
+    return (x + 255) // 256 * 256
+
+
+def read_plan(ws, num_seqs):
+    raw = ws.cpu().numpy()
+    hdr = raw[:256].view(np.int32)
+    status, num_items, num_pairs, split_tokens, max_splits = (int(hdr[0]), int(hdr[2]),
+                                                              int(hdr[3]), int(hdr[4]), int(hdr[5]))
+    pairs = raw[256:256 + 16 * num_pairs].view(np.int32).reshape(num_pairs, 4)
+    nsplit_off = 256 + _align256(num_seqs * max_splits * 16)
+    nsplit = raw[nsplit_off:nsplit_off + 4 * num_seqs].view(np.int32)
+    return dict(status=status, num_items=num_items, split_tokens=split_tokens,
+                max_splits=max_splits, pairs=pairs, nsplit=nsplit)
+
+
+def check_plan(plan, lens, num_kv_heads, explicit_split=0):
+    assert plan["status"] == 0
+    pairs, nsplit, ms, S = plan["pairs"], plan["nsplit"], plan["max_splits"], plan["split_tokens"]
+    assert plan["num_items"] == len(pairs) * num_kv_heads
+    if explicit_split:
+        assert S == explicit_split
+    seq, split, n, tb, te = (pairs[:, 0], pairs[:, 1] & 0xFFFF, pairs[:, 1] >> 16,
+                             pairs[:, 2], pairs[:, 3])
+    assert np.all(te > tb)
+    # longest first, by 128-token chunk count (capped at 64 chunks)
+    key = np.minimum((te - tb + 127) // 128, 64)
+    assert np.all(np.diff(key) <= 0), "pairs not sorted longest first"
+    for i, L in enumerate(lens):
+        mine = np.nonzero(seq == i)[0]
+        assert len(mine) == nsplit[i], (i, len(mine), nsplit[i])
+        if L == 0:
+            assert nsplit[i] == 0
+            continue
+        assert 1 <= nsplit[i] <= ms
+        assert np.all(n[mine] == nsplit[i])
+        order = np.argsort(split[mine])
+        assert np.array_equal(split[mine][order], np.arange(nsplit[i]))
+        b, e = tb[mine][order], te[mine][order]
+        assert b[0] == 0 and e[-1] == L and np.array_equal(b[1:], e[:-1]), f"seq {i} not tiled"
+        if explicit_split:
+            assert np.all(e - b <= explicit_split)
+            assert np.all((e - b)[:-1] == explicit_split)
+
+
+@pytest.mark.parametrize("name,split", [("gqa", 0), ("long", 0), ("mha", 0), ("prefix_cow", 0),
+                                        ("gqa", 384), ("long", 4096)])
+def test_plan_tiles_every_sequence_longest_first(name, split):
+    b = W.FULL[name]("cuda")
+    B, Hq, D = b.q.shape
+    ws = ops.decode_workspace(B, Hq, D, b.max_context_len, b.block_size, split)
+    run_step(b, split_tokens=split, workspace=ws, write=False)
+    plan = read_plan(ws, B)
+    check_plan(plan, b.context_lens.cpu().tolist(), b.num_kv_heads, split)
+
+
+def test_plan_cuts_tails_when_sequences_are_few_and_long():
+    # a few long sequences: the automatic split must leave short pieces for the
+    # end of the list, not only whole split-size pieces
+    b = W.FULL["long"]("cuda")
+    B, Hq, D = b.q.shape
+    ws = ops.decode_workspace(B, Hq, D, b.max_context_len, b.block_size)
+    run_step(b, workspace=ws, write=False)
+    plan = read_plan(ws, B)
+    sizes = plan["pairs"][:, 3] - plan["pairs"][:, 2]
+    S = plan["split_tokens"]
+    assert sizes[0] == S
+    assert np.sum(sizes <= S // 2) >= 64, "no short pieces at the end of the list"
