@@ -245,23 +245,38 @@ def time_device(step, K, W, stream, use_graph, world):
     return ms / K, launches
 
 
-def time_decode_only(b, ops, out, ws, split, path, stream, K):
-    """Average duration of the decode call alone (plan + main + merge kernels)
-    and of the main kernel share, with events around each call."""
+def time_decode_only(b, ops, out, ws, split, path, stream, K, use_graph=True):
+    """Average duration of the decode call alone (plan + main + merge kernels),
+    with events around each call; replayed from a CUDA graph like the step, so
+    host launch overhead stays out of the device time."""
     max_ctx = b.max_context_len
+
+    def call():
+        ops.pa_decode(out, b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens,
+                      max_ctx, b.scale, ws, split_tokens=split, path=path, stream=stream)
+
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(K)]
     with torch.cuda.stream(stream):
         for _ in range(3):
-            ops.pa_decode(out, b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens,
-                          max_ctx, b.scale, ws, split_tokens=split, path=path, stream=stream)
+            call()
         torch.cuda.synchronize()
+        graph = None
+        if use_graph:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=stream):
+                call()
+            graph.replay()
+            torch.cuda.synchronize()
         for a, z in ev:
             a.record(stream)
-            ops.pa_decode(out, b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens,
-                          max_ctx, b.scale, ws, split_tokens=split, path=path, stream=stream)
+            if graph is not None:
+                graph.replay()
+            else:
+                call()
             z.record(stream)
         torch.cuda.synchronize()
+    del graph
     ts = [a.elapsed_time(z) for a, z in ev]
     return statistics.median(ts), ts
 
@@ -392,7 +407,8 @@ def run_ours(args, rank, world, local):
     ms = max_over_ranks(ms, world)
     torch.cuda.synchronize()
     status = ops.pa_decode_status(ws, stream)
-    dec_ms, _ = time_decode_only(b, ops, out, ws, args.split, path, stream, max(10, args.steps))
+    dec_ms, _ = time_decode_only(b, ops, out, ws, args.split, path, stream, max(10, args.steps),
+                                 not args.no_graph)
     e2e_ms, h2d, d2h = time_e2e(b, ops, ws, args.split, path, stream, max(5, args.steps // 2), 3)
     e2e_ms = max_over_ranks(e2e_ms, world)
 
@@ -441,7 +457,8 @@ def run_ours(args, rank, world, local):
             out2 = torch.empty((B2, Hq2, D2), dtype=torch.float32, device="cuda")
             st2 = step_fn(b, ops, out2, ws2, 0, ops.PA_PATH_AUTO, stream)
             ms2, _ = time_device(st2, max(10, args.steps // 2), 3, stream, not args.no_graph, 1)
-            d2, _ = time_decode_only(b, ops, out2, ws2, 0, ops.PA_PATH_AUTO, stream, 10)
+            d2, _ = time_decode_only(b, ops, out2, ws2, 0, ops.PA_PATH_AUTO, stream, 10,
+                                     not args.no_graph)
             kb = b.kv_bytes_logical()
             sec[b.name] = {"step_gbps": round(kb / (ms2 * 1e-3) / 1e9, 1),
                            "decode_gbps": round(kb / (d2 * 1e-3) / 1e9, 1),

@@ -22,10 +22,13 @@
 //               8 positions ahead through a shared-memory descriptor queue.
 //               When a stream runs out of items its positions carry END, then
 //               empty "bubble" slots, and finally a STOP for each stream.
-//   warp 0      producer: for each descriptor, waits for the stage and loads
-//               each page's K and V tile (two 64-column halves each) plus the
-//               Q tile with 2-D TMA (128-byte swizzle) into a 3-stage ring;
-//               completion by mbarrier transaction count.
+//   warp 0      producer: for each descriptor loads each page's K and V tile
+//               (two 64-column halves each) plus the Q tile with 2-D TMA
+//               (128-byte swizzle) into a 3-stage ring; completion by mbarrier
+//               transaction count. K and Q' of a stage are refilled as soon as
+//               the score MMA has read them, V once the P.V MMA has: the score
+//               MMA and the softmax of a chunk run while its V is still in
+//               flight, and V's slot is held only for the P.V MMA.
 //   warps 1, 2  MMA issuers (one elected lane each), one per stream: S^T into
 //               the stream's TMEM columns, then O^T once its softmax group has
 //               published P; warp 1 also allocates and frees TMEM.
@@ -78,11 +81,12 @@ struct TcLayout {
   static constexpr int PBUF = (NPV / 8) * 2048;      // P^T buffer bytes (one per group)
   static constexpr size_t OFF_P = static_cast<size_t>(kNst) * kStage;
   static constexpr size_t OFF_BAR = OFF_P + 2 * PBUF;
-  // barriers: full[3][2], empty[3]; per group: s_full, s_free, p_full,
-  // o_full, o_free, group barrier, MMA drain; descriptor queue full/empty
-  static constexpr int NBAR = 3 * kNst + 14 + 2 * kQd;
+  // barriers: kfull[3][2], vfull[3][2], kempty[3], vempty[3]; per group:
+  // s_full, s_free, p_full, o_full, o_free, group barrier, MMA drain;
+  // descriptor queue full/empty
+  static constexpr int NBAR = 6 * kNst + 14 + 2 * kQd;
   static constexpr size_t OFF_META = (OFF_BAR + NBAR * 8 + 15) / 16 * 16;  // 16-B vector stores
-  static constexpr size_t OFF_DESC = (OFF_META + kNst * sizeof(ChunkMeta) + 15) / 16 * 16;
+  static constexpr size_t OFF_DESC = (OFF_META + 2 * kNst * sizeof(ChunkMeta) + 15) / 16 * 16;
   static constexpr size_t OFF_RED = OFF_DESC + kQd * sizeof(ChunkDesc);
   static constexpr size_t OFF_LRED = OFF_RED + 2 * 2 * 4 * 16 * 4;
   static constexpr size_t OFF_MISC = OFF_LRED + 2 * 4 * 16 * 4;
@@ -203,12 +207,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* pbuf = smem + Ly::OFF_P;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Ly::OFF_BAR);
-  // full[2 * stage + group]: one barrier per (stage, stream) so a stream's
-  // consumers see every phase of the barriers they wait on (the two streams
-  // alternate over an odd number of stages)
-  uint64_t* full = bars;                 // [kNst][2]
-  uint64_t* empty = bars + 2 * kNst;     // [kNst]
-  uint64_t* s_full = bars + 3 * kNst;    // [2] per group
+  // A stage holds K and Q' (released once the score MMA has read them) and V
+  // (released after the P.V MMA), each with its own full / empty barriers.
+  // kfull / vfull[2 * stage + group]: one barrier per (stage, stream) so a
+  // stream's consumers see every phase of the barriers they wait on (the two
+  // streams alternate over an odd number of stages).
+  uint64_t* kfull = bars;                // [kNst][2]
+  uint64_t* vfull = bars + 2 * kNst;     // [kNst][2]
+  uint64_t* kempty = bars + 4 * kNst;    // [kNst]
+  uint64_t* vempty = bars + 5 * kNst;    // [kNst]
+  uint64_t* s_full = bars + 6 * kNst;    // [2] per group
   uint64_t* s_free = s_full + 2;
   uint64_t* p_full = s_free + 2;
   uint64_t* o_full = p_full + 2;
@@ -217,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = grp + 2;             // [2] MMA drain
   uint64_t* desc_full = drain + 2;       // [kQd]
   uint64_t* desc_empty = desc_full + kQd;  // [kQd]
-  ChunkMeta* meta = reinterpret_cast<ChunkMeta*>(smem + Ly::OFF_META);
+  ChunkMeta* meta = reinterpret_cast<ChunkMeta*>(smem + Ly::OFF_META);   // [kNst][2]
   ChunkDesc* desc = reinterpret_cast<ChunkDesc*>(smem + Ly::OFF_DESC);
   float* red = reinterpret_cast<float*>(smem + Ly::OFF_RED);    // [2 grp][2][4][16]
   float* lred = reinterpret_cast<float*>(smem + Ly::OFF_LRED);  // [2 grp][4][16]
@@ -230,9 +238,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNst; ++s) {
-      mbar_init(&full[2 * s], 1);
-      mbar_init(&full[2 * s + 1], 1);
-      mbar_init(&empty[s], 1);
+      for (int g = 0; g < 2; ++g) {
+        mbar_init(&kfull[2 * s + g], 1);
+        mbar_init(&vfull[2 * s + g], 1);
+      }
+      mbar_init(&kempty[s], 1);
+      mbar_init(&vempty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
@@ -279,9 +290,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tm_q);
     }
     int stops = 0;
-    uint32_t c = 0;
+    uint32_t ck = 0, cv = 0;   // positions whose K / V copies (or markers) were issued
     bool ok = true;
-    for (;; ++c) {
+    for (uint32_t c = 0;; ++c) {
       const int qd = c % kQd;
       if (!mbar_wait(&desc_full[qd], (c / kQd) & 1u, abrt, status)) {
         ok = false;
@@ -301,45 +312,61 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       mbar_arrive(&desc_empty[qd]);   // every lane has its copy of the descriptor
       const int stage = c % kNst;
-      if (!mbar_wait(&empty[stage], ((c / kNst) & 1u) ^ 1u, abrt, status)) {
+      const uint32_t epar = ((c / kNst) & 1u) ^ 1u;
+      const int bi = 2 * stage + (c & 1);
+      const bool data = !(flags & (kEnd | kBubble | kStop));
+      uint8_t* st = smem + static_cast<size_t>(stage) * kStage;
+      // K and Q' (and the chunk's metadata) once the score MMA of the stage's
+      // previous chunk is done
+      if (!mbar_wait(&kempty[stage], epar, abrt, status)) {
         ok = false;
         break;
       }
-      uint8_t* st = smem + static_cast<size_t>(stage) * kStage;
-      uint64_t* fb = &full[2 * stage + (c & 1)];
-      if (!(flags & (kEnd | kBubble | kStop))) {
+      if (data) {
         if (lane == 0) {
-          reinterpret_cast<uint4*>(&meta[stage])[0] = m0;
-          reinterpret_cast<uint4*>(&meta[stage])[1] = m1;
-          // K and V: one box of 2*BS half-rows per page; Q': the group's query
-          // rows, first halves then second halves (NS/2 rows each)
-          mbar_arrive_expect_tx(fb, static_cast<uint32_t>(npg * BS * 512 + Ly::NS * 128));
-          tma_load_2d(st + 2 * kTile, &tm_q, 0, q_row, fb);
-          tma_load_2d(st + 2 * kTile + (Ly::NS / 2) * 128, &tm_q, 64, q_row, fb);
+          reinterpret_cast<uint4*>(&meta[bi])[0] = m0;
+          reinterpret_cast<uint4*>(&meta[bi])[1] = m1;
+          // K: one box of 2*BS half-rows per page; Q': the group's query rows,
+          // first halves then second halves (NS/2 rows each)
+          mbar_arrive_expect_tx(&kfull[bi], static_cast<uint32_t>(npg * BS * 256 + Ly::NS * 128));
+          tma_load_2d(st + 2 * kTile, &tm_q, 0, q_row, &kfull[bi]);
+          tma_load_2d(st + 2 * kTile + (Ly::NS / 2) * 128, &tm_q, 64, q_row, &kfull[bi]);
         }
         __syncwarp();
-        if (lane < npg) {
-          const int row = (blk * Hkv + kvh) * BS * 2;   // first half-row of the tile
-          const int off = lane * BS * 256;
-          tma_load_2d(st + off, &tm_k, 0, row, fb);
-          tma_load_2d(st + kTile + off, &tm_v, 0, row, fb);
-        }
+        if (lane < npg)
+          tma_load_2d(st + lane * BS * 256, &tm_k, 0, (blk * Hkv + kvh) * BS * 2, &kfull[bi]);
       } else {
         if (lane == 0) {
-          meta[stage].flags = flags;
-          mbar_arrive(fb);
+          meta[bi].flags = flags;
+          mbar_arrive(&kfull[bi]);
         }
         __syncwarp();
       }
-      if ((flags & kStop) && ++stops == 2) {
-        ++c;
+      ++ck;
+      // V once the P.V MMA of the stage's previous chunk is done
+      if (!mbar_wait(&vempty[stage], epar, abrt, status)) {
+        ok = false;
         break;
       }
+      if (data) {
+        if (lane == 0) mbar_arrive_expect_tx(&vfull[bi], static_cast<uint32_t>(npg * BS * 256));
+        __syncwarp();
+        if (lane < npg)
+          tma_load_2d(st + kTile + lane * BS * 256, &tm_v, 0, (blk * Hkv + kvh) * BS * 2,
+                      &vfull[bi]);
+      } else {
+        if (lane == 0) mbar_arrive(&vfull[bi]);
+        __syncwarp();
+      }
+      ++cv;
+      if ((flags & kStop) && ++stops == 2) break;
     }
     if (!ok && lane == 0) {
-      // copies may still be landing in the last kNst stages: let them finish
-      for (uint32_t cc = c > kNst ? c - kNst : 0; cc < c; ++cc)
-        drain_wait(&full[2 * (cc % kNst) + (cc & 1)], (cc / (2 * kNst)) & 1u);
+      // copies may still be landing in the last kNst positions: let them finish
+      for (uint32_t cc = ck > kNst ? ck - kNst : 0; cc < ck; ++cc)
+        drain_wait(&kfull[2 * (cc % kNst) + (cc & 1)], (cc / (2 * kNst)) & 1u);
+      for (uint32_t cc = cv > kNst ? cv - kNst : 0; cc < cv; ++cc)
+        drain_wait(&vfull[2 * (cc % kNst) + (cc & 1)], (cc / (2 * kNst)) & 1u);
     }
   } else if (warp == kSchedWarp) {
     // ------------------------------------------------------------ scheduler
@@ -494,20 +521,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t n = 0;   // data chunks of this group so far
       for (uint32_t c = t;; c += 2) {
         const int stage = c % kNst;
-        if (!mbar_wait(&full[2 * stage + t], (c / (2 * kNst)) & 1u, abrt, status)) break;
-        const ChunkMeta mt = meta[stage];
+        const uint32_t fpar = (c / (2 * kNst)) & 1u;
+        if (!mbar_wait(&kfull[2 * stage + t], fpar, abrt, status)) break;
+        const ChunkMeta mt = meta[2 * stage + t];
         if (mt.flags & kStop) break;
         const uint32_t par = n & 1u;
         if (mt.flags & kEnd) {
           // release only after the softmax group has seen END (it acknowledges
           // on p_full); a slot refilled earlier could complete the next phase of
-          // full[] before the group observed this one
+          // kfull[] before the group observed this one
           if (!mbar_wait(&p_full[t], par, abrt, status)) break;
-          mbar_arrive(&empty[stage]);
+          mbar_arrive(&kempty[stage]);
+          // V's slot only after the producer has passed this position's V half
+          // (its vfull arrival): an earlier release would complete two phases
+          // of vempty[] before the producer waits on the first
+          if (!mbar_wait(&vfull[2 * stage + t], fpar, abrt, status)) break;
+          mbar_arrive(&vempty[stage]);
           continue;
         }
         if (mt.flags & kBubble) {   // only this warp looks at bubbles
-          mbar_arrive(&empty[stage]);
+          mbar_arrive(&kempty[stage]);
+          if (!mbar_wait(&vfull[2 * stage + t], fpar, abrt, status)) break;
+          mbar_arrive(&vempty[stage]);
           continue;
         }
         // Half-row scores: the K region holds 256 half-rows (token, half) of
@@ -527,9 +562,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         mma_commit(&s_full[t]);
-        // O^T = V^T . P^T once the softmax group has written P
+        mma_commit(&kempty[stage]);   // K and Q' are free once these MMAs completed
+        // O^T = V^T . P^T once the softmax group has written P and V has landed
         if (!mbar_wait(&p_full[t], par, abrt, status)) break;
         if (!mbar_wait(&o_free[t], par ^ 1u, abrt, status)) break;
+        if (!mbar_wait(&vfull[2 * stage + t], fpar, abrt, status)) break;
         tc_fence_after();
         const int nks = (mt.valid + 15) >> 4;
         for (int ks = 0; ks < nks; ++ks) {
@@ -540,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_f16(o_tm, a, b, idesc_pv, ks > 0 ? 1u : 0u);
         }
         mma_commit(&o_full[t]);
-        mma_commit(&empty[stage]);
+        mma_commit(&vempty[stage]);
         ++n;
       }
       // all MMAs this thread issued have completed before TMEM is released
@@ -575,8 +612,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     for (uint32_t c = t;; c += 2) {
       const int stage = c % kNst;
-      if (!mbar_wait(&full[2 * stage + t], (c / (2 * kNst)) & 1u, abrt, status)) break;
-      const ChunkMeta mt = meta[stage];
+      const uint32_t fpar = (c / (2 * kNst)) & 1u;
+      if (!mbar_wait(&kfull[2 * stage + t], fpar, abrt, status)) break;
+      const ChunkMeta mt = meta[2 * stage + t];
       if (mt.flags & kEnd) {
         mbar_arrive(&p_full[t]);   // acknowledge END so the slot can be released
         break;
@@ -649,8 +687,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                        col[8 * ng + 2] | (col[8 * ng + 3] << 16),
                        col[8 * ng + 4] | (col[8 * ng + 5] << 16),
                        col[8 * ng + 6] | (col[8 * ng + 7] << 16));
-      if (own_t >= mt.valid) {
-        // past the chunk's valid tokens: make V finite (zero) for the MMA
+      if (own_t >= mt.valid && own_t < ((mt.valid + 15) & ~15)) {
+        // past the chunk's valid tokens but inside the last 16-token step of
+        // the P.V MMA: make V finite (zero) once the stage's V has landed
+        if (!mbar_wait(&vfull[2 * stage + t], fpar, abrt, status)) break;
         uint8_t* vrow = smem + static_cast<size_t>(stage) * kStage + vrow_off;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {

@@ -43,6 +43,7 @@ struct MergeParams {
   const uint8_t* ws;
   size_t nsplit_off, ml_off, o_off;
   int32_t num_seqs, num_q_heads, num_kv_heads, head_dim, max_splits;
+  int32_t merge_warps;   // set by launch_merge
 };
 
 // Both launch with programmatic stream serialisation (PDL): the kernel may be

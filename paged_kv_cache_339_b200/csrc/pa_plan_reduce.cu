@@ -231,60 +231,74 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
 
 constexpr int kMergeThreads = 256;
 
-// One warp per output row (sequence, query head) for head_dim 128, one
-// half-warp per row for head_dim 64: each lane owns 4 consecutive columns.
-// The row's splits are read in batches of 8 independent 16-byte loads, and
-// the per-split weights 2^(m_p - M) / L travel between lanes by shuffle.
+// W warps per output row (sequence, query head) for head_dim 128 (per pair of
+// rows for head_dim 64, a half-warp per row); each lane owns 4 consecutive
+// columns. Warp w of a row takes splits w, w + W, ...: its first 8 partials are
+// requested before the row's weights are known, every lane reads the (m, l)
+// pairs it needs itself (broadcast loads), and the W partial sums meet in
+// shared memory. W is chosen on the host so a warp rarely sees more than 8
+// splits.
 template <int D>
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(MergeParams p) {
   constexpr int VPR = D / 4;        // float4 columns per row = lanes per row
   constexpr int RPW = 32 / VPR;     // rows per warp
-  pdl_wait();   // every partial of the decode kernel is written and visible
-  const int lane = threadIdx.x & 31;
-  const int cv = lane % VPR, base = lane - cv;
+  constexpr int NW = kMergeThreads / 32;
+  __shared__ float4 s_acc[NW][32];
+  const int W = p.merge_warps;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int wr = warp % W, grp = warp / W;
+  const int cv = lane % VPR;
   const int total_rows = p.num_seqs * p.num_q_heads;
-  const int row = (blockIdx.x * (kMergeThreads / 32) + (threadIdx.x >> 5)) * RPW + lane / VPR;
+  const int row = (blockIdx.x * (NW / W) + grp) * RPW + lane / VPR;
   const int32_t* nsplit = reinterpret_cast<const int32_t*>(p.ws + p.nsplit_off);
+  // the split counts come from the planning kernel, complete before the
+  // decode kernel this one depends on started
   const int n = row < total_rows ? nsplit[row / p.num_q_heads] : 0;
   int nw = n;   // loop bound shared by the rows of the warp
 #pragma unroll
   for (int o = VPR; o < 32; o <<= 1) nw = max(nw, __shfl_xor_sync(0xffffffffu, nw, o));
-  if (nw <= 1) return;   // no split row here: the decode kernel wrote the output
-
-  const size_t r = row < total_rows ? static_cast<size_t>(row) : 0;
-  const float2* ml = reinterpret_cast<const float2*>(p.ws + p.ml_off) + r * p.max_splits;
-  const float4* src = reinterpret_cast<const float4*>(p.ws + p.o_off) + r * p.max_splits * VPR + cv;
-
-  float M = -INFINITY;
-  for (int s = cv; s < nw; s += VPR)
-    if (s < n) M = fmaxf(M, ml[s].x);
-#pragma unroll
-  for (int o = VPR / 2; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  float L = 0.f;
-  for (int s = cv; s < nw; s += VPR)
-    if (s < n) {
-      const float2 e = ml[s];
-      L += e.y * exp2f(e.x - M);
-    }
-#pragma unroll
-  for (int o = VPR / 2; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-  const float inv = n > 1 ? 1.0f / L : 0.f;
+  pdl_wait();   // every partial of the decode kernel is written and visible
 
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s0 = 0; s0 < nw; s0 += VPR) {
-    const int sl = s0 + cv;
-    const float wl = sl < n ? exp2f(ml[sl].x - M) * inv : 0.f;
-    const int jn = min(VPR, nw - s0);
-    for (int j0 = 0; j0 < jn; j0 += 8) {
-      float4 v[8];
+  if (nw > 1) {
+    const size_t r = static_cast<size_t>(row < total_rows ? row : 0);
+    const float2* ml = reinterpret_cast<const float2*>(p.ws + p.ml_off) + r * p.max_splits;
+    const float4* src =
+        reinterpret_cast<const float4*>(p.ws + p.o_off) + r * p.max_splits * VPR + cv;
+    float4 v[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int sj = s0 + j0 + j;
-        v[j] = sj < n ? __ldg(src + static_cast<size_t>(sj) * VPR) : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < 8; ++j) {
+      const int sj = wr + W * j;
+      v[j] = sj < n ? __ldg(src + static_cast<size_t>(sj) * VPR) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    float M = -INFINITY;
+    for (int s = cv; s < nw; s += VPR)
+      if (s < n) M = fmaxf(M, ml[s].x);
+#pragma unroll
+    for (int o = VPR / 2; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.f;
+    for (int s = cv; s < nw; s += VPR)
+      if (s < n) {
+        const float2 e = ml[s];
+        L += e.y * exp2f(e.x - M);
+      }
+#pragma unroll
+    for (int o = VPR / 2; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    const float inv = n > 1 ? 1.0f / L : 0.f;
+    for (int i0 = 0;; i0 += 8) {
+      if (i0 > 0) {
+        if (wr + W * i0 >= nw) break;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int sj = wr + W * (i0 + j);
+          v[j] = sj < n ? __ldg(src + static_cast<size_t>(sj) * VPR)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
       }
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const float w = __shfl_sync(0xffffffffu, wl, base + j0 + j);
+        const int sj = wr + W * (i0 + j);
+        const float w = sj < n ? exp2f(ml[sj].x - M) * inv : 0.f;
         acc.x = fmaf(w, v[j].x, acc.x);
         acc.y = fmaf(w, v[j].y, acc.y);
         acc.z = fmaf(w, v[j].z, acc.z);
@@ -292,14 +306,34 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(MergeParams p) {
       }
     }
   }
-  if (n > 1) reinterpret_cast<float4*>(p.out)[r * VPR + cv] = acc;
+  if (W == 1) {
+    if (n > 1) reinterpret_cast<float4*>(p.out)[static_cast<size_t>(row) * VPR + cv] = acc;
+    return;
+  }
+  s_acc[warp][lane] = acc;
+  __syncthreads();
+  if (wr == 0 && n > 1) {
+    for (int w = 1; w < W; ++w) {
+      const float4 b = s_acc[warp + w][lane];
+      acc.x += b.x;
+      acc.y += b.y;
+      acc.z += b.z;
+      acc.w += b.w;
+    }
+    reinterpret_cast<float4*>(p.out)[static_cast<size_t>(row) * VPR + cv] = acc;
+  }
 }
 
 }  // namespace
 
-cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream) {
-  if (p.max_splits <= 1 || p.num_seqs == 0) return cudaSuccess;
-  const int rows_per_cta = (kMergeThreads / 32) * (p.head_dim == 64 ? 2 : 1);
+cudaError_t launch_merge(const MergeParams& p_in, cudaStream_t stream) {
+  if (p_in.max_splits <= 1 || p_in.num_seqs == 0) return cudaSuccess;
+  MergeParams p = p_in;
+  // warps per row: about 8 splits per warp, a power of two up to 8
+  int W = 1;
+  while (W < 8 && W * 8 < p.max_splits) W *= 2;
+  p.merge_warps = W;
+  const int rows_per_cta = (kMergeThreads / 32 / W) * (p.head_dim == 64 ? 2 : 1);
   const int rows = p.num_seqs * p.num_q_heads;
   const dim3 grid((rows + rows_per_cta - 1) / rows_per_cta);
   if (p.head_dim == 64) return launch_pdl(merge_kernel<64>, grid, dim3(kMergeThreads), 0, stream, p);
