@@ -203,6 +203,7 @@ pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
   pp.ws = ws;
   pp.pairs_off = lay.pairs_off;
   pp.nsplit_off = lay.nsplit_off;
+  pp.slist_off = lay.slist_off;
   pp.num_seqs = num_seqs;
   pp.num_q_heads = num_q_heads;
   pp.num_kv_heads = cache->num_kv_heads;
@@ -245,7 +246,7 @@ pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
   MergeParams mp;
   mp.out = out;
   mp.ws = ws;
-  mp.nsplit_off = lay.nsplit_off;
+  mp.slist_off = lay.slist_off;
   mp.ml_off = lay.ml_off;
   mp.o_off = lay.o_off;
   mp.num_seqs = num_seqs;

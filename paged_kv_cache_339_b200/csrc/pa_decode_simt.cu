@@ -152,9 +152,15 @@ __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
     while (k < num_items) {
       const int pi = k / Hkv, kvh = k - pi * Hkv;
       const WorkPair wp = pairs[pi];
-      if (lane == 0) kraw = atomicAdd(&hdr->work_counter, 1);  // next claim in flight
       const int32_t* bt_row = p.block_tables + static_cast<size_t>(wp.seq) * p.bt_stride;
+      bool claimed = false;
       for (int cs = wp.t_begin; cs < wp.t_end; cs += CHUNK) {
+        // next claim in flight two chunks before this item ends (a claim held
+        // for a whole item would lengthen the tail)
+        if (!claimed && wp.t_end - cs <= 2 * CHUNK) {
+          if (lane == 0) kraw = atomicAdd(&hdr->work_counter, 1);
+          claimed = true;
+        }
         const int valid = min(CHUNK, wp.t_end - cs);
         const int npg = (valid + BS - 1) / BS;
         int blk = 0;
@@ -210,6 +216,7 @@ __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
         ++c;
       }
       if (!ok) break;
+      if (!claimed && lane == 0) kraw = atomicAdd(&hdr->work_counter, 1);
       k = __shfl_sync(kFull, kraw, 0);
     }
     if (ok) {

@@ -379,8 +379,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Per-stream state (warp-uniform), plus a window of block-table entries:
     // lane j holds entries wbase + j and wbase + 32 + j of the current item.
     // The next item of each stream is prefetched one step per emission
-    // (claim -> work pair -> first table window). The loop below is unrolled
-    // over the two streams so each stream's state sits in its own registers.
+    // (claim -> work pair -> first table window), starting three chunks
+    // before the current item ends. The loop below is unrolled over the two
+    // streams so each stream's state sits in its own registers.
     struct Stream {
       int seq, kvh, split_n, tb, te, cs;   // current item, next chunk start
       int wbase, w0, w1;                   // table window of the current item
@@ -475,7 +476,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           atomicCAS(status, 0, 1 /* PA_ERR_INVALID_ARG */);
           blk = 0;
         }
-        prefetch_step(cur);   // advance the next item's prefetch by one step
+        // advance the next item's prefetch by one step; the claim itself waits
+        // until the current item has at most 3 chunks left, so a stream never
+        // holds an unstarted item for long (it would lengthen the tail)
+        if (cur.nst != 0 || cur.te - cur.cs <= 3 * kChunk) prefetch_step(cur);
       }
       const int qd = c % kQd;
       if (!mbar_wait(&desc_empty[qd], ((c / kQd) & 1u) ^ 1u, abrt, status)) return false;

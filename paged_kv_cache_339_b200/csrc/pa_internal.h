@@ -13,7 +13,7 @@ struct PlanParams {
   const int32_t* context_lens;
   float* out;
   uint8_t* ws;
-  size_t pairs_off, nsplit_off;
+  size_t pairs_off, nsplit_off, slist_off;
   int32_t num_seqs, num_q_heads, num_kv_heads, head_dim;
   int32_t bt_stride, block_size, max_context_len;
   int32_t split_tokens;   // explicit split, or 0 = choose on the device
@@ -41,9 +41,8 @@ struct DecodeParams {
 struct MergeParams {
   float* out;
   const uint8_t* ws;
-  size_t nsplit_off, ml_off, o_off;
+  size_t slist_off, ml_off, o_off;
   int32_t num_seqs, num_q_heads, num_kv_heads, head_dim, max_splits;
-  int32_t merge_warps;   // set by launch_merge
 };
 
 // Both launch with programmatic stream serialisation (PDL): the kernel may be

@@ -73,18 +73,19 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
   __shared__ int s_hist[kKeys + 1];
   __shared__ int s_fill[kKeys + 1];
   __shared__ PieceRule s_rule;
-  __shared__ int s_total;
+  __shared__ int s_nsl, s_maxn;
   extern __shared__ int s_len[];   // [num_seqs]
 
   WsHeader* hdr = reinterpret_cast<WsHeader*>(p.ws);
   WorkPair* pairs = reinterpret_cast<WorkPair*>(p.ws + p.pairs_off);
   int32_t* nsplit = reinterpret_cast<int32_t*>(p.ws + p.nsplit_off);
+  int2* slist = reinterpret_cast<int2*>(p.ws + p.slist_off);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nthreads = blockDim.x, nwarps = nthreads >> 5;
   const int64_t cap = static_cast<int64_t>(p.bt_stride) * p.block_size;
   auto valid_len = [&](int L) { return !(L < 0 || L > p.max_context_len || L > cap); };
 
-  // 1. validate lengths, total and maximum
+  // 1. validate lengths; total
   long long tot = 0;
   int bad = 0;
   for (int i = tid; i < p.num_seqs; i += nthreads) {
@@ -96,9 +97,10 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
       tot += L;
     }
   }
-  for (int k = tid; k <= kKeys; k += nthreads) {
-    s_hist[k] = 0;
-    s_fill[k] = 0;
+  for (int k = tid; k <= kKeys; k += nthreads) s_hist[k] = 0;
+  if (tid == 0) {
+    s_nsl = 0;
+    s_maxn = 0;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -110,31 +112,34 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
     s_bad[warp] = bad;
   }
   __syncthreads();
-  if (tid == 0) {
-    long long t = 0;
-    int b = 0;
-    for (int w = 0; w < nwarps; ++w) {
-      t += s_sum[w];
-      b |= s_bad[w];
+  if (warp == 0) {
+    long long t = lane < nwarps ? s_sum[lane] : 0;
+    int b = lane < nwarps ? s_bad[lane] : 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      t += __shfl_xor_sync(0xffffffffu, t, o);
+      b |= __shfl_xor_sync(0xffffffffu, b, o);
     }
-    int S = p.split_tokens;
-    if (S <= 0) {
-      // Aim for ~items_per_cta work items per persistent CTA.
-      long long per_cta = (t * p.num_kv_heads + p.num_ctas - 1) / p.num_ctas;
-      long long want = (per_cta + p.items_per_cta - 1) / p.items_per_cta;
-      want = (want + kAutoSplitQuantum - 1) / kAutoSplitQuantum * kAutoSplitQuantum;
-      if (want < p.min_split) want = p.min_split;
-      if (want > (1 << 30)) want = 1 << 30;
-      S = static_cast<int>(want);
+    if (lane == 0) {
+      int S = p.split_tokens;
+      if (S <= 0) {
+        // Aim for ~items_per_cta work items per persistent CTA.
+        long long per_cta = (t * p.num_kv_heads + p.num_ctas - 1) / p.num_ctas;
+        long long want = (per_cta + p.items_per_cta - 1) / p.items_per_cta;
+        want = (want + kAutoSplitQuantum - 1) / kAutoSplitQuantum * kAutoSplitQuantum;
+        if (want < p.min_split) want = p.min_split;
+        if (want > (1 << 30)) want = 1 << 30;
+        S = static_cast<int>(want);
+      }
+      s_rule.S = S;
+      s_rule.cut = 0;
+      s_rule.e = 0;
+      s_rule.sB = S;
+      s_rule.ms = p.max_splits;
+      hdr->status = b ? 1 /* PA_ERR_INVALID_ARG */ : 0;
+      hdr->split_tokens = S;
+      hdr->max_splits = p.max_splits;
     }
-    s_rule.S = S;
-    s_rule.cut = 0;
-    s_rule.e = 0;
-    s_rule.sB = S;
-    s_rule.ms = p.max_splits;
-    hdr->status = b ? 1 /* PA_ERR_INVALID_ARG */ : 0;
-    hdr->split_tokens = S;
-    hdr->max_splits = p.max_splits;
   }
   __syncthreads();
   const int S = s_rule.S;
@@ -148,16 +153,17 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) rem += __shfl_xor_sync(0xffffffffu, rem, o);
-    __syncthreads();
     if (lane == 0) s_sum[warp] = rem;
     __syncthreads();
-    if (tid == 0) {
-      long long r = 0;
-      for (int w = 0; w < nwarps; ++w) r += s_sum[w];
-      // When the whole pieces run out, the CTAs are on average half an S-piece
-      // from their end; about that much short-piece work evens them out.
+    if (warp == 0) {
+      long long r = lane < nwarps ? s_sum[lane] : 0;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
+      // When the whole pieces run out, the CTAs are on average half an
+      // S-piece from their end; about that much short-piece work evens them
+      // out.
       const long long target = static_cast<long long>(p.num_ctas) * S / (2 * p.num_kv_heads);
-      if (r < target && p.num_seqs > 0) {
+      if (lane == 0 && r < target && p.num_seqs > 0) {
         const long long per_seq = static_cast<long long>(p.num_seqs) * S;
         s_rule.cut = 1;
         s_rule.e = static_cast<int>(min((target - r + per_seq - 1) / per_seq, 1LL << 20));
@@ -168,17 +174,24 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
   }
   const PieceRule rule = s_rule;
 
-  // 3. pieces per sequence and the length histogram; sequences with nothing
+  // 3. pieces per sequence (a thread per sequence): split counts, the list of
+  // split sequences for the merge, and the length histogram (a sequence's
+  // pieces form at most three runs of equal length); sequences with nothing
   // to attend to get zero rows
   for (int i = tid; i < p.num_seqs; i += nthreads) {
     const int L = s_len[i];
     int nA = 0, sb = 0, k = 0;
     if (valid_len(L) && L > 0) seq_pieces(L, rule, nA, sb, k);
-    nsplit[i] = nA + k;
+    const int n = nA + k;
+    nsplit[i] = n;
+    if (n > 1) {
+      slist[atomicAdd(&s_nsl, 1)] = make_int2(i, n);
+      atomicMax(&s_maxn, n);
+    }
     if (nA > 0) atomicAdd(&s_hist[piece_key(S)], nA);
     if (k > 1) atomicAdd(&s_hist[piece_key(sb)], k - 1);
     if (k > 0) atomicAdd(&s_hist[piece_key(L - nA * S - (k - 1) * sb)], 1);
-    if (nA + k == 0) {
+    if (n == 0) {
       float4* row = reinterpret_cast<float4*>(
           p.out + static_cast<size_t>(i) * p.num_q_heads * p.head_dim);
       const int n4 = p.num_q_heads * p.head_dim / 4;
@@ -186,44 +199,65 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
     }
   }
   __syncthreads();
-  // 4. longest first: bucket bases in descending length order
-  if (tid == 0) {
-    int base = 0;
-    for (int k = kKeys; k >= 1; --k) {
-      s_fill[k] = base;
-      base += s_hist[k];
+  // 4. longest first: bucket bases in descending length order (warp 0 scans
+  // the kKeys buckets, two per lane)
+  if (warp == 0) {
+    const int k0 = kKeys - 2 * lane, k1 = k0 - 1;   // descending keys
+    const int h0 = s_hist[k0], h1 = k1 >= 1 ? s_hist[k1] : 0;
+    int inc = h0 + h1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += n;
     }
-    s_total = base;
+    const int excl = inc - h0 - h1;
+    s_fill[k0] = excl;
+    if (k1 >= 1) s_fill[k1] = excl + h0;
+    if (lane == 31) {
+      hdr->num_pairs = inc;
+      hdr->num_items = inc * p.num_kv_heads;
+      hdr->work_counter = 0;
+      hdr->num_split_seqs = s_nsl;
+      hdr->max_nsplit = s_maxn;
+    }
   }
   __syncthreads();
-  // 5. place every piece: a warp per sequence, a lane per piece. The order
-  // inside a bucket is whatever the atomics give; results do not depend on it
-  // (every piece's split index and token range are fixed by the sequence).
-  for (int i = warp; i < p.num_seqs; i += nwarps) {
+  // 5. place every piece: a thread per sequence reserves each run's slots
+  // with one atomic. The order inside a bucket is whatever the atomics give;
+  // results do not depend on it (every piece's split index and token range
+  // are fixed by the sequence).
+  for (int i = tid; i < p.num_seqs; i += nthreads) {
     const int L = s_len[i];
     if (!valid_len(L) || L == 0) continue;
     int nA, sb, k;
     seq_pieces(L, rule, nA, sb, k);
     const int n = nA + k;
-    for (int j = lane; j < n; j += 32) {
-      WorkPair w;
-      w.seq = i;
-      w.split_n = j | (n << 16);
-      if (j < nA) {
+    WorkPair w;
+    w.seq = i;
+    if (nA > 0) {
+      const int pos = atomicAdd(&s_fill[piece_key(S)], nA);
+      for (int j = 0; j < nA; ++j) {
+        w.split_n = j | (n << 16);
         w.t_begin = j * S;
         w.t_end = w.t_begin + S;
-      } else {
-        w.t_begin = nA * S + (j - nA) * sb;
-        w.t_end = min(L, w.t_begin + sb);
+        pairs[pos + j] = w;
       }
-      pairs[atomicAdd(&s_fill[piece_key(w.t_end - w.t_begin)], 1)] = w;
     }
-  }
-  __syncthreads();
-  if (tid == 0) {
-    hdr->num_pairs = s_total;
-    hdr->num_items = s_total * p.num_kv_heads;
-    hdr->work_counter = 0;
+    if (k > 1) {
+      const int pos = atomicAdd(&s_fill[piece_key(sb)], k - 1);
+      for (int q = 0; q < k - 1; ++q) {
+        w.split_n = (nA + q) | (n << 16);
+        w.t_begin = nA * S + q * sb;
+        w.t_end = w.t_begin + sb;
+        pairs[pos + q] = w;
+      }
+    }
+    if (k > 0) {
+      w.split_n = (n - 1) | (n << 16);
+      w.t_begin = nA * S + (k - 1) * sb;
+      w.t_end = L;
+      pairs[atomicAdd(&s_fill[piece_key(L - w.t_begin)], 1)] = w;
+    }
   }
   // complete only after the kernel before this one (the KV write) has
   pdl_wait();
@@ -231,119 +265,134 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
 
 constexpr int kMergeThreads = 256;
 
-// W warps per output row (sequence, query head) for head_dim 128 (per pair of
-// rows for head_dim 64, a half-warp per row); each lane owns 4 consecutive
-// columns. Warp w of a row takes splits w, w + W, ...: its first 8 partials are
-// requested before the row's weights are known, every lane reads the (m, l)
-// pairs it needs itself (broadcast loads), and the W partial sums meet in
-// shared memory. W is chosen on the host so a warp rarely sees more than 8
-// splits.
+// Rows (sequence, query head) of the split sequences only, from the list the
+// planning kernel wrote. W warps per row for head_dim 128 (per pair of rows
+// for head_dim 64, a half-warp per row); each lane owns 4 consecutive
+// columns. Warp w of a row takes splits w, w + W, ...: its first 8 partials
+// are requested before the row's weights are known, every lane reads the
+// (m, l) pairs it needs itself (broadcast loads), and the W partial sums meet
+// in shared memory. W (a power of two up to 8) is picked from the largest
+// split count so a warp rarely sees more than 8 splits.
 template <int D>
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(MergeParams p) {
   constexpr int VPR = D / 4;        // float4 columns per row = lanes per row
   constexpr int RPW = 32 / VPR;     // rows per warp
   constexpr int NW = kMergeThreads / 32;
   __shared__ float4 s_acc[NW][32];
-  const int W = p.merge_warps;
+  const WsHeader* hdr = reinterpret_cast<const WsHeader*>(p.ws);
+  const int2* slist = reinterpret_cast<const int2*>(p.ws + p.slist_off);
+  const float2* ml_all = reinterpret_cast<const float2*>(p.ws + p.ml_off);
+  const float4* po_all = reinterpret_cast<const float4*>(p.ws + p.o_off);
+  float4* out4 = reinterpret_cast<float4*>(p.out);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int wr = warp % W, grp = warp / W;
   const int cv = lane % VPR;
-  const int total_rows = p.num_seqs * p.num_q_heads;
-  const int row = (blockIdx.x * (NW / W) + grp) * RPW + lane / VPR;
-  const int32_t* nsplit = reinterpret_cast<const int32_t*>(p.ws + p.nsplit_off);
-  // the split counts come from the planning kernel, complete before the
-  // decode kernel this one depends on started
-  const int n = row < total_rows ? nsplit[row / p.num_q_heads] : 0;
-  int nw = n;   // loop bound shared by the rows of the warp
-#pragma unroll
-  for (int o = VPR; o < 32; o <<= 1) nw = max(nw, __shfl_xor_sync(0xffffffffu, nw, o));
   pdl_wait();   // every partial of the decode kernel is written and visible
 
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (nw > 1) {
-    const size_t r = static_cast<size_t>(row < total_rows ? row : 0);
-    const float2* ml = reinterpret_cast<const float2*>(p.ws + p.ml_off) + r * p.max_splits;
-    const float4* src =
-        reinterpret_cast<const float4*>(p.ws + p.o_off) + r * p.max_splits * VPR + cv;
-    float4 v[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int sj = wr + W * j;
-      v[j] = sj < n ? __ldg(src + static_cast<size_t>(sj) * VPR) : make_float4(0.f, 0.f, 0.f, 0.f);
+  const int Hq = p.num_q_heads;
+  const int total_rows = hdr->num_split_seqs * Hq;
+  const int maxn = hdr->max_nsplit;
+  int W = 1;
+  while (W < 8 && W * 8 < maxn) W *= 2;
+  const int wr = warp % W, grp = warp / W;
+  const int rows_per_cta = (NW / W) * RPW;
+  // a grid of a few CTAs per SM walks all row groups
+  for (int rbase = blockIdx.x * rows_per_cta; rbase < total_rows;
+       rbase += gridDim.x * rows_per_cta) {
+    const int lr = rbase + grp * RPW + lane / VPR;   // row of the split list
+    int n = 0;
+    size_t row = 0;
+    if (lr < total_rows) {
+      const int2 e = slist[lr / Hq];
+      n = e.y;
+      row = static_cast<size_t>(e.x) * Hq + lr % Hq;
     }
-    float M = -INFINITY;
-    for (int s = cv; s < nw; s += VPR)
-      if (s < n) M = fmaxf(M, ml[s].x);
+    int nw = n;   // loop bound shared by the rows of the warp
 #pragma unroll
-    for (int o = VPR / 2; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float L = 0.f;
-    for (int s = cv; s < nw; s += VPR)
-      if (s < n) {
-        const float2 e = ml[s];
-        L += e.y * exp2f(e.x - M);
+    for (int o = VPR; o < 32; o <<= 1) nw = max(nw, __shfl_xor_sync(0xffffffffu, nw, o));
+
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (nw > 1) {
+      const float2* ml = ml_all + row * p.max_splits;
+      const float4* src = po_all + row * p.max_splits * VPR + cv;
+      float4 v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int sj = wr + W * j;
+        v[j] = sj < n ? __ldg(src + static_cast<size_t>(sj) * VPR)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
       }
+      float M = -INFINITY;
+      for (int s = cv; s < nw; s += VPR)
+        if (s < n) M = fmaxf(M, ml[s].x);
 #pragma unroll
-    for (int o = VPR / 2; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    const float inv = n > 1 ? 1.0f / L : 0.f;
-    for (int i0 = 0;; i0 += 8) {
-      if (i0 > 0) {
-        if (wr + W * i0 >= nw) break;
+      for (int o = VPR / 2; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+      float L = 0.f;
+      for (int s = cv; s < nw; s += VPR)
+        if (s < n) {
+          const float2 e = ml[s];
+          L += e.y * exp2f(e.x - M);
+        }
+#pragma unroll
+      for (int o = VPR / 2; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+      const float inv = n > 1 ? 1.0f / L : 0.f;
+      for (int i0 = 0;; i0 += 8) {
+        if (i0 > 0) {
+          if (wr + W * i0 >= nw) break;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int sj = wr + W * (i0 + j);
+            v[j] = sj < n ? __ldg(src + static_cast<size_t>(sj) * VPR)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int sj = wr + W * (i0 + j);
-          v[j] = sj < n ? __ldg(src + static_cast<size_t>(sj) * VPR)
-                        : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float w = sj < n ? exp2f(ml[sj].x - M) * inv : 0.f;
+          acc.x = fmaf(w, v[j].x, acc.x);
+          acc.y = fmaf(w, v[j].y, acc.y);
+          acc.z = fmaf(w, v[j].z, acc.z);
+          acc.w = fmaf(w, v[j].w, acc.w);
         }
       }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int sj = wr + W * (i0 + j);
-        const float w = sj < n ? exp2f(ml[sj].x - M) * inv : 0.f;
-        acc.x = fmaf(w, v[j].x, acc.x);
-        acc.y = fmaf(w, v[j].y, acc.y);
-        acc.z = fmaf(w, v[j].z, acc.z);
-        acc.w = fmaf(w, v[j].w, acc.w);
+    }
+    if (W == 1) {
+      if (n > 1) out4[row * VPR + cv] = acc;
+      continue;
+    }
+    s_acc[warp][lane] = acc;
+    __syncthreads();
+    if (wr == 0 && n > 1) {
+      for (int w = 1; w < W; ++w) {
+        const float4 b = s_acc[warp + w][lane];
+        acc.x += b.x;
+        acc.y += b.y;
+        acc.z += b.z;
+        acc.w += b.w;
       }
+      out4[row * VPR + cv] = acc;
     }
-  }
-  if (W == 1) {
-    if (n > 1) reinterpret_cast<float4*>(p.out)[static_cast<size_t>(row) * VPR + cv] = acc;
-    return;
-  }
-  s_acc[warp][lane] = acc;
-  __syncthreads();
-  if (wr == 0 && n > 1) {
-    for (int w = 1; w < W; ++w) {
-      const float4 b = s_acc[warp + w][lane];
-      acc.x += b.x;
-      acc.y += b.y;
-      acc.z += b.z;
-      acc.w += b.w;
-    }
-    reinterpret_cast<float4*>(p.out)[static_cast<size_t>(row) * VPR + cv] = acc;
+    __syncthreads();   // s_acc is reused by the next row group
   }
 }
 
 }  // namespace
 
-cudaError_t launch_merge(const MergeParams& p_in, cudaStream_t stream) {
-  if (p_in.max_splits <= 1 || p_in.num_seqs == 0) return cudaSuccess;
-  MergeParams p = p_in;
-  // warps per row: about 8 splits per warp, a power of two up to 8
-  int W = 1;
-  while (W < 8 && W * 8 < p.max_splits) W *= 2;
-  p.merge_warps = W;
-  const int rows_per_cta = (kMergeThreads / 32 / W) * (p.head_dim == 64 ? 2 : 1);
+cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream) {
+  if (p.max_splits <= 1 || p.num_seqs == 0) return cudaSuccess;
+  // at most 4 CTAs per SM: they fit beside a decode CTA, so all of them are
+  // resident (and past their launch) when the decode kernel finishes
   const int rows = p.num_seqs * p.num_q_heads;
-  const dim3 grid((rows + rows_per_cta - 1) / rows_per_cta);
+  const dim3 grid(rows < 4 * num_sms() ? rows : 4 * num_sms());
   if (p.head_dim == 64) return launch_pdl(merge_kernel<64>, grid, dim3(kMergeThreads), 0, stream, p);
   if (p.head_dim == 128) return launch_pdl(merge_kernel<128>, grid, dim3(kMergeThreads), 0, stream, p);
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_plan(const PlanParams& p, cudaStream_t stream) {
-  // many warps even for small batches: a warp places one sequence's pieces
-  const int threads = kPlanMaxThreads;
+  // a thread per sequence
+  int threads = (p.num_seqs + 31) / 32 * 32;
+  threads = threads < 128 ? 128 : (threads > kPlanMaxThreads ? kPlanMaxThreads : threads);
   const size_t smem = static_cast<size_t>(p.num_seqs) * sizeof(int);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
   if (smem > 48 * 1024) {

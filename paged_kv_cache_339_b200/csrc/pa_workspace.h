@@ -1,7 +1,8 @@
 // Layout of the caller-provided decode workspace (shared by host and device
 // code). All offsets are multiples of 256 bytes from the workspace start.
 //
-//   [header 256 B][work pairs][splits per sequence][partial (m, l)][partial o]
+//   [header 256 B][work pairs][splits per sequence][split-sequence list]
+//   [partial (m, l)][partial o]
 //
 // The header holds the device status word (first 4 bytes), the work counter
 // the persistent decode kernels claim items from, and the plan the planning
@@ -21,7 +22,9 @@ struct WsHeader {
   int32_t num_pairs;     // (sequence, split) pairs
   int32_t split_tokens;  // tokens per split chosen for this call
   int32_t max_splits;    // split capacity per sequence in this workspace
-  int32_t reserved[58];
+  int32_t num_split_seqs;  // sequences cut into more than one piece (merge list length)
+  int32_t max_nsplit;      // largest piece count of a sequence
+  int32_t reserved[56];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
@@ -49,7 +52,7 @@ inline int32_t auto_min_split(int32_t max_ctx) {
 
 struct WsLayout {
   int32_t max_splits;
-  size_t pairs_off, nsplit_off, ml_off, o_off, total;
+  size_t pairs_off, nsplit_off, slist_off, ml_off, o_off, total;
 };
 
 inline WsLayout ws_layout(int32_t num_seqs, int32_t num_q_heads,
@@ -68,6 +71,8 @@ inline WsLayout ws_layout(int32_t num_seqs, int32_t num_q_heads,
   off += align256(B * ms * 16);
   w.nsplit_off = off;
   off += align256(B * 4);
+  w.slist_off = off;   // (sequence, pieces) of every split sequence
+  off += align256(B * 8);
   w.ml_off = off;
   off += align256(B * H * ms * 8);
   w.o_off = off;

@@ -40,8 +40,12 @@ def read_plan(ws, num_seqs):
     pairs = raw[256:256 + 16 * num_pairs].view(np.int32).reshape(num_pairs, 4)
     nsplit_off = 256 + _align256(num_seqs * max_splits * 16)
     nsplit = raw[nsplit_off:nsplit_off + 4 * num_seqs].view(np.int32)
+    num_split_seqs, max_nsplit = int(hdr[6]), int(hdr[7])
+    slist_off = nsplit_off + _align256(num_seqs * 4)
+    slist = raw[slist_off:slist_off + 8 * num_split_seqs].view(np.int32).reshape(-1, 2)
     return dict(status=status, num_items=num_items, split_tokens=split_tokens,
-                max_splits=max_splits, pairs=pairs, nsplit=nsplit)
+                max_splits=max_splits, pairs=pairs, nsplit=nsplit, slist=slist,
+                max_nsplit=max_nsplit)
 
 
 def check_plan(plan, lens, num_kv_heads, explicit_split=0):
@@ -50,7 +54,7 @@ def check_plan(plan, lens, num_kv_heads, explicit_split=0):
     assert plan["num_items"] == len(pairs) * num_kv_heads
     if explicit_split:
         assert S == explicit_split
-    seq, split, n, tb, te = (pairs[:, 0], pairs[:, 1] & 0xFFFF, pairs[:, 1] >> 16,
+    seq, splitix, n, tb, te = (pairs[:, 0], pairs[:, 1] & 0xFFFF, pairs[:, 1] >> 16,
                              pairs[:, 2], pairs[:, 3])
     assert np.all(te > tb)
     # longest first, by 128-token chunk count (capped at 64 chunks)
@@ -64,13 +68,18 @@ def check_plan(plan, lens, num_kv_heads, explicit_split=0):
             continue
         assert 1 <= nsplit[i] <= ms
         assert np.all(n[mine] == nsplit[i])
-        order = np.argsort(split[mine])
-        assert np.array_equal(split[mine][order], np.arange(nsplit[i]))
+        order = np.argsort(splitix[mine])
+        assert np.array_equal(splitix[mine][order], np.arange(nsplit[i]))
         b, e = tb[mine][order], te[mine][order]
         assert b[0] == 0 and e[-1] == L and np.array_equal(b[1:], e[:-1]), f"seq {i} not tiled"
         if explicit_split:
             assert np.all(e - b <= explicit_split)
             assert np.all((e - b)[:-1] == explicit_split)
+    # the merge list: exactly the sequences with more than one piece
+    split = {i: int(nsplit[i]) for i in range(len(lens)) if nsplit[i] > 1}
+    listed = {int(s): int(n) for s, n in plan["slist"]}
+    assert len(listed) == len(plan["slist"]) and listed == split
+    assert plan["max_nsplit"] == max(nsplit.max(initial=0), 0)
 
 
 @pytest.mark.parametrize("name,split", [("gqa", 0), ("long", 0), ("mha", 0), ("prefix_cow", 0),
