@@ -89,12 +89,15 @@ struct TcLayout {
   static constexpr size_t OFF_DESC = (OFF_META + 2 * kNst * sizeof(ChunkMeta) + 15) / 16 * 16;
   static constexpr size_t OFF_RED = OFF_DESC + kQd * sizeof(ChunkDesc);
   static constexpr size_t OFF_LRED = OFF_RED + 2 * 2 * 4 * 16 * 4;
-  static constexpr size_t OFF_MISC = OFF_LRED + 2 * 4 * 16 * 4;
+  static constexpr size_t OFF_MISC = OFF_LRED + 2 * 2 * 4 * 16 * 4;
   static constexpr size_t SMEM_USED = OFF_MISC + 16;
   static constexpr size_t SMEM = SMEM_USED + 1024;   // slack to align the base to 1 KB
   static constexpr int NS = GT <= 8 ? 16 : 32;       // score MMA N: two halves x heads
   // per stream: two score accumulators (NS columns each) and the O^T accumulator
   static constexpr int COLS_PER_STREAM = 2 * NS + NPV;
+  // End-of-item work deferred into the next chunk (needs 2 GT + 4 spare
+  // registers per softmax thread; the 16-head tile has none)
+  static constexpr bool DEFER_END = GT <= 8;
   static constexpr uint32_t TMEM_COLS = 2 * COLS_PER_STREAM <= 128 ? 128 : 256;
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(kStage % 1024 == 0 && OFF_P % 1024 == 0, "swizzled tiles need 1 KB alignment");
@@ -179,10 +182,13 @@ __device__ __forceinline__ void split16(float p, uint16_t& hi, uint16_t& lo) {
   }
 }
 
+// Barrier among the 4 warps of a softmax group: one arrival per warp. The
+// result is made warp-uniform so a time-out never splits a warp.
 __device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t& phase, volatile int* abrt,
                                            int* status) {
-  mbar_arrive(bar);
-  const bool ok = mbar_wait(bar, phase, abrt, status);
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+  const bool ok = __all_sync(kFull, mbar_wait(bar, phase, abrt, status));
   phase ^= 1u;
   return ok;
 }
@@ -228,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   ChunkMeta* meta = reinterpret_cast<ChunkMeta*>(smem + Ly::OFF_META);   // [kNst][2]
   ChunkDesc* desc = reinterpret_cast<ChunkDesc*>(smem + Ly::OFF_DESC);
   float* red = reinterpret_cast<float*>(smem + Ly::OFF_RED);    // [2 grp][2][4][16]
-  float* lred = reinterpret_cast<float*>(smem + Ly::OFF_LRED);  // [2 grp][4][16]
+  float* lred = reinterpret_cast<float*>(smem + Ly::OFF_LRED);  // [2 grp][2 item parity][4][16]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Ly::OFF_MISC);
   volatile int* abrt = reinterpret_cast<volatile int*>(smem + Ly::OFF_MISC + 4);
 
@@ -247,16 +253,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_free[b], 128);
-      mbar_init(&p_full[b], 128);
+      // the softmax groups arrive once per warp (lane 0, after __syncwarp)
+      mbar_init(&s_free[b], 4);
+      mbar_init(&p_full[b], 4);
       mbar_init(&o_full[b], 1);
-      mbar_init(&o_free[b], 128);
-      mbar_init(&grp[b], 128);
+      mbar_init(&o_free[b], 4);
+      mbar_init(&grp[b], 4);
       mbar_init(&drain[b], 1);
     }
     for (int q = 0; q < kQd; ++q) {
-      mbar_init(&desc_full[q], 32);
-      mbar_init(&desc_empty[q], 32);
+      mbar_init(&desc_full[q], 1);                           // scheduler, lane 0
+      mbar_init(&desc_empty[q], 1);                          // producer, lane 0
     }
     *abrt = 0;
     fence_barrier_init();
@@ -282,12 +289,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     // Takes ring position c's descriptor from the scheduler, waits for the
-    // stage, and issues the chunk's copies: Q' (two boxes) and one K and one
-    // V box per page; or forwards an END / bubble / STOP marker.
+    // stage halves, and issues the chunk's copies: Q' (two boxes) and one K
+    // box per page, then one V box per page; or forwards an END / bubble /
+    // STOP marker.
     if (lane == 0) {
       prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
       prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_v);
     }
     int stops = 0;
     uint32_t ck = 0, cv = 0;   // positions whose K / V copies (or markers) were issued
@@ -310,55 +318,61 @@ __global__ void __launch_bounds__(kThreads, 1)
         m1 = reinterpret_cast<const uint4*>(&d.meta)[1];
         q_row = d.q_row;
       }
-      mbar_arrive(&desc_empty[qd]);   // every lane has its copy of the descriptor
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&desc_empty[qd]);   // every lane has its copy of the descriptor
       const int stage = c % kNst;
       const uint32_t epar = ((c / kNst) & 1u) ^ 1u;
       const int bi = 2 * stage + (c & 1);
       const bool data = !(flags & (kEnd | kBubble | kStop));
       uint8_t* st = smem + static_cast<size_t>(stage) * kStage;
-      // K and Q' (and the chunk's metadata) once the score MMA of the stage's
-      // previous chunk is done
-      if (!mbar_wait(&kempty[stage], epar, abrt, status)) {
-        ok = false;
-        break;
-      }
-      if (data) {
-        if (lane == 0) {
-          reinterpret_cast<uint4*>(&meta[bi])[0] = m0;
-          reinterpret_cast<uint4*>(&meta[bi])[1] = m1;
-          // K: one box of 2*BS half-rows per page; Q': the group's query rows,
-          // first halves then second halves (NS/2 rows each)
-          mbar_arrive_expect_tx(&kfull[bi], static_cast<uint32_t>(npg * BS * 256 + Ly::NS * 128));
-          tma_load_2d(st + 2 * kTile, &tm_q, 0, q_row, &kfull[bi]);
-          tma_load_2d(st + 2 * kTile + (Ly::NS / 2) * 128, &tm_q, 64, q_row, &kfull[bi]);
+      {
+        // K and Q' (and the chunk's metadata) once the score MMA of the
+        // stage's previous chunk is done
+        if (!mbar_wait(&kempty[stage], epar, abrt, status)) {
+          ok = false;
+          break;
         }
-        __syncwarp();
-        if (lane < npg)
-          tma_load_2d(st + lane * BS * 256, &tm_k, 0, (blk * Hkv + kvh) * BS * 2, &kfull[bi]);
-      } else {
-        if (lane == 0) {
-          meta[bi].flags = flags;
-          mbar_arrive(&kfull[bi]);
+        if (data) {
+          if (lane == 0) {
+            reinterpret_cast<uint4*>(&meta[bi])[0] = m0;
+            reinterpret_cast<uint4*>(&meta[bi])[1] = m1;
+            // K: one box of 2*BS half-rows per page; Q': the group's query
+            // rows, first halves then second halves (NS/2 rows each)
+            mbar_arrive_expect_tx(&kfull[bi],
+                                  static_cast<uint32_t>(npg * BS * 256 + Ly::NS * 128));
+            tma_load_2d(st + 2 * kTile, &tm_q, 0, q_row, &kfull[bi]);
+            tma_load_2d(st + 2 * kTile + (Ly::NS / 2) * 128, &tm_q, 64, q_row, &kfull[bi]);
+          }
+          __syncwarp();
+          if (lane < npg)
+            tma_load_2d(st + lane * BS * 256, &tm_k, 0, (blk * Hkv + kvh) * BS * 2, &kfull[bi]);
+        } else {
+          if (lane == 0) {
+            meta[bi].flags = flags;
+            mbar_arrive(&kfull[bi]);
+          }
+          __syncwarp();
         }
-        __syncwarp();
+        ++ck;
       }
-      ++ck;
-      // V once the P.V MMA of the stage's previous chunk is done
-      if (!mbar_wait(&vempty[stage], epar, abrt, status)) {
-        ok = false;
-        break;
+      {
+        // V once the P.V MMA of the stage's previous chunk is done
+        if (!mbar_wait(&vempty[stage], epar, abrt, status)) {
+          ok = false;
+          break;
+        }
+        if (data) {
+          if (lane == 0) mbar_arrive_expect_tx(&vfull[bi], static_cast<uint32_t>(npg * BS * 256));
+          __syncwarp();
+          if (lane < npg)
+            tma_load_2d(st + kTile + lane * BS * 256, &tm_v, 0, (blk * Hkv + kvh) * BS * 2,
+                        &vfull[bi]);
+        } else {
+          if (lane == 0) mbar_arrive(&vfull[bi]);
+          __syncwarp();
+        }
+        ++cv;
       }
-      if (data) {
-        if (lane == 0) mbar_arrive_expect_tx(&vfull[bi], static_cast<uint32_t>(npg * BS * 256));
-        __syncwarp();
-        if (lane < npg)
-          tma_load_2d(st + kTile + lane * BS * 256, &tm_v, 0, (blk * Hkv + kvh) * BS * 2,
-                      &vfull[bi]);
-      } else {
-        if (lane == 0) mbar_arrive(&vfull[bi]);
-        __syncwarp();
-      }
-      ++cv;
       if ((flags & kStop) && ++stops == 2) break;
     }
     if (!ok && lane == 0) {
@@ -503,7 +517,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else if (lane == 0) {
         d.meta.flags = kind == 1 ? kEnd : (kind == 2 ? kBubble : kStop);
       }
-      mbar_arrive(&desc_full[qd]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&desc_full[qd]);
       ++c;
       return !(kind == 3 && ++stops == 2);
     };
@@ -607,20 +622,52 @@ __global__ void __launch_bounds__(kThreads, 1)
     // own token's V half-rows in the stage: (t / sh) * sh * 256 + (t % sh) * 128, + sh * 128
     const int vrow_off = kTile + (own_t / sh) * sh * 256 + (own_t % sh) * 128;
     float* red_t = red + t * 128;
-    float* lred_t = lred + t * 64;
+    float* lred_t = lred + t * 128;
     uint64_t* gbar = &grp[t];
-    float m_run[GT], l_thr[GT], o[GT];
-    uint32_t gphase = 0, n = 0;
     float2* ml = reinterpret_cast<float2*>(p.ws + p.ml_off);
     float* po = reinterpret_cast<float*>(p.ws + p.o_off);
+    float m_run[GT], l_thr[GT], o[GT];
+    uint32_t gphase = 0, n = 0;
+    // an item's end: per-warp sums of l are written at its last chunk into
+    // lred_t[item parity]; the cross-warp sum, normalisation and stores
+    // (finish) run after the next chunk's max barrier, once that chunk's P is
+    // published, or at END after one barrier
+    float o_pend[Ly::DEFER_END ? GT : 1], m_pend[Ly::DEFER_END ? GT : 1];
+    int pend_seq = 0, pend_kvh = 0, pend_split = 0;
+    bool pend = false;
+    uint32_t lpar = 0;   // parity of the next item to end
+    auto finish = [&](const float* lr, int seq, int kvh, int split_raw, const float* ov_,
+                      const float* mv_) {
+      const int nsp = item_nsplit(split_raw);
+      const int split = item_split(split_raw);
+#pragma unroll
+      for (int g = 0; g < GT; ++g) {
+        if (g >= G) break;
+        const float L = lr[g] + lr[16 + g] + lr[32 + g] + lr[48 + g];
+        const size_t row = static_cast<size_t>(seq) * p.num_q_heads + kvh * G + g;
+        if (nsp == 1) {
+          p.out[row * kD + r] = ov_[g] / L;
+        } else {
+          const size_t pr_ = row * p.max_splits + split;
+          po[pr_ * kD + r] = ov_[g];
+          if (r == 0) ml[pr_] = make_float2(mv_[g], L);
+        }
+      }
+    };
 
     for (uint32_t c = t;; c += 2) {
       const int stage = c % kNst;
       const uint32_t fpar = (c / (2 * kNst)) & 1u;
-      if (!mbar_wait(&kfull[2 * stage + t], fpar, abrt, status)) break;
+      if (!__all_sync(kFull, mbar_wait(&kfull[2 * stage + t], fpar, abrt, status))) break;
       const ChunkMeta mt = meta[2 * stage + t];
       if (mt.flags & kEnd) {
-        mbar_arrive(&p_full[t]);   // acknowledge END so the slot can be released
+        if (Ly::DEFER_END && pend) {
+          if (!group_sync(gbar, gphase, abrt, status)) break;
+          finish(lred_t + (lpar ^ 1u) * 64, pend_seq, pend_kvh, pend_split, o_pend, m_pend);
+          pend = false;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[t]);   // acknowledge END so the slot can be released
         break;
       }
       if (mt.flags & kFirst) {
@@ -633,7 +680,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const uint32_t par = n & 1u;
       // ---- scores of tokens tk0 and tk0 + 64 (both halves summed)
-      if (!mbar_wait(&s_full[t], par, abrt, status)) break;
+      if (!__all_sync(kFull, mbar_wait(&s_full[t], par, abrt, status))) break;
       tc_fence_after();
       float sv0[Ly::NS], sv1[Ly::NS];
       tmem_ld16(lane_addr + s_col, sv0);
@@ -643,7 +690,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld16(lane_addr + s_col + Ly::NS + 16, sv1 + 16);
       }
       tc_fence_before();
-      mbar_arrive(&s_free[t]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[t]);
       const bool ok0 = tk0 < mt.valid, ok1 = tk0 + 64 < mt.valid;
       float sa[GT], sb[GT];
 #pragma unroll
@@ -691,55 +739,67 @@ __global__ void __launch_bounds__(kThreads, 1)
                        col[8 * ng + 2] | (col[8 * ng + 3] << 16),
                        col[8 * ng + 4] | (col[8 * ng + 5] << 16),
                        col[8 * ng + 6] | (col[8 * ng + 7] << 16));
+      bool vok = true;
       if (own_t >= mt.valid && own_t < ((mt.valid + 15) & ~15)) {
         // past the chunk's valid tokens but inside the last 16-token step of
         // the P.V MMA: make V finite (zero) once the stage's V has landed
-        if (!mbar_wait(&vfull[2 * stage + t], fpar, abrt, status)) break;
-        uint8_t* vrow = smem + static_cast<size_t>(stage) * kStage + vrow_off;
+        vok = mbar_wait(&vfull[2 * stage + t], fpar, abrt, status);
+        if (vok) {
+          uint8_t* vrow = smem + static_cast<size_t>(stage) * kStage + vrow_off;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          reinterpret_cast<uint4*>(vrow)[i] = make_uint4(0, 0, 0, 0);
-          reinterpret_cast<uint4*>(vrow + sh * 128)[i] = make_uint4(0, 0, 0, 0);
+          for (int i = 0; i < 8; ++i) {
+            reinterpret_cast<uint4*>(vrow)[i] = make_uint4(0, 0, 0, 0);
+            reinterpret_cast<uint4*>(vrow + sh * 128)[i] = make_uint4(0, 0, 0, 0);
+          }
         }
       }
+      if (!__all_sync(kFull, vok)) break;
       fence_proxy_async_smem();
-      mbar_arrive(&p_full[t]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[t]);
+      if (Ly::DEFER_END && pend) {
+        // the previous item's end, while the P.V MMA runs (the max barrier
+        // above made every warp's l sums visible)
+        finish(lred_t + (lpar ^ 1u) * 64, pend_seq, pend_kvh, pend_split, o_pend, m_pend);
+        pend = false;
+      }
       // ---- correction: O = alpha * O + O_chunk (thread r owns column d = r)
-      if (!mbar_wait(&o_full[t], par, abrt, status)) break;
+      if (!__all_sync(kFull, mbar_wait(&o_full[t], par, abrt, status))) break;
       tc_fence_after();
       float ov[NPV];
       tmem_ld16(lane_addr + o_col, ov);
       if constexpr (NPV == 32) tmem_ld16(lane_addr + o_col + 16, ov + 16);
       tc_fence_before();
-      mbar_arrive(&o_free[t]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_free[t]);
 #pragma unroll
       for (int g = 0; g < GT; ++g) o[g] = fmaf(o[g], alpha[g], ov[g] + ov[GT + g]);
       ++n;
 
       if (mt.flags & kLast) {
-        // sum of l over the group's 128 tokens
+        // per-warp sum of l over the group's 128 tokens
+        float* lr = lred_t + (Ly::DEFER_END ? lpar : 0u) * 64;
 #pragma unroll
         for (int g = 0; g < GT; ++g) {
           float lg = l_thr[g];
 #pragma unroll
           for (int off = 16; off > 0; off >>= 1) lg += __shfl_xor_sync(kFull, lg, off);
-          if (lane == 0) lred_t[wq * 16 + g] = lg;
+          if (lane == 0) lr[wq * 16 + g] = lg;
         }
-        if (!group_sync(gbar, gphase, abrt, status)) break;
-        const int nsp = item_nsplit(mt.split_raw);
-        const int split = item_split(mt.split_raw);
+        if constexpr (Ly::DEFER_END) {
 #pragma unroll
-        for (int g = 0; g < GT; ++g) {
-          if (g >= G) break;
-          const float L = lred_t[g] + lred_t[16 + g] + lred_t[32 + g] + lred_t[48 + g];
-          const size_t row = static_cast<size_t>(mt.seq) * p.num_q_heads + mt.kvh * G + g;
-          if (nsp == 1) {
-            p.out[row * kD + r] = o[g] / L;
-          } else {
-            const size_t pr_ = row * p.max_splits + split;
-            po[pr_ * kD + r] = o[g];
-            if (r == 0) ml[pr_] = make_float2(m_run[g], L);
+          for (int g = 0; g < GT; ++g) {
+            o_pend[g] = o[g];
+            m_pend[g] = m_run[g];
           }
+          pend_seq = mt.seq;
+          pend_kvh = mt.kvh;
+          pend_split = mt.split_raw;
+          pend = true;
+          lpar ^= 1u;
+        } else {
+          if (!group_sync(gbar, gphase, abrt, status)) break;
+          finish(lr, mt.seq, mt.kvh, mt.split_raw, o, m_run);
         }
       }
     }
