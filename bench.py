@@ -246,17 +246,15 @@ def time_device(step, K, W, stream, use_graph, world):
 
 
 def time_decode_only(b, ops, out, ws, split, path, stream, K, use_graph=True):
-    """Average duration of the decode call alone (plan + main + merge kernels),
-    with events around each call; replayed from a CUDA graph like the step, so
-    host launch overhead stays out of the device time."""
+    """Average duration of the decode call alone (plan + main + merge kernels):
+    K calls back to back between two events on the launching stream, replayed
+    from a CUDA graph like the step, so the device never waits for the host."""
     max_ctx = b.max_context_len
 
     def call():
         ops.pa_decode(out, b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens,
                       max_ctx, b.scale, ws, split_tokens=split, path=path, stream=stream)
 
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(K)]
     with torch.cuda.stream(stream):
         for _ in range(3):
             call()
@@ -268,17 +266,17 @@ def time_decode_only(b, ops, out, ws, split, path, stream, K, use_graph=True):
                 call()
             graph.replay()
             torch.cuda.synchronize()
-        for a, z in ev:
-            a.record(stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
             if graph is not None:
                 graph.replay()
             else:
                 call()
-            z.record(stream)
+        e1.record(stream)
         torch.cuda.synchronize()
     del graph
-    ts = [a.elapsed_time(z) for a, z in ev]
-    return statistics.median(ts), ts
+    return e0.elapsed_time(e1) / K
 
 
 def time_e2e(b, ops, ws, split, path, stream, K, W):
@@ -407,7 +405,7 @@ def run_ours(args, rank, world, local):
     ms = max_over_ranks(ms, world)
     torch.cuda.synchronize()
     status = ops.pa_decode_status(ws, stream)
-    dec_ms, _ = time_decode_only(b, ops, out, ws, args.split, path, stream, max(10, args.steps),
+    dec_ms = time_decode_only(b, ops, out, ws, args.split, path, stream, max(10, args.steps),
                                  not args.no_graph)
     e2e_ms, h2d, d2h = time_e2e(b, ops, ws, args.split, path, stream, max(5, args.steps // 2), 3)
     e2e_ms = max_over_ranks(e2e_ms, world)
@@ -457,7 +455,7 @@ def run_ours(args, rank, world, local):
             out2 = torch.empty((B2, Hq2, D2), dtype=torch.float32, device="cuda")
             st2 = step_fn(b, ops, out2, ws2, 0, ops.PA_PATH_AUTO, stream)
             ms2, _ = time_device(st2, max(10, args.steps // 2), 3, stream, not args.no_graph, 1)
-            d2, _ = time_decode_only(b, ops, out2, ws2, 0, ops.PA_PATH_AUTO, stream, 10,
+            d2 = time_decode_only(b, ops, out2, ws2, 0, ops.PA_PATH_AUTO, stream, 10,
                                      not args.no_graph)
             kb = b.kv_bytes_logical()
             sec[b.name] = {"step_gbps": round(kb / (ms2 * 1e-3) / 1e9, 1),

@@ -72,9 +72,6 @@ cudaError_t cached_ctas(bool tc, int dtype, int head_dim, int group, int* out) {
   return cudaSuccess;
 }
 
-constexpr int kItemsPerCta = 12;      // CUDA-core kernel: per persistent CTA
-constexpr int kItemsPerStreamTc = 8;  // tensor-core kernel: per item stream
-
 }  // namespace
 
 void record_cuda_error(cudaError_t e) {
@@ -216,7 +213,6 @@ pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
   pp.max_splits = lay.max_splits;
   // the tensor-core kernel runs two independent item streams per CTA
   pp.num_ctas = use_tc ? 2 * ctas : ctas;
-  pp.items_per_cta = use_tc ? kItemsPerStreamTc : kItemsPerCta;
   e = launch_plan(pp, s);
   if (e != cudaSuccess) return cuda_fail(e);
 

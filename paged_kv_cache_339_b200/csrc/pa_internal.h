@@ -19,8 +19,7 @@ struct PlanParams {
   int32_t split_tokens;   // explicit split, or 0 = choose on the device
   int32_t min_split;      // lower bound of an automatic split
   int32_t max_splits;
-  int32_t num_ctas;       // persistent CTAs of the decode kernel
-  int32_t items_per_cta;  // target work items per CTA (automatic split)
+  int32_t num_ctas;       // item streams of the decode kernel (CTAs x streams per CTA)
 };
 
 // Everything a decode main kernel needs; filled by the C-ABI shim.

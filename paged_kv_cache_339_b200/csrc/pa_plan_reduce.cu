@@ -5,10 +5,11 @@
 // the pairs longest first (bucketed by 128-token chunk count), so the
 // persistent decode kernels, which claim pairs in list order, end on short
 // pieces and finish together. Pieces: as many whole S-token pieces as fit,
-// then the rest of the sequence. With an automatic split, when those rests
-// hold too little work to even out the CTAs' finishing times (a few long
-// sequences), each sequence's last few S-token pieces are cut into pieces
-// of about S/4 tokens instead.
+// then the rest of the sequence. The automatic S is one stream's fair share
+// of the work (splits cost partial results and a merge, so only sequences
+// longer than that are cut); when the rests hold too little work to even
+// out the streams' finishing times (a few long sequences), each sequence's
+// last S-token pieces are cut into tail pieces of about an eighth of a share.
 //
 // merge_kernel combines the partial softmax results of sequences that were
 // split: with per-split running max m_p (log2 units), sum l_p and
@@ -121,12 +122,14 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
       b |= __shfl_xor_sync(0xffffffffu, b, o);
     }
     if (lane == 0) {
+      // one stream's fair share of the work, in tokens of one KV head
+      const long long share = (t * p.num_kv_heads + p.num_ctas - 1) / p.num_ctas;
       int S = p.split_tokens;
       if (S <= 0) {
-        // Aim for ~items_per_cta work items per persistent CTA.
-        long long per_cta = (t * p.num_kv_heads + p.num_ctas - 1) / p.num_ctas;
-        long long want = (per_cta + p.items_per_cta - 1) / p.items_per_cta;
-        want = (want + kAutoSplitQuantum - 1) / kAutoSplitQuantum * kAutoSplitQuantum;
+        // Whole pieces of up to one share: every split costs partial results
+        // and a merge, so only sequences longer than a share are cut; the
+        // longest-first order evens the CTAs out with the short sequences.
+        long long want = (share + kAutoSplitQuantum - 1) / kAutoSplitQuantum * kAutoSplitQuantum;
         if (want < p.min_split) want = p.min_split;
         if (want > (1 << 30)) want = 1 << 30;
         S = static_cast<int>(want);
@@ -134,7 +137,11 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
       s_rule.S = S;
       s_rule.cut = 0;
       s_rule.e = 0;
-      s_rule.sB = S;
+      // tail pieces, if the list needs them: about an eighth of a share
+      long long sb = share / 8 / kAutoSplitQuantum * kAutoSplitQuantum;
+      if (sb < kAutoSplitQuantum) sb = kAutoSplitQuantum;
+      if (sb > S) sb = S;
+      s_rule.sB = static_cast<int>(sb);
       s_rule.ms = p.max_splits;
       hdr->status = b ? 1 /* PA_ERR_INVALID_ARG */ : 0;
       hdr->split_tokens = S;
@@ -144,12 +151,15 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
   __syncthreads();
   const int S = s_rule.S;
 
-  // 2. work in the rests (the pieces shorter than S), per KV head
+  // 2. short work: the rests (pieces shorter than S) of at most two tail
+  // pieces, in tokens of one KV head
   if (p.split_tokens <= 0) {
+    const int short_max = 2 * s_rule.sB;
     long long rem = 0;
     for (int i = tid; i < p.num_seqs; i += nthreads) {
       const int L = s_len[i];
-      if (valid_len(L)) rem += L % S;
+      const int rest = valid_len(L) ? L % S : 0;
+      if (rest <= short_max) rem += rest;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) rem += __shfl_xor_sync(0xffffffffu, rem, o);
@@ -159,15 +169,16 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
       long long r = lane < nwarps ? s_sum[lane] : 0;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
-      // When the whole pieces run out, the CTAs are on average half an
-      // S-piece from their end; about that much short-piece work evens them
-      // out.
-      const long long target = static_cast<long long>(p.num_ctas) * S / (2 * p.num_kv_heads);
+      // The list should end on enough short work to even the streams out:
+      // about two tail pieces per stream. Few or equally long sequences
+      // leave too little in short rests; then the last whole pieces (and
+      // rest) of every sequence are cut into tail pieces.
+      const long long target =
+          2LL * p.num_ctas * s_rule.sB / p.num_kv_heads;   // tokens of one KV head
       if (lane == 0 && r < target && p.num_seqs > 0) {
         const long long per_seq = static_cast<long long>(p.num_seqs) * S;
         s_rule.cut = 1;
         s_rule.e = static_cast<int>(min((target - r + per_seq - 1) / per_seq, 1LL << 20));
-        s_rule.sB = max(128, S / 4 / 128 * 128);
       }
     }
     __syncthreads();

@@ -23,7 +23,7 @@ struct WsHeader {
   int32_t split_tokens;  // tokens per split chosen for this call
   int32_t max_splits;    // split capacity per sequence in this workspace
   int32_t num_split_seqs;  // sequences cut into more than one piece (merge list length)
-  int32_t max_nsplit;      // largest piece count of a sequence
+  int32_t max_nsplit;      // largest piece count of a split sequence (0: none split)
   int32_t reserved[56];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
