@@ -209,7 +209,7 @@ def step_fn(b, ops, out, ws, split, path, stream):
         ops.pa_write_kv(b.k_cache, b.v_cache, b.key, b.value, b.slot_mapping, stream=stream)
         ops.pa_decode(out, b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, max_ctx,
                       b.scale, ws, split_tokens=split, path=path, stream=stream)
-        return n + 1 + 3   # write, plan, decode, merge
+        return n + 1 + 2   # write, plan, decode
     return step
 
 
@@ -246,7 +246,7 @@ def time_device(step, K, W, stream, use_graph, world):
 
 
 def time_decode_only(b, ops, out, ws, split, path, stream, K, use_graph=True):
-    """Average duration of the decode call alone (plan + main + merge kernels):
+    """Average duration of the decode call alone (plan + main kernels):
     K calls back to back between two events on the launching stream, replayed
     from a CUDA graph like the step, so the device never waits for the host."""
     max_ctx = b.max_context_len
@@ -430,7 +430,7 @@ def run_ours(args, rank, world, local):
         "decode_status": int(status),
         "gpu_launches": per_step * args.steps,
         "roofline": {
-            "bound": "hbm", "kernel": "pa_decode (plan + decode main + merge)",
+            "bound": "hbm", "kernel": "pa_decode (plan + decode main, merge fused)",
             "achieved": round(dec_gbps, 1), "peak": peak, "unit": "GB/s",
             "frac": round(dec_gbps / peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
             "algorithmic_bytes_per_launch": kv_bytes,

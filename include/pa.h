@@ -179,6 +179,12 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
  * probabilities at ~16 significant bits (two 16-bit terms).
  * PA_ERR_UNSUPPORTED also for more than 56,320 sequences in one call (the
  * planning kernel keeps the lengths in one CTA's shared memory).
+ * Enqueues two kernels: a planning kernel, then the decode kernel. The
+ * planning kernel is launched with programmatic stream serialisation: it may
+ * start while the kernel before it in the stream is finishing, reads
+ * context_lens at once and waits for that kernel before it completes. A
+ * kernel right before pa_decode that lets its dependents launch early
+ * (griddepcontrol.launch_dependents) must have written context_lens by then.
  */
 pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
                     const int32_t* block_tables, int32_t bt_stride,

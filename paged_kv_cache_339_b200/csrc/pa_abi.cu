@@ -200,7 +200,7 @@ pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
   pp.ws = ws;
   pp.pairs_off = lay.pairs_off;
   pp.nsplit_off = lay.nsplit_off;
-  pp.slist_off = lay.slist_off;
+  pp.cnt_off = lay.cnt_off;
   pp.num_seqs = num_seqs;
   pp.num_q_heads = num_q_heads;
   pp.num_kv_heads = cache->num_kv_heads;
@@ -224,6 +224,7 @@ pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
   dp.block_tables = block_tables;
   dp.ws = ws;
   dp.pairs_off = lay.pairs_off;
+  dp.cnt_off = lay.cnt_off;
   dp.ml_off = lay.ml_off;
   dp.o_off = lay.o_off;
   dp.bt_stride = bt_stride;
@@ -239,19 +240,6 @@ pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
   e = use_tc ? launch_decode_tc(dp, ctas, s) : launch_decode_simt(dp, ctas, s);
   if (e != cudaSuccess) return cuda_fail(e);
 
-  MergeParams mp;
-  mp.out = out;
-  mp.ws = ws;
-  mp.slist_off = lay.slist_off;
-  mp.ml_off = lay.ml_off;
-  mp.o_off = lay.o_off;
-  mp.num_seqs = num_seqs;
-  mp.num_q_heads = num_q_heads;
-  mp.num_kv_heads = cache->num_kv_heads;
-  mp.head_dim = cache->head_dim;
-  mp.max_splits = lay.max_splits;
-  e = launch_merge(mp, s);
-  if (e != cudaSuccess) return cuda_fail(e);
 
   return PA_OK;
 }

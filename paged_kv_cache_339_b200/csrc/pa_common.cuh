@@ -235,4 +235,61 @@ __device__ __forceinline__ void pdl_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
+// ---------------------------------------------------------------------------
+// Split-context merge, done by the last piece of a (sequence, KV head) to
+// finish. With per-piece running max m_p (log2 units), sum l_p and
+// unnormalised accumulator a_p:
+//   M = max_p m_p,  L = sum_p l_p 2^(m_p - M),  o = sum_p a_p 2^(m_p - M) / L.
+// This regrouping is exact algebra on the softmax sums; the pages do not
+// discuss splitting a context. The pieces were written by other CTAs of the
+// same grid, so they are read through L2 (ld.global.cg).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void merge_split_rows(float* out, const float2* ml, const float* po,
+                                                 size_t row0, int nrows, int D, int nsp,
+                                                 int max_splits, int tid, int nthreads) {
+  // a thread per (row, 4 columns); one pass over the pieces with a running
+  // maximum, 8 pieces' loads in flight at a time
+  const int vpr = D / 4;
+  for (int idx = tid; idx < nrows * vpr; idx += nthreads) {
+    const int h = idx / vpr, c4 = idx - h * vpr;
+    const size_t row = row0 + h;
+    const float2* mr = ml + row * max_splits;
+    const float4* pr = reinterpret_cast<const float4*>(po + row * max_splits * D) + c4;
+    float M = -INFINITY, L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < nsp; s0 += 8) {
+      float2 e[8];
+      float4 v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const bool in = s0 + j < nsp;
+        e[j] = in ? __ldcg(mr + s0 + j) : make_float2(-INFINITY, 0.f);
+        v[j] = in ? __ldcg(pr + static_cast<size_t>(s0 + j) * vpr) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      float mb = M;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) mb = fmaxf(mb, e[j].x);
+      const float sc = exp2f(M - mb);   // M = -inf on the first batch: 0
+      L *= sc;
+      acc.x *= sc;
+      acc.y *= sc;
+      acc.z *= sc;
+      acc.w *= sc;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float w = exp2f(e[j].x - mb);   // 0 for the padding entries
+        L = fmaf(e[j].y, w, L);
+        acc.x = fmaf(w, v[j].x, acc.x);
+        acc.y = fmaf(w, v[j].y, acc.y);
+        acc.z = fmaf(w, v[j].z, acc.z);
+        acc.w = fmaf(w, v[j].w, acc.w);
+      }
+      M = mb;
+    }
+    const float inv = 1.0f / L;
+    reinterpret_cast<float4*>(out + row * D)[c4] =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  }
+}
+
 }  // namespace pa

@@ -109,6 +109,7 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 template <typename T, int D, int GPW>
 __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
     simt_decode_kernel(const DecodeParams p) {
+  __shared__ volatile int s_last;   // this piece completed its sequence
   using Tr = SimtTraits<T, D, GPW>;
   constexpr int CHUNK = Tr::CHUNK, ROW = Tr::ROW, NST = Tr::NST;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -136,7 +137,7 @@ __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
   }
   __syncthreads();
   pdl_wait();   // the plan (and the KV write before it) are complete from here on
-  pdl_launch_dependents();   // the merge kernel may get resident; it waits for us
+  // (no early launch of dependents: the next call's plan rewrites the workspace)
 
   const int num_items = hdr->num_items;
   const int Hkv = p.num_kv_heads, BS = p.block_size;
@@ -401,6 +402,7 @@ __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
         const int split = item_split(mt.split_raw);
         float2* ml = reinterpret_cast<float2*>(p.ws + p.ml_off);
         float* po = reinterpret_cast<float*>(p.ws + p.o_off);
+        const size_t row0 = static_cast<size_t>(mt.seq) * p.num_q_heads + mt.kvh * G;
         for (int idx = tid; idx < G * D; idx += Tr::NCW * 32) {
           const int h = idx / D, d = idx - (idx / D) * D;
           const int hgi = h / GPW, g = h - hgi * GPW;
@@ -413,7 +415,7 @@ __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
             L = fmaf(src[GPW * D + GPW + g], sc, L);
             O = fmaf(src[g * D + d], sc, O);
           }
-          const size_t row = static_cast<size_t>(mt.seq) * p.num_q_heads + mt.kvh * G + h;
+          const size_t row = row0 + h;
           if (single) {
             p.out[row * D + d] = O / L;
           } else {
@@ -422,7 +424,20 @@ __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
             if (d == 0) ml[pr_] = make_float2(M, L);
           }
         }
+        if (!single) __threadfence();   // this piece's partial result, before it is counted
         if (!group_sync(&gbar[0], gphase, abrt, status)) break;
+        if (!single) {
+          // the last piece of the (sequence, KV head) to finish merges them all
+          if (tid == 0)
+            s_last = atomicAdd(reinterpret_cast<int*>(p.ws + p.cnt_off) +
+                                   static_cast<size_t>(mt.seq) * Hkv + mt.kvh,
+                               1) == nsp - 1;
+          if (!group_sync(&gbar[0], gphase, abrt, status)) break;
+          if (s_last) {
+            __threadfence();   // every other piece counted before us is visible
+            merge_split_rows(p.out, ml, po, row0, G, D, nsp, p.max_splits, tid, Tr::NCW * 32);
+          }
+        }
       }
       ++c;
     }

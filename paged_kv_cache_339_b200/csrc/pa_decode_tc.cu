@@ -35,8 +35,8 @@
 //   warps 3-6,  softmax and correction groups, one per stream: thread r owns
 //   7-10        token r of a chunk for the softmax (tcgen05.ld of its S^T row)
 //               and output column d = r for the correction O = alpha O + O_c;
-//               partial results of split items go to the workspace for the
-//               merge kernel.
+//               a split item writes its partial result to the workspace, and
+//               the last piece of a (sequence, KV head) to finish merges them.
 // No load uses cluster multicast; every wait is bounded (see pa_common.cuh).
 #include <cudaTypedefs.h>
 
@@ -207,6 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap tm_q) {
   using Ly = TcLayout<GT>;
   constexpr int NPV = Ly::NPV;
+  __shared__ volatile int s_last[2];   // per group: this piece completed its sequence
   extern __shared__ uint8_t smem_raw[];
   // 1 KB alignment for the 128-byte-swizzled tiles
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -280,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   pdl_wait();   // the plan (and the KV write before it) are complete from here on
-  pdl_launch_dependents();   // the merge kernel may get resident; it waits for us
+  // (no early launch of dependents: the next call's plan rewrites the workspace)
 
   const int num_items = hdr->num_items;
   const int Hkv = p.num_kv_heads, BS = p.block_size;
@@ -626,6 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* gbar = &grp[t];
     float2* ml = reinterpret_cast<float2*>(p.ws + p.ml_off);
     float* po = reinterpret_cast<float*>(p.ws + p.o_off);
+    int* cnt = reinterpret_cast<int*>(p.ws + p.cnt_off);
     float m_run[GT], l_thr[GT], o[GT];
     uint32_t gphase = 0, n = 0;
     // an item's end: per-warp sums of l are written at its last chunk into
@@ -636,15 +638,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     int pend_seq = 0, pend_kvh = 0, pend_split = 0;
     bool pend = false;
     uint32_t lpar = 0;   // parity of the next item to end
+    // an item's result: the output rows, or the piece's partial result and,
+    // for the last piece of the (sequence, KV head) to finish, the merge of
+    // all of them; false when a barrier gave up
     auto finish = [&](const float* lr, int seq, int kvh, int split_raw, const float* ov_,
-                      const float* mv_) {
+                      const float* mv_) -> bool {
       const int nsp = item_nsplit(split_raw);
       const int split = item_split(split_raw);
+      const size_t row0 = static_cast<size_t>(seq) * p.num_q_heads + kvh * G;
 #pragma unroll
       for (int g = 0; g < GT; ++g) {
         if (g >= G) break;
         const float L = lr[g] + lr[16 + g] + lr[32 + g] + lr[48 + g];
-        const size_t row = static_cast<size_t>(seq) * p.num_q_heads + kvh * G + g;
+        const size_t row = row0 + g;
         if (nsp == 1) {
           p.out[row * kD + r] = ov_[g] / L;
         } else {
@@ -653,6 +659,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (r == 0) ml[pr_] = make_float2(mv_[g], L);
         }
       }
+      if (nsp == 1) return true;
+      __threadfence();   // this piece's partial result, before it is counted
+      if (!group_sync(gbar, gphase, abrt, status)) return false;
+      if (wq == 0 && lane == 0)
+        s_last[t] = atomicAdd(cnt + static_cast<size_t>(seq) * Hkv + kvh, 1) == nsp - 1;
+      if (!group_sync(gbar, gphase, abrt, status)) return false;
+      if (s_last[t]) {
+        __threadfence();   // every other piece counted before us is visible
+        merge_split_rows(p.out, ml, po, row0, G, kD, nsp, p.max_splits, r, 128);
+      }
+      return true;
     };
 
     for (uint32_t c = t;; c += 2) {
@@ -663,7 +680,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (mt.flags & kEnd) {
         if (Ly::DEFER_END && pend) {
           if (!group_sync(gbar, gphase, abrt, status)) break;
-          finish(lred_t + (lpar ^ 1u) * 64, pend_seq, pend_kvh, pend_split, o_pend, m_pend);
+          if (!finish(lred_t + (lpar ^ 1u) * 64, pend_seq, pend_kvh, pend_split, o_pend, m_pend))
+            break;
           pend = false;
         }
         __syncwarp();
@@ -760,7 +778,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (Ly::DEFER_END && pend) {
         // the previous item's end, while the P.V MMA runs (the max barrier
         // above made every warp's l sums visible)
-        finish(lred_t + (lpar ^ 1u) * 64, pend_seq, pend_kvh, pend_split, o_pend, m_pend);
+        if (!finish(lred_t + (lpar ^ 1u) * 64, pend_seq, pend_kvh, pend_split, o_pend, m_pend))
+          break;
         pend = false;
       }
       // ---- correction: O = alpha * O + O_chunk (thread r owns column d = r)
@@ -799,7 +818,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           lpar ^= 1u;
         } else {
           if (!group_sync(gbar, gphase, abrt, status)) break;
-          finish(lr, mt.seq, mt.kvh, mt.split_raw, o, m_run);
+          if (!finish(lr, mt.seq, mt.kvh, mt.split_raw, o, m_run)) break;
         }
       }
     }

@@ -13,7 +13,7 @@ struct PlanParams {
   const int32_t* context_lens;
   float* out;
   uint8_t* ws;
-  size_t pairs_off, nsplit_off, slist_off;
+  size_t pairs_off, nsplit_off, cnt_off;
   int32_t num_seqs, num_q_heads, num_kv_heads, head_dim;
   int32_t bt_stride, block_size, max_context_len;
   int32_t split_tokens;   // explicit split, or 0 = choose on the device
@@ -30,24 +30,16 @@ struct DecodeParams {
   float* out;
   const int32_t* block_tables;
   uint8_t* ws;
-  size_t pairs_off, ml_off, o_off;
+  size_t pairs_off, cnt_off, ml_off, o_off;
   int32_t bt_stride, num_blocks, num_kv_heads, num_q_heads, head_dim,
       block_size, num_seqs, max_splits;
   float scale_log2;  // scale * log2(e): scores kept in log2 units
   int32_t dtype;     // pa_dtype
 };
 
-struct MergeParams {
-  float* out;
-  const uint8_t* ws;
-  size_t slist_off, ml_off, o_off;
-  int32_t num_seqs, num_q_heads, num_kv_heads, head_dim, max_splits;
-};
-
-// Both launch with programmatic stream serialisation (PDL): the kernel may be
-// scheduled while its predecessor in the stream finishes.
+// Launched with programmatic stream serialisation (PDL): the plan may be
+// scheduled while its predecessor in the stream (the KV write) finishes.
 cudaError_t launch_plan(const PlanParams& p, cudaStream_t stream);
-cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream);
 
 // CUDA-core decode. Returns cudaErrorInvalidValue for an unsupported shape.
 bool simt_supported(int dtype, int head_dim, int group);

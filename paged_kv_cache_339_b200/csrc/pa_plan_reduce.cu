@@ -1,4 +1,4 @@
-// Work planning and split-context merge for pa_decode.
+// Work planning for pa_decode.
 //
 // plan_kernel (one CTA) reads the context lengths, checks them, picks the
 // split size S and cuts every sequence into pieces (work pairs). It lists
@@ -11,12 +11,9 @@
 // out the streams' finishing times (a few long sequences), each sequence's
 // last S-token pieces are cut into tail pieces of about an eighth of a share.
 //
-// merge_kernel combines the partial softmax results of sequences that were
-// split: with per-split running max m_p (log2 units), sum l_p and
-// unnormalised accumulator a_p,
-//   M = max_p m_p,  L = sum_p l_p 2^(m_p - M),  o = sum_p a_p 2^(m_p - M) / L.
-// This regrouping is exact algebra on the softmax sums; the pages do not
-// discuss splitting a context.
+// The partial results of a split sequence are merged inside the decode
+// kernels by the last piece to finish (pa_common.cuh, merge_split_rows); the
+// plan zeroes the merge counters they count on.
 //
 // Launched with programmatic stream serialisation: it may start while the KV
 // write before it is still running (it reads only the lengths), and waits for
@@ -74,13 +71,12 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
   __shared__ int s_hist[kKeys + 1];
   __shared__ int s_fill[kKeys + 1];
   __shared__ PieceRule s_rule;
-  __shared__ int s_nsl, s_maxn;
   extern __shared__ int s_len[];   // [num_seqs]
 
   WsHeader* hdr = reinterpret_cast<WsHeader*>(p.ws);
   WorkPair* pairs = reinterpret_cast<WorkPair*>(p.ws + p.pairs_off);
   int32_t* nsplit = reinterpret_cast<int32_t*>(p.ws + p.nsplit_off);
-  int2* slist = reinterpret_cast<int2*>(p.ws + p.slist_off);
+  int32_t* cnt = reinterpret_cast<int32_t*>(p.ws + p.cnt_off);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nthreads = blockDim.x, nwarps = nthreads >> 5;
   const int64_t cap = static_cast<int64_t>(p.bt_stride) * p.block_size;
@@ -99,10 +95,7 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
     }
   }
   for (int k = tid; k <= kKeys; k += nthreads) s_hist[k] = 0;
-  if (tid == 0) {
-    s_nsl = 0;
-    s_maxn = 0;
-  }
+
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     tot += __shfl_xor_sync(0xffffffffu, tot, o);
@@ -185,8 +178,8 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
   }
   const PieceRule rule = s_rule;
 
-  // 3. pieces per sequence (a thread per sequence): split counts, the list of
-  // split sequences for the merge, and the length histogram (a sequence's
+  // 3. pieces per sequence (a thread per sequence): split counts, zeroed merge
+  // counters of split sequences, and the length histogram (a sequence's
   // pieces form at most three runs of equal length); sequences with nothing
   // to attend to get zero rows
   for (int i = tid; i < p.num_seqs; i += nthreads) {
@@ -195,10 +188,8 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
     if (valid_len(L) && L > 0) seq_pieces(L, rule, nA, sb, k);
     const int n = nA + k;
     nsplit[i] = n;
-    if (n > 1) {
-      slist[atomicAdd(&s_nsl, 1)] = make_int2(i, n);
-      atomicMax(&s_maxn, n);
-    }
+    if (n > 1)
+      for (int h = 0; h < p.num_kv_heads; ++h) cnt[static_cast<size_t>(i) * p.num_kv_heads + h] = 0;
     if (nA > 0) atomicAdd(&s_hist[piece_key(S)], nA);
     if (k > 1) atomicAdd(&s_hist[piece_key(sb)], k - 1);
     if (k > 0) atomicAdd(&s_hist[piece_key(L - nA * S - (k - 1) * sb)], 1);
@@ -228,8 +219,6 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
       hdr->num_pairs = inc;
       hdr->num_items = inc * p.num_kv_heads;
       hdr->work_counter = 0;
-      hdr->num_split_seqs = s_nsl;
-      hdr->max_nsplit = s_maxn;
     }
   }
   __syncthreads();
@@ -274,131 +263,7 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
   pdl_wait();
 }
 
-constexpr int kMergeThreads = 256;
-
-// Rows (sequence, query head) of the split sequences only, from the list the
-// planning kernel wrote. W warps per row for head_dim 128 (per pair of rows
-// for head_dim 64, a half-warp per row); each lane owns 4 consecutive
-// columns. Warp w of a row takes splits w, w + W, ...: its first 8 partials
-// are requested before the row's weights are known, every lane reads the
-// (m, l) pairs it needs itself (broadcast loads), and the W partial sums meet
-// in shared memory. W (a power of two up to 8) is picked from the largest
-// split count so a warp rarely sees more than 8 splits.
-template <int D>
-__global__ void __launch_bounds__(kMergeThreads) merge_kernel(MergeParams p) {
-  constexpr int VPR = D / 4;        // float4 columns per row = lanes per row
-  constexpr int RPW = 32 / VPR;     // rows per warp
-  constexpr int NW = kMergeThreads / 32;
-  __shared__ float4 s_acc[NW][32];
-  const WsHeader* hdr = reinterpret_cast<const WsHeader*>(p.ws);
-  const int2* slist = reinterpret_cast<const int2*>(p.ws + p.slist_off);
-  const float2* ml_all = reinterpret_cast<const float2*>(p.ws + p.ml_off);
-  const float4* po_all = reinterpret_cast<const float4*>(p.ws + p.o_off);
-  float4* out4 = reinterpret_cast<float4*>(p.out);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int cv = lane % VPR;
-  pdl_wait();   // every partial of the decode kernel is written and visible
-
-  const int Hq = p.num_q_heads;
-  const int total_rows = hdr->num_split_seqs * Hq;
-  const int maxn = hdr->max_nsplit;
-  int W = 1;
-  while (W < 8 && W * 8 < maxn) W *= 2;
-  const int wr = warp % W, grp = warp / W;
-  const int rows_per_cta = (NW / W) * RPW;
-  // a grid of a few CTAs per SM walks all row groups
-  for (int rbase = blockIdx.x * rows_per_cta; rbase < total_rows;
-       rbase += gridDim.x * rows_per_cta) {
-    const int lr = rbase + grp * RPW + lane / VPR;   // row of the split list
-    int n = 0;
-    size_t row = 0;
-    if (lr < total_rows) {
-      const int2 e = slist[lr / Hq];
-      n = e.y;
-      row = static_cast<size_t>(e.x) * Hq + lr % Hq;
-    }
-    int nw = n;   // loop bound shared by the rows of the warp
-#pragma unroll
-    for (int o = VPR; o < 32; o <<= 1) nw = max(nw, __shfl_xor_sync(0xffffffffu, nw, o));
-
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (nw > 1) {
-      const float2* ml = ml_all + row * p.max_splits;
-      const float4* src = po_all + row * p.max_splits * VPR + cv;
-      float4 v[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int sj = wr + W * j;
-        v[j] = sj < n ? __ldg(src + static_cast<size_t>(sj) * VPR)
-                      : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-      float M = -INFINITY;
-      for (int s = cv; s < nw; s += VPR)
-        if (s < n) M = fmaxf(M, ml[s].x);
-#pragma unroll
-      for (int o = VPR / 2; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-      float L = 0.f;
-      for (int s = cv; s < nw; s += VPR)
-        if (s < n) {
-          const float2 e = ml[s];
-          L += e.y * exp2f(e.x - M);
-        }
-#pragma unroll
-      for (int o = VPR / 2; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-      const float inv = n > 1 ? 1.0f / L : 0.f;
-      for (int i0 = 0;; i0 += 8) {
-        if (i0 > 0) {
-          if (wr + W * i0 >= nw) break;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int sj = wr + W * (i0 + j);
-            v[j] = sj < n ? __ldg(src + static_cast<size_t>(sj) * VPR)
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int sj = wr + W * (i0 + j);
-          const float w = sj < n ? exp2f(ml[sj].x - M) * inv : 0.f;
-          acc.x = fmaf(w, v[j].x, acc.x);
-          acc.y = fmaf(w, v[j].y, acc.y);
-          acc.z = fmaf(w, v[j].z, acc.z);
-          acc.w = fmaf(w, v[j].w, acc.w);
-        }
-      }
-    }
-    if (W == 1) {
-      if (n > 1) out4[row * VPR + cv] = acc;
-      continue;
-    }
-    s_acc[warp][lane] = acc;
-    __syncthreads();
-    if (wr == 0 && n > 1) {
-      for (int w = 1; w < W; ++w) {
-        const float4 b = s_acc[warp + w][lane];
-        acc.x += b.x;
-        acc.y += b.y;
-        acc.z += b.z;
-        acc.w += b.w;
-      }
-      out4[row * VPR + cv] = acc;
-    }
-    __syncthreads();   // s_acc is reused by the next row group
-  }
-}
-
 }  // namespace
-
-cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream) {
-  if (p.max_splits <= 1 || p.num_seqs == 0) return cudaSuccess;
-  // at most 4 CTAs per SM: they fit beside a decode CTA, so all of them are
-  // resident (and past their launch) when the decode kernel finishes
-  const int rows = p.num_seqs * p.num_q_heads;
-  const dim3 grid(rows < 4 * num_sms() ? rows : 4 * num_sms());
-  if (p.head_dim == 64) return launch_pdl(merge_kernel<64>, grid, dim3(kMergeThreads), 0, stream, p);
-  if (p.head_dim == 128) return launch_pdl(merge_kernel<128>, grid, dim3(kMergeThreads), 0, stream, p);
-  return cudaErrorInvalidValue;
-}
 
 cudaError_t launch_plan(const PlanParams& p, cudaStream_t stream) {
   // a thread per sequence

@@ -1,12 +1,14 @@
 // Layout of the caller-provided decode workspace (shared by host and device
 // code). All offsets are multiples of 256 bytes from the workspace start.
 //
-//   [header 256 B][work pairs][splits per sequence][split-sequence list]
+//   [header 256 B][work pairs][splits per sequence][merge counters]
 //   [partial (m, l)][partial o]
 //
 // The header holds the device status word (first 4 bytes), the work counter
 // the persistent decode kernels claim items from, and the plan the planning
-// kernel chose (split size, number of items). Partial results are indexed
+// kernel chose (split size, number of items). A merge counter per
+// (sequence, KV head) counts the finished pieces of a split sequence; the
+// last piece merges them. Partial results are indexed
 // [sequence][query head][split].
 #pragma once
 
@@ -22,9 +24,7 @@ struct WsHeader {
   int32_t num_pairs;     // (sequence, split) pairs
   int32_t split_tokens;  // tokens per split chosen for this call
   int32_t max_splits;    // split capacity per sequence in this workspace
-  int32_t num_split_seqs;  // sequences cut into more than one piece (merge list length)
-  int32_t max_nsplit;      // largest piece count of a split sequence (0: none split)
-  int32_t reserved[56];
+  int32_t reserved[58];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
@@ -52,7 +52,7 @@ inline int32_t auto_min_split(int32_t max_ctx) {
 
 struct WsLayout {
   int32_t max_splits;
-  size_t pairs_off, nsplit_off, slist_off, ml_off, o_off, total;
+  size_t pairs_off, nsplit_off, cnt_off, ml_off, o_off, total;
 };
 
 inline WsLayout ws_layout(int32_t num_seqs, int32_t num_q_heads,
@@ -71,8 +71,8 @@ inline WsLayout ws_layout(int32_t num_seqs, int32_t num_q_heads,
   off += align256(B * ms * 16);
   w.nsplit_off = off;
   off += align256(B * 4);
-  w.slist_off = off;   // (sequence, pieces) of every split sequence
-  off += align256(B * 8);
+  w.cnt_off = off;   // merge counters [sequence][KV head] (KV heads <= query heads)
+  off += align256(B * H * 4);
   w.ml_off = off;
   off += align256(B * H * ms * 8);
   w.o_off = off;

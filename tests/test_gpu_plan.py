@@ -40,12 +40,8 @@ def read_plan(ws, num_seqs):
     pairs = raw[256:256 + 16 * num_pairs].view(np.int32).reshape(num_pairs, 4)
     nsplit_off = 256 + _align256(num_seqs * max_splits * 16)
     nsplit = raw[nsplit_off:nsplit_off + 4 * num_seqs].view(np.int32)
-    num_split_seqs, max_nsplit = int(hdr[6]), int(hdr[7])
-    slist_off = nsplit_off + _align256(num_seqs * 4)
-    slist = raw[slist_off:slist_off + 8 * num_split_seqs].view(np.int32).reshape(-1, 2)
     return dict(status=status, num_items=num_items, split_tokens=split_tokens,
-                max_splits=max_splits, pairs=pairs, nsplit=nsplit, slist=slist,
-                max_nsplit=max_nsplit)
+                max_splits=max_splits, pairs=pairs, nsplit=nsplit)
 
 
 def check_plan(plan, lens, num_kv_heads, explicit_split=0):
@@ -75,11 +71,6 @@ def check_plan(plan, lens, num_kv_heads, explicit_split=0):
         if explicit_split:
             assert np.all(e - b <= explicit_split)
             assert np.all((e - b)[:-1] == explicit_split)
-    # the merge list: exactly the sequences with more than one piece
-    split = {i: int(nsplit[i]) for i in range(len(lens)) if nsplit[i] > 1}
-    listed = {int(s): int(n) for s, n in plan["slist"]}
-    assert len(listed) == len(plan["slist"]) and listed == split
-    assert plan["max_nsplit"] == max(split.values(), default=0)
 
 
 @pytest.mark.parametrize("name,split", [("gqa", 0), ("long", 0), ("mha", 0), ("prefix_cow", 0),
