@@ -316,6 +316,89 @@ def time_e2e(b, ops, ws, split, path, stream, K, W):
     return e0.elapsed_time(e1) / K, h2d, d2h
 
 
+def time_graph(fn, stream, K):
+    """Average device time of fn (captured once in a CUDA graph), K replays
+    back to back between two events."""
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) / K
+
+
+def next_rows(ops, stream, rank):
+    """Measurements beyond the decode step: the paged-vs-contiguous cost of the
+    block table (same kernel, same lengths, blocks adjacent instead of
+    shuffled), a prefill-sized KV write, and block swap-out / swap-in between
+    the device pools and pinned host memory."""
+    from paged_kv_cache_339_b200 import workloads as W
+    res = {}
+    for name, mk in (("mha", W.mha), ("gqa", W.gqa)):
+        row = {}
+        for placement in ("shuffled", "contiguous"):
+            b = mk("cuda", seed={"mha": 1002, "gqa": 1003}[name] + 100 * rank,
+                   contiguous=placement == "contiguous")
+            B, Hq, D = b.q.shape
+            ws = ops.decode_workspace(B, Hq, D, b.max_context_len, b.block_size, 0)
+            out = torch.empty((B, Hq, D), dtype=torch.float32, device="cuda")
+            ms = time_decode_only(b, ops, out, ws, 0, ops.PA_PATH_AUTO, stream, 20)
+            row[placement + "_decode_gbps"] = round(b.kv_bytes_logical() / (ms * 1e-3) / 1e9, 1)
+            del b, ws, out
+            torch.cuda.empty_cache()
+        row["table_cost_pct"] = round(
+            100.0 * (1.0 - row["shuffled_decode_gbps"] / row["contiguous_decode_gbps"]), 2)
+        res["paged_vs_contiguous_" + name] = row
+    # prefill-sized write: T tokens of the MHA shape into distinct slots
+    T, H, D, BS, NB = 16384, 32, 128, 16, 2048
+    kc = torch.zeros((NB, H, BS, D), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    key = torch.randn((T, H, D), device="cuda").to(torch.bfloat16)
+    val = torch.randn((T, H, D), device="cuda").to(torch.bfloat16)
+    slots = torch.randperm(NB * BS, device="cuda")[:T].to(torch.int64)
+    ms = time_graph(lambda: ops.pa_write_kv(kc, vc, key, val, slots, stream=stream), stream, 20)
+    nbytes = 2 * T * H * D * 2
+    res["prefill_write"] = {"tokens": T, "bytes_written": nbytes,
+                            "gbps_written": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                            "ms": round(ms, 4)}
+    # swap: P blocks of that pool out to pinned host memory and back
+    P = 1024
+    hk = torch.empty((P, H, BS, D), dtype=torch.bfloat16, pin_memory=True)
+    hv = torch.empty_like(hk, pin_memory=True)
+    src = torch.randperm(NB, device="cuda")[:P].to(torch.int64)
+    pairs_out = torch.stack([src, torch.arange(P, device="cuda")], 1).contiguous()
+    pairs_in = torch.stack([torch.arange(P, device="cuda"), src], 1).contiguous()
+    blk = 2 * H * BS * D * 2
+    sw = {}
+    for label, pairs, d in (("out", pairs_out, ops.PA_SWAP_OUT), ("in", pairs_in, ops.PA_SWAP_IN)):
+        with torch.cuda.stream(stream):
+            ops.pa_swap_blocks(kc, vc, hk, hv, pairs, d, stream=stream)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(5):
+                ops.pa_swap_blocks(kc, vc, hk, hv, pairs, d, stream=stream)
+            e1.record(stream)
+            torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / 5
+        sw[label + "_gbps"] = round(P * blk / (ms * 1e-3) / 1e9, 1)
+    res["swap"] = dict(blocks=P, bytes=P * blk, **sw)
+    del kc, vc, key, val, hk, hv
+    torch.cuda.empty_cache()
+    return res
+
+
 def kernel_source_hash():
     """Hash of the decode kernels' sources (the traffic figure is only reported
     while it was measured on these exact sources)."""
@@ -465,6 +548,7 @@ def run_ours(args, rank, world, local):
                            "status": ops.pa_decode_status(ws2, stream)}
             del ws2, out2
         res["secondary"] = sec
+        res["next"] = next_rows(ops, stream, rank)
         del b
         torch.cuda.empty_cache()
         b = make_batch(args.workload, "cuda", rank, args.block_size)

@@ -9,10 +9,12 @@
  * borrowed from operating systems"; glossary "Paged attention", section "What
  * is Paged Attention?").
  *
- * Three device operations:
+ * Four device operations:
  *   pa_write_kv    - store each new token's K and V into its slot;
  *   pa_copy_blocks - copy whole blocks: the copy-on-write step when a sequence
  *                    diverges inside a shared block;
+ *   pa_swap_blocks - move whole blocks between the device pools and a pool in
+ *                    host memory (preemption by swapping);
  *   pa_decode      - single-query attention of every sequence over its paged
  *                    context.
  *
@@ -123,6 +125,39 @@ pa_status pa_write_kv(const pa_kv_cache* cache, const void* key,
  */
 pa_status pa_copy_blocks(const pa_kv_cache* cache, const int64_t* block_pairs,
                          int32_t num_pairs, pa_stream_t stream);
+
+/* Direction of pa_swap_blocks. */
+typedef enum {
+  PA_SWAP_OUT = 0, /* device pools -> host pool */
+  PA_SWAP_IN = 1   /* host pool -> device pools */
+} pa_swap_dir;
+
+/*
+ * pa_swap_blocks - move whole blocks between the device pools and a host pool.
+ *
+ * When memory runs out, the server preempts: it evicts a sequence and later
+ * recomputes or swaps its blocks back ("Paged Attention: Virtual Memory for
+ * the KV Cache", section "What it does not fix"). This is the swap: for each
+ * pair p, with (src, dst) = (block_pairs[2p], block_pairs[2p + 1]),
+ *   PA_SWAP_OUT: host_k[dst] = k_cache[src]; host_v[dst] = v_cache[src]
+ *   PA_SWAP_IN:  k_cache[dst] = host_k[src]; v_cache[dst] = host_v[src]
+ * all heads of the block, bytes unchanged (the host pool keeps the cache's
+ * in-block order; a block is num_kv_heads * block_size * head_dim elements).
+ *
+ *   host_k, host_v  page-locked host memory mapped into the device address
+ *                   space (cudaHostAlloc / cudaHostRegister with the mapped
+ *                   flag, or a pinned PyTorch tensor), host_num_blocks blocks
+ *                   each, 16-byte aligned; PA_ERR_INVALID_ARG for memory the
+ *                   device cannot address
+ *   block_pairs     device int64 [num_pairs][2]; pairs with an index outside
+ *                   its pool are skipped; every dst distinct
+ *   direction       a pa_swap_dir
+ * One kernel reads (or writes) the host pool directly over the host link; no
+ * copy engine call per block. num_pairs == 0 is a no-op returning PA_OK.
+ */
+pa_status pa_swap_blocks(const pa_kv_cache* cache, void* host_k, void* host_v,
+                         int32_t host_num_blocks, const int64_t* block_pairs,
+                         int32_t num_pairs, int32_t direction, pa_stream_t stream);
 
 /* Kernel choice for pa_decode (see pa_decode_options.path). */
 typedef enum {

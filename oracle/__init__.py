@@ -2,8 +2,9 @@
 
 from .paged_attention import (ORACLE, PagedAttentionOracle, attend, copy_blocks,
                               decode, decode_one, gather, logical_pool, merge,
-                              partial, physical_pool, tile_offset, write_kv)
+                              partial, physical_pool, swap_blocks, tile_offset,
+                              write_kv)
 
 __all__ = ["ORACLE", "PagedAttentionOracle", "attend", "copy_blocks", "decode",
            "decode_one", "gather", "logical_pool", "merge", "partial",
-           "physical_pool", "tile_offset", "write_kv"]
+           "physical_pool", "swap_blocks", "tile_offset", "write_kv"]

@@ -45,6 +45,10 @@ Pages: "Paged Attention: Virtual Memory for the KV Cache" (P1),
 * Copy-on-write: a sequence that diverges inside a shared block first gets its
   own copy of that block (P1, "Sharing comes almost for free"; P2, "Virtual
   Memory as the Blueprint").
+* Swapping blocks out to host memory and back: when memory runs out the
+  server evicts a sequence and later recomputes or swaps its blocks back (P1,
+  "What it does not fix"). A swap is a block copy between the device pools
+  and a host pool, in either direction.
 * Split-context partial softmax and merge: not on the pages. It is the exact
   algebraic regrouping of the softmax sum over a partition of the tokens; the
   oracle keeps it only to pin that regrouping (see ``partial`` / ``merge``).
@@ -202,6 +206,25 @@ class PagedAttentionOracle:
         return k_out, v_out
 
 
+    def swap_blocks(self, dev_k: np.ndarray, dev_v: np.ndarray, host_k: np.ndarray,
+                    host_v: np.ndarray, pairs: np.ndarray, direction: int):
+        """Swap (P1, "What it does not fix"): direction 0 (out) copies device
+        block src to host block dst, direction 1 (in) host block src to device
+        block dst, both pools; pairs with an index outside its pool are
+        skipped. Returns new (dev_k, dev_v, host_k, host_v)."""
+        dk, dv, hk, hv = dev_k.copy(), dev_v.copy(), host_k.copy(), host_v.copy()
+        if direction == 0:
+            src_k, src_v, dst_k, dst_v = dev_k, dev_v, hk, hv
+        else:
+            src_k, src_v, dst_k, dst_v = host_k, host_v, dk, dv
+        for src, dst in np.asarray(pairs).reshape(-1, 2).tolist():
+            if not (0 <= src < len(src_k) and 0 <= dst < len(dst_k)):
+                continue
+            dst_k[dst] = src_k[src]
+            dst_v[dst] = src_v[src]
+        return dk, dv, hk, hv
+
+
 ORACLE = PagedAttentionOracle()
 
 # Module-level names for the common calls.
@@ -214,5 +237,6 @@ decode = ORACLE.decode
 decode_one = ORACLE.decode_one
 write_kv = ORACLE.write_kv
 copy_blocks = ORACLE.copy_blocks
+swap_blocks = ORACLE.swap_blocks
 partial = ORACLE.partial
 merge = ORACLE.merge

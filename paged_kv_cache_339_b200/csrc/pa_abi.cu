@@ -132,6 +132,44 @@ pa_status pa_copy_blocks(const pa_kv_cache* cache, const int64_t* block_pairs, i
   return e == cudaSuccess ? PA_OK : cuda_fail(e);
 }
 
+// Device address of page-locked host memory the device can reach; nullptr if
+// it cannot (pageable memory, or not mapped).
+static void* device_view_of_host(void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  if (a.type != cudaMemoryTypeHost) return nullptr;
+  return a.devicePointer;
+}
+
+pa_status pa_swap_blocks(const pa_kv_cache* cache, void* host_k, void* host_v,
+                         int32_t host_num_blocks, const int64_t* block_pairs, int32_t num_pairs,
+                         int32_t direction, pa_stream_t stream) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (num_pairs < 0 || host_num_blocks < 0) return PA_ERR_INVALID_ARG;
+  if (direction != PA_SWAP_OUT && direction != PA_SWAP_IN) return PA_ERR_INVALID_ARG;
+  if (num_pairs == 0) return PA_OK;
+  if (block_pairs == nullptr || host_k == nullptr || host_v == nullptr) return PA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(block_pairs) & 7u) || !aligned16(host_k) || !aligned16(host_v))
+    return PA_ERR_MISALIGNED;
+  void* hk = device_view_of_host(host_k);
+  void* hv = device_view_of_host(host_v);
+  if (hk == nullptr || hv == nullptr) return PA_ERR_INVALID_ARG;
+  const int64_t block_bytes = static_cast<int64_t>(cache->num_kv_heads) * cache->block_size *
+                              cache->head_dim * elem_bytes(cache->dtype);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e =
+      direction == PA_SWAP_OUT
+          ? launch_swap_blocks(hk, hv, cache->k_cache, cache->v_cache, block_pairs, num_pairs,
+                               block_bytes, cache->num_blocks, host_num_blocks, s)
+          : launch_swap_blocks(cache->k_cache, cache->v_cache, hk, hv, block_pairs, num_pairs,
+                               block_bytes, host_num_blocks, cache->num_blocks, s);
+  return e == cudaSuccess ? PA_OK : cuda_fail(e);
+}
+
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
                                 int32_t max_context_len, int32_t block_size,
                                 int32_t split_tokens) {

@@ -63,6 +63,9 @@ cudaError_t launch_copy_blocks(void* k_cache, void* v_cache,
                                const int64_t* pairs, int32_t num_pairs,
                                int64_t block_bytes, int32_t num_blocks,
                                cudaStream_t stream);
+cudaError_t launch_swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                               const int64_t* pairs, int32_t num_pairs, int64_t block_bytes,
+                               int32_t src_blocks, int32_t dst_blocks, cudaStream_t stream);
 
 int num_sms();
 

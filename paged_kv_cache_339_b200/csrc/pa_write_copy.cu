@@ -10,6 +10,10 @@
 // copy a diverging sequence gets of a shared block ("Sharing comes almost for
 // free").
 //
+// swap: the same block copy between the device pools and a host pool the
+// device can address (preemption by swapping, "What it does not fix"); the
+// kernel reads or writes host memory directly over the host link.
+//
 // Both are grid-stride loops over 16-byte vectors so consecutive threads touch
 // consecutive bytes of a row (coalesced on both sides). Indices outside the
 // pool are skipped, never dereferenced.
@@ -70,6 +74,23 @@ __global__ void __launch_bounds__(kCopyThreads)
   }
 }
 
+__global__ void __launch_bounds__(kCopyThreads)
+    swap_blocks_kernel(uint4* __restrict__ dk, uint4* __restrict__ dv,
+                       const uint4* __restrict__ sk, const uint4* __restrict__ sv,
+                       const int64_t* __restrict__ pairs, int32_t num_pairs, int64_t block_vecs,
+                       int32_t src_blocks, int32_t dst_blocks) {
+  const int64_t total = block_vecs * num_pairs;
+  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+       idx < total; idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t p = idx / block_vecs;
+    const int64_t v = idx - p * block_vecs;
+    const int64_t src = pairs[2 * p], dst = pairs[2 * p + 1];
+    if (src < 0 || src >= src_blocks || dst < 0 || dst >= dst_blocks) continue;
+    dk[dst * block_vecs + v] = sk[src * block_vecs + v];
+    dv[dst * block_vecs + v] = sv[src * block_vecs + v];
+  }
+}
+
 int grid_for(int64_t work) {
   const int64_t want = (work + kCopyThreads - 1) / kCopyThreads;
   const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
@@ -101,6 +122,16 @@ cudaError_t launch_copy_blocks(void* k_cache, void* v_cache,
                        stream>>>(static_cast<uint4*>(k_cache),
                                  static_cast<uint4*>(v_cache), pairs,
                                  num_pairs, block_vecs, num_blocks);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                               const int64_t* pairs, int32_t num_pairs, int64_t block_bytes,
+                               int32_t src_blocks, int32_t dst_blocks, cudaStream_t stream) {
+  const int64_t block_vecs = block_bytes / 16;
+  swap_blocks_kernel<<<grid_for(block_vecs * num_pairs), kCopyThreads, 0, stream>>>(
+      static_cast<uint4*>(dst_k), static_cast<uint4*>(dst_v), static_cast<const uint4*>(src_k),
+      static_cast<const uint4*>(src_v), pairs, num_pairs, block_vecs, src_blocks, dst_blocks);
   return cudaGetLastError();
 }
 

@@ -45,7 +45,8 @@ class PagedAttnError(RuntimeError):
 
 _lib = None
 
-EXPORTS = ("pa_write_kv", "pa_copy_blocks", "pa_decode_workspace_size", "pa_decode",
+EXPORTS = ("pa_write_kv", "pa_copy_blocks", "pa_swap_blocks", "pa_decode_workspace_size",
+           "pa_decode",
            "pa_decode_noalloc", "pa_decode_status", "pa_status_string", "pa_last_cuda_error",
            "pa_version")
 
@@ -64,6 +65,8 @@ def _load():
     lib.pa_write_kv.restype = ctypes.c_int
     lib.pa_copy_blocks.argtypes = [ctypes.POINTER(PaKvCache), i64p, i32, vp]
     lib.pa_copy_blocks.restype = ctypes.c_int
+    lib.pa_swap_blocks.argtypes = [ctypes.POINTER(PaKvCache), vp, vp, i32, i64p, i32, i32, vp]
+    lib.pa_swap_blocks.restype = ctypes.c_int
     lib.pa_decode_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
     lib.pa_decode_workspace_size.restype = ctypes.c_size_t
     lib.pa_decode.argtypes = [ctypes.POINTER(PaKvCache), vp, vp, vp, i32, vp, i32, i32, i32,
@@ -150,6 +153,32 @@ def pa_copy_blocks(k_cache, v_cache, block_pairs, stream=None) -> None:
     ptr = _dev_tensor(block_pairs, "block_pairs", torch.int64) if P else None
     st = _load().pa_copy_blocks(ctypes.byref(desc), ptr, P, _stream(stream))
     _check("pa_copy_blocks", st)
+
+
+PA_SWAP_OUT, PA_SWAP_IN = 0, 1
+
+
+def pa_swap_blocks(k_cache, v_cache, host_k, host_v, block_pairs, direction, stream=None) -> None:
+    """Move blocks between the device pools and a pinned host pool (host_k,
+    host_v: pinned CPU tensors shaped like the pools, any number of blocks).
+    PA_SWAP_OUT: host[dst] = device[src]; PA_SWAP_IN: device[dst] = host[src],
+    for every (src, dst) row of the int64 [P, 2] device tensor block_pairs."""
+    desc = kv_cache_desc(k_cache, v_cache)
+    for name, t in (("host_k", host_k), ("host_v", host_v)):
+        if not isinstance(t, torch.Tensor) or t.is_cuda or not t.is_pinned():
+            raise TypeError(f"{name} must be a pinned CPU tensor")
+        if not t.is_contiguous() or t.dtype != k_cache.dtype or t.shape[1:] != k_cache.shape[1:]:
+            raise ValueError(f"{name} must be contiguous [blocks, {', '.join(map(str, k_cache.shape[1:]))}] "
+                             f"{k_cache.dtype}")
+    if host_k.shape != host_v.shape:
+        raise ValueError("host_k and host_v must have the same shape")
+    P = block_pairs.shape[0] if block_pairs.numel() else 0
+    if P and tuple(block_pairs.shape) != (P, 2):
+        raise ValueError("block_pairs must be [num_pairs, 2]")
+    ptr = _dev_tensor(block_pairs, "block_pairs", torch.int64) if P else None
+    st = _load().pa_swap_blocks(ctypes.byref(desc), host_k.data_ptr(), host_v.data_ptr(),
+                                host_k.shape[0], ptr, P, int(direction), _stream(stream))
+    _check("pa_swap_blocks", st)
 
 
 def pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, block_size,

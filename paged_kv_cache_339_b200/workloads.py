@@ -153,10 +153,15 @@ def _assemble(name, dtype, BS, Hq, Hkv, D, lens, tables, num_blocks, gen, seed,
         cow_pairs=pairs.to(device), meta=meta or {})
 
 
-def _place(lens, BS, num_blocks, gen):
+def _place(lens, BS, num_blocks, gen, contiguous=False):
     """Hand out physical blocks from a seeded permutation of the pool, in
-    sequence order; returns one table per sequence."""
+    sequence order; returns one table per sequence. contiguous=True hands
+    them out in pool order instead (each sequence's blocks adjacent, for the
+    paged-vs-contiguous comparison); the permutation is drawn either way so
+    every later draw is the same."""
     perm = torch.randperm(num_blocks, generator=gen).tolist()
+    if contiguous:
+        perm = list(range(num_blocks))
     tables, k = [], 0
     for L in lens:
         nb = (L + BS - 1) // BS
@@ -183,15 +188,16 @@ def tiny(device="cpu", seed=1001):
 
 def mha(device="cpu", seed=1002, num_seqs=64, num_heads=32, head_dim=128,
         min_len=128, max_len=2048, block_size=16, num_blocks=16384,
-        dtype=torch.bfloat16):
+        dtype=torch.bfloat16, contiguous=False):
     """MHA decode step: context lengths uniform in [min_len, max_len], blocks
     drawn from a shuffled pool."""
     gen = torch.Generator().manual_seed(seed)
     lens = torch.randint(min_len, max_len + 1, (num_seqs,), generator=gen).tolist()
     need = sum((L + block_size - 1) // block_size for L in lens)
     num_blocks = max(num_blocks, need)
-    tables = _place(lens, block_size, num_blocks, gen)
+    tables = _place(lens, block_size, num_blocks, gen, contiguous)
     name = f"mha_b{num_seqs}_h{num_heads}_d{head_dim}_bs{block_size}_ctx{min_len}-{max_len}"
+    name += "_contiguous" if contiguous else ""
     return _assemble(name, dtype, block_size, num_heads, num_heads, head_dim,
                      lens, tables, num_blocks, gen, seed, device)
 
@@ -207,16 +213,16 @@ def lognormal_lens(num_seqs, mean, sigma, lo, hi, gen):
 
 def gqa(device="cpu", seed=1003, num_seqs=256, num_q_heads=32, num_kv_heads=8,
         head_dim=128, mean_len=512, sigma=1.0, min_len=16, max_len=4096,
-        block_size=16, dtype=torch.bfloat16, free_frac=0.10):
+        block_size=16, dtype=torch.bfloat16, free_frac=0.10, contiguous=False):
     """GQA high-concurrency decode: log-normal lengths, pool sized to fit all
     sequences plus `free_frac` free blocks, shuffled."""
     gen = torch.Generator().manual_seed(seed)
     lens = lognormal_lens(num_seqs, mean_len, sigma, min_len, max_len, gen)
     need = sum((L + block_size - 1) // block_size for L in lens)
     num_blocks = int(math.ceil(need * (1.0 + free_frac)))
-    tables = _place(lens, block_size, num_blocks, gen)
+    tables = _place(lens, block_size, num_blocks, gen, contiguous)
     name = (f"gqa_b{num_seqs}_hq{num_q_heads}_hkv{num_kv_heads}_d{head_dim}"
-            f"_bs{block_size}_lognormal{mean_len}")
+            f"_bs{block_size}_lognormal{mean_len}") + ("_contiguous" if contiguous else "")
     return _assemble(name, dtype, block_size, num_q_heads, num_kv_heads,
                      head_dim, lens, tables, num_blocks, gen, seed, device)
 

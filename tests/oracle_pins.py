@@ -340,6 +340,39 @@ def check_copy_blocks(orc):
         assert np.array_equal(k2[b], kc[b]) and np.array_equal(v2[b], vc[b])
 
 
+def check_swap_blocks(orc):
+    """Swap out copies device blocks to host blocks, swap in copies them back;
+    the other side and every untouched block are unchanged, pairs outside
+    either pool are skipped, and a sequence evicted and brought back into
+    other blocks (its table rewritten) reads the same context ("What it does
+    not fix": preemption by swapping)."""
+    r = _rng(18)
+    NB, NH, H, BS, D = 6, 4, 2, 4, 3
+    dk = r.integers(0, 1 << 16, size=(NB, H, BS, D), dtype=np.uint16)
+    dv = r.integers(0, 1 << 16, size=(NB, H, BS, D), dtype=np.uint16)
+    hk = r.integers(0, 1 << 16, size=(NH, H, BS, D), dtype=np.uint16)
+    hv = r.integers(0, 1 << 16, size=(NH, H, BS, D), dtype=np.uint16)
+    out_pairs = np.array([[1, 3], [4, 0], [9, 1], [2, 7], [-1, 2]])
+    dk1, dv1, hk1, hv1 = orc.swap_blocks(dk, dv, hk, hv, out_pairs, 0)
+    assert np.array_equal(dk1, dk) and np.array_equal(dv1, dv)
+    assert np.array_equal(hk1[3], dk[1]) and np.array_equal(hv1[3], dv[1])
+    assert np.array_equal(hk1[0], dk[4]) and np.array_equal(hv1[0], dv[4])
+    for b in (1, 2):   # skipped pairs left the host blocks alone
+        assert np.array_equal(hk1[b], hk[b]) and np.array_equal(hv1[b], hv[b])
+    in_pairs = np.array([[3, 5], [0, 2], [5, 0], [1, 6]])
+    dk2, dv2, hk2, hv2 = orc.swap_blocks(dk1, dv1, hk1, hv1, in_pairs, 1)
+    assert np.array_equal(hk2, hk1) and np.array_equal(hv2, hv1)
+    assert np.array_equal(dk2[5], dk[1]) and np.array_equal(dv2[5], dv[1])
+    assert np.array_equal(dk2[2], dk[4]) and np.array_equal(dv2[2], dv[4])
+    for b in (0, 1, 3, 4):
+        assert np.array_equal(dk2[b], dk[b]) and np.array_equal(dv2[b], dv[b])
+    # evict a 6-token sequence held in blocks [1, 4], bring it back into [5, 2]
+    L = 6
+    before = orc.gather(dk, np.array([1, 4]), L)
+    after = orc.gather(dk2, np.array([5, 2]), L)
+    assert np.array_equal(before, after)
+
+
 # ---------------------------------------------------------------------------
 # Split-context regrouping
 # ---------------------------------------------------------------------------
@@ -385,5 +418,5 @@ ALL_CHECKS = [
     check_identity_table_is_contiguous, check_permutation_invariance,
     check_gqa_is_repeated_mha, check_context_len_bounds, check_prefix_sharing,
     check_copy_on_write, check_write_layout, check_write_then_gather,
-    check_copy_blocks, check_merge_partition, check_tile_layout,
+    check_copy_blocks, check_swap_blocks, check_merge_partition, check_tile_layout,
 ]

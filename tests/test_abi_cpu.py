@@ -88,6 +88,15 @@ def test_host_side_rejections(lib):
     assert lib.pa_copy_blocks(ctypes.byref(c), 0x3000, 0, None) == ops.PA_OK
     assert lib.pa_copy_blocks(ctypes.byref(c), None, 2, None) == ops.PA_ERR_INVALID_ARG
     assert lib.pa_copy_blocks(ctypes.byref(c), 0x3004, 2, None) == ops.PA_ERR_MISALIGNED
+    # swap: checked before the host pool's memory type is asked for
+    sw = lib.pa_swap_blocks
+    assert sw(ctypes.byref(c), 0x8000, 0x9000, 4, 0x3000, 0, 0, None) == ops.PA_OK
+    assert sw(ctypes.byref(c), 0x8000, 0x9000, 4, 0x3000, 2, 2, None) == ops.PA_ERR_INVALID_ARG
+    assert sw(ctypes.byref(c), 0x8000, 0x9000, -1, 0x3000, 2, 0, None) == ops.PA_ERR_INVALID_ARG
+    assert sw(ctypes.byref(c), None, 0x9000, 4, 0x3000, 2, 1, None) == ops.PA_ERR_INVALID_ARG
+    assert sw(ctypes.byref(c), 0x8000, 0x9000, 4, None, 2, 1, None) == ops.PA_ERR_INVALID_ARG
+    assert sw(ctypes.byref(c), 0x8008, 0x9000, 4, 0x3000, 2, 1, None) == ops.PA_ERR_MISALIGNED
+    assert sw(ctypes.byref(c), 0x8000, 0x9000, 4, 0x3004, 2, 1, None) == ops.PA_ERR_MISALIGNED
 
 
 def test_workspace_size_layout(lib):

@@ -130,7 +130,24 @@ class TileGroupOf8(PagedAttentionOracle):
         return ((t // sh) * nh + d // 64) * sh * 64 + (t % sh) * 64 + d % 64
 
 
-MUTANTS = [TileHalvesSwapped, TileGroupOf8, NoScale, NegatedScores, KeysValuesSwapped, GqaModulo,
+class SwapDirectionIgnored(PagedAttentionOracle):
+    def swap_blocks(self, dev_k, dev_v, host_k, host_v, pairs, direction):
+        return super().swap_blocks(dev_k, dev_v, host_k, host_v, pairs, 0)
+
+
+class SwapPairsReversed(PagedAttentionOracle):
+    def swap_blocks(self, dev_k, dev_v, host_k, host_v, pairs, direction):
+        return super().swap_blocks(dev_k, dev_v, host_k, host_v,
+                                   np.asarray(pairs)[:, ::-1], direction)
+
+
+class SwapKeysOnly(PagedAttentionOracle):
+    def swap_blocks(self, dev_k, dev_v, host_k, host_v, pairs, direction):
+        dk, _, hk, _ = super().swap_blocks(dev_k, dev_v, host_k, host_v, pairs, direction)
+        return dk, dev_v.copy(), hk, host_v.copy()
+
+
+MUTANTS = [SwapDirectionIgnored, SwapPairsReversed, SwapKeysOnly, TileHalvesSwapped, TileGroupOf8, NoScale, NegatedScores, KeysValuesSwapped, GqaModulo,
            GatherIndexSwap, GatherWrongOffset, ContextOffByOne,
            NoMaxSubtraction, NoNormalisation, WriteSlotSwap, WriteKeyIntoBoth,
            WriteNegativeSlotWraps, CopyReversed, MergeWithoutRescale,
