@@ -281,38 +281,69 @@ def time_decode_only(b, ops, out, ws, split, path, stream, K, use_graph=True):
 
 def time_e2e(b, ops, ws, split, path, stream, K, W):
     """Same metric through the public API from pinned host buffers: every step
-    copies its inputs host->device and reads the result back."""
+    copies its inputs host->device and reads its result back. Two buffer sets
+    and a copy stream pipeline it the way a serving loop would: step i+1's
+    inputs go up while step i computes, step i's result comes back as soon as
+    it is done. All copies are inside the timed region."""
     host = {k: getattr(b, k).cpu().pin_memory() for k in
             ("q", "key", "value", "slot_mapping", "block_tables", "context_lens", "cow_pairs")}
-    dev = {k: torch.empty_like(v, device="cuda") for k, v in host.items()}
-    out = torch.empty(b.q.shape, dtype=torch.float32, device="cuda")
-    out_h = torch.empty(b.q.shape, dtype=torch.float32).pin_memory()
+    dev = [{k: torch.empty_like(v, device="cuda") for k, v in host.items()} for _ in range(2)]
+    out = [torch.empty(b.q.shape, dtype=torch.float32, device="cuda") for _ in range(2)]
+    out_h = [torch.empty(b.q.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = out_h.numel() * 4
+    d2h = out_h[0].numel() * 4
     max_ctx = b.max_context_len
+    cs = torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+    up = [ev(), ev()]      # inputs of a slot are on the device
+    done = [ev(), ev()]    # the step that used a slot has finished
 
-    def step():
-        for k in host:
-            dev[k].copy_(host[k], non_blocking=True)
-        if dev["cow_pairs"].numel():
-            ops.pa_copy_blocks(b.k_cache, b.v_cache, dev["cow_pairs"], stream=stream)
-        ops.pa_write_kv(b.k_cache, b.v_cache, dev["key"], dev["value"], dev["slot_mapping"],
-                        stream=stream)
-        ops.pa_decode(out, dev["q"], b.k_cache, b.v_cache, dev["block_tables"],
-                      dev["context_lens"], max_ctx, b.scale, ws, split_tokens=split, path=path,
-                      stream=stream)
-        out_h.copy_(out, non_blocking=True)
+    def upload(i):
+        sl = i & 1
+        with torch.cuda.stream(cs):
+            cs.wait_event(done[sl])          # the step two back has released the slot
+            for k in host:
+                dev[sl][k].copy_(host[k], non_blocking=True)
+            up[sl].record(cs)
 
-    with torch.cuda.stream(stream):
-        for _ in range(W):
-            step()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(K):
-            step()
-        e1.record(stream)
-        torch.cuda.synchronize()
+    def compute(i):
+        sl, d = i & 1, dev[i & 1]
+        with torch.cuda.stream(stream):
+            stream.wait_event(up[sl])
+            if d["cow_pairs"].numel():
+                ops.pa_copy_blocks(b.k_cache, b.v_cache, d["cow_pairs"], stream=stream)
+            ops.pa_write_kv(b.k_cache, b.v_cache, d["key"], d["value"], d["slot_mapping"],
+                            stream=stream)
+            ops.pa_decode(out[sl], d["q"], b.k_cache, b.v_cache, d["block_tables"],
+                          d["context_lens"], max_ctx, b.scale, ws, split_tokens=split,
+                          path=path, stream=stream)
+            done[sl].record(stream)
+
+    def download(i):
+        sl = i & 1
+        with torch.cuda.stream(cs):
+            cs.wait_event(done[sl])
+            out_h[sl].copy_(out[sl], non_blocking=True)
+
+    def run(n):
+        upload(0)
+        for i in range(n):
+            compute(i)
+            if i + 1 < n:
+                upload(i + 1)
+            download(i)
+
+    for e in done:
+        e.record(stream)
+    run(W)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    cs.wait_event(e0)
+    run(K)
+    stream.wait_stream(cs)
+    e1.record(stream)
+    torch.cuda.synchronize()
     return e0.elapsed_time(e1) / K, h2d, d2h
 
 
