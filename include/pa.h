@@ -168,17 +168,22 @@ typedef enum {
 
 typedef struct {
   /* Tokens per work item (context split). 0 = chosen on the device from the
-     actual context lengths (a multiple of 128, at least 256, and at most 64
-     splits per sequence for max_context_len). Otherwise a positive multiple
-     of block_size with ceil(max_context_len / split_tokens) <= 256. */
+     actual context lengths: pieces of up to one item stream's share of the
+     whole batch (a multiple of 128, at least 256 and at least
+     max_context_len / 64), listed longest first, with the ends of the
+     sequences cut finer when the batch has too little short work to even out
+     the finish. Otherwise a positive multiple of block_size with
+     ceil(max_context_len / split_tokens) <= 256, every piece split_tokens
+     long except each sequence's last. */
   int32_t split_tokens;
   int32_t path;        /* a pa_decode_path */
 } pa_decode_options;
 
 /*
  * pa_decode_workspace_size - bytes of device workspace pa_decode needs for the
- * given shapes (work list, one partial result per (sequence, query head,
- * split), status word). split_tokens as in pa_decode_options.
+ * given shapes (status word and plan, work list, piece counts, a merge counter
+ * per (sequence, KV head), one partial result per (sequence, query head,
+ * piece)). split_tokens as in pa_decode_options.
  */
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
                                 int32_t head_dim, int32_t max_context_len,
