@@ -4,8 +4,8 @@
  * The KV cache is a pool of fixed-size physical blocks, each holding the keys
  * and values of `block_size` tokens; every sequence keeps a block table that
  * lists, in logical order, which physical blocks hold it, and the attention
- * kernel follows that table instead of assuming the sequence is laid out end
- * to end ("Paged Attention: Virtual Memory for the KV Cache", section "The fix
+ * kernel follows that table instead of assuming one unbroken stretch of
+ * memory per sequence ("Paged Attention: Virtual Memory for the KV Cache", section "The fix
  * borrowed from operating systems"; glossary "Paged attention", section "What
  * is Paged Attention?").
  *
@@ -200,7 +200,8 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
  *   s_j = scale * <q[i][h], K_j>
  *   out[i][h] = sum_j exp(s_j - max s) V_j / sum_j exp(s_j - max s)
  * with bt = block_tables, L_i = context_lens[i]; L_i == 0 gives a zero row.
- * The sequence is read through its table as if it were contiguous (glossary
+ * The sequence is read through its table in logical order, as though its
+ * tokens sat back to back (glossary
  * "Paged attention", "What is Paged Attention?"). The pages never write the
  * formula; this is the plain scaled dot-product reading.
  *

@@ -29,7 +29,8 @@ Pages: "Paged Attention: Virtual Memory for the KV Cache" (P1),
 * Block table. Each sequence keeps an ordered list of the physical blocks that
   hold it; logical token ``j`` lives in block ``table[j // block_size]`` at
   offset ``j % block_size`` (P1, "The fix borrowed from operating systems").
-* The kernel reads the logical sequence as if it were contiguous (P3, "What is
+* The kernel walks the logical sequence in order, as though its tokens sat
+  back to back (P3, "What is
   Paged Attention?"). So the oracle gathers each sequence into one contiguous
   array and then runs ordinary attention on it.
 * Attention formula. The pages name the operation but never write it (P2's
@@ -38,9 +39,8 @@ Pages: "Paged Attention: Virtual Memory for the KV Cache" (P1),
   ``o = softmax(scale * q . K^T) . V`` over the first ``context_len`` tokens,
   query head ``h`` using KV head ``h // (num_q_heads // num_kv_heads)``
   (grouped-query attention is named in P1, "What it does not fix").
-* Writing a token into its slot: a request fills its current block and asks for
-  another only when it needs one (P1, "The fix borrowed from operating
-  systems"); slot ``s`` addresses block ``s // block_size``, offset
+* Writing a token into its slot: a request takes a new block only once its
+  current one is full (P1, "The fix borrowed from operating systems"); slot ``s`` addresses block ``s // block_size``, offset
   ``s % block_size``. A negative slot means "no write" (padding).
 * Copy-on-write: a sequence that diverges inside a shared block first gets its
   own copy of that block (P1, "Sharing comes almost for free"; P2, "Virtual
@@ -103,7 +103,7 @@ class PagedAttentionOracle:
         """Contiguous ``[context_len, num_kv_heads, head_dim]`` view of one
         sequence: logical token j comes from block table_row[j // block_size],
         offset j % block_size (P3, "What is Paged Attention?": the sequence is
-        read as if it were contiguous)."""
+        read in logical order, as though stored back to back)."""
         block_size = cache.shape[2]
         j = np.arange(context_len)
         blocks = np.asarray(table_row)[j // block_size]

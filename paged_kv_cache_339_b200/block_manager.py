@@ -127,8 +127,9 @@ class BlockManager:
         return [r + [0] * (stride - len(r)) for r in rows]
 
     def reserved_unused_tokens(self, seq_id: int) -> int:
-        """Slots held but not used by seq_id: at most block_size - 1 ("at most
-        one partly filled block per request")."""
+        """Slots held but not used by seq_id: at most block_size - 1 (only a
+        sequence's last block can be partly used, P1 "The fix borrowed from
+        operating systems")."""
         return len(self.tables[seq_id]) * self.block_size - self.lengths[seq_id]
 
     def check_invariants(self) -> None:

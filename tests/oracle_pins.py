@@ -159,7 +159,8 @@ def check_convex_combination(orc):
 def check_identity_table_is_contiguous(orc):
     """Identity table over a pool laid out from a contiguous array gathers the
     array back exactly, ragged last block included (glossary 'What is Paged
-    Attention?': the sequence is read as if contiguous)."""
+    Attention?': the sequence is read in logical order, as though stored back
+    to back)."""
     r = _rng(8)
     for L, BS in ((1, 4), (13, 4), (16, 16), (33, 16), (70, 8)):
         X = r.normal(size=(L, 3, 5))

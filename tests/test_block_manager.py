@@ -29,7 +29,8 @@ def test_incremental_allocation_and_slots():
 
 
 def test_waste_at_most_one_partial_block():
-    """'Waste falls to at most one partly filled block per request'."""
+    """Only a sequence's last block can be partly used, so its unused slots
+    stay below one block (P1, 'The fix borrowed from operating systems')."""
     rnd = random.Random(0)
     bm = BlockManager(num_blocks=4000, block_size=16)
     for s in range(50):
