@@ -299,6 +299,43 @@ def long_context(device="cpu", seed=1005, num_seqs=8, num_q_heads=64,
                      head_dim, lens, tables, num_blocks, gen, seed, device)
 
 
+def random_batch(device="cpu", seed=0, tensor_core_shape=False):
+    """A small decode step with randomly drawn shapes, for broad parity
+    coverage: dtype, head_dim 64/128, block size 8/16/32, 1-3 KV heads,
+    1-16 query heads per KV head, 1-6 sequences whose lengths mix the edge
+    cases (0, 1, a block boundary +- 1) with random lengths up to 700.
+    tensor_core_shape=True draws only shapes the tensor-core kernel takes
+    (16-bit, head_dim 128, 4-16 query heads per KV head, >= 16 query rows)."""
+    gen = torch.Generator().manual_seed((6000 if tensor_core_shape else 5000) + seed)
+    pick = lambda xs: xs[int(torch.randint(len(xs), (1,), generator=gen).item())]
+    if tensor_core_shape:
+        dtype = pick([torch.float16, torch.bfloat16])
+        D = 128
+    else:
+        dtype = pick([torch.float32, torch.float16, torch.bfloat16])
+        D = pick([64, 128])
+    BS = pick([8, 16, 32])
+    Hkv = pick([1, 2, 3])
+    G = pick([4, 5, 6, 8, 12, 16] if tensor_core_shape else [1, 2, 3, 4, 5, 6, 8, 12, 16])
+    B = int(torch.randint(1, 7, (1,), generator=gen).item())
+    if tensor_core_shape:
+        B = max(B, -(-16 // (G * Hkv)))
+    lens = []
+    for _ in range(B):
+        kind = int(torch.randint(4, (1,), generator=gen).item())
+        if kind == 0:
+            lens.append(pick([0, 1, BS - 1, BS, BS + 1, 2 * BS + 1]))
+        else:
+            lens.append(int(torch.randint(1, 701, (1,), generator=gen).item()))
+    need = sum((L + BS - 1) // BS for L in lens)
+    NB = need + 3
+    tables = _place(lens, BS, NB, gen)
+    name = (f"random{'tc' if tensor_core_shape else ''}{seed}_b{B}_hq{G * Hkv}_hkv{Hkv}"
+            f"_d{D}_bs{BS}_{str(dtype)[6:]}")
+    return _assemble(name, dtype, BS, G * Hkv, Hkv, D, lens, tables, NB, gen,
+                     (6000 if tensor_core_shape else 5000) + seed, device)
+
+
 # Full-size workloads, in the order of the task's configuration list.
 FULL = {
     "tiny": tiny,
