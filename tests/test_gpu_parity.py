@@ -220,6 +220,41 @@ def test_shared_prefix_equals_private_copies_bit_identical():
         assert torch.equal(shared, private)
 
 
+def test_cow_step_leaves_the_other_sibling_bit_identical():
+    """Copy-on-write ("Sharing comes almost for free"): one sibling of each
+    pair copies the shared partial block and writes into its copy; the
+    other sibling, which does not step, decodes bit-identically before and
+    after, and the copied block equals its source byte for byte."""
+    b = W.SMALL["prefix_cow"]("cuda")
+    coins = b.meta["coins"]
+    diverge = [2 * j + c for j, c in enumerate(coins)]
+    keep = [2 * j + 1 - c for j, c in enumerate(coins)]
+    lens = (b.context_lens - 1).contiguous()     # the new tokens are not in the context
+    B, Hq, D = b.q.shape
+    max_ctx = int(lens.max().item())
+
+    def decode():
+        ws = ops.decode_workspace(B, Hq, D, max_ctx, b.block_size)
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device="cuda")
+        ops.pa_decode(out, b.q, b.k_cache, b.v_cache, b.block_tables, lens, max_ctx, b.scale, ws)
+        torch.cuda.synchronize()
+        assert ops.pa_decode_status(ws) == ops.PA_OK
+        return out
+
+    before = decode()
+    ops.pa_copy_blocks(b.k_cache, b.v_cache, b.cow_pairs)
+    torch.cuda.synchronize()
+    for src, dst in b.cow_pairs.cpu().tolist():
+        assert np.array_equal(bits(b.k_cache[dst]), bits(b.k_cache[src]))
+        assert np.array_equal(bits(b.v_cache[dst]), bits(b.v_cache[src]))
+    slots = b.slot_mapping.clone()
+    slots[keep] = -1                              # only the diverging siblings step
+    ops.pa_write_kv(b.k_cache, b.v_cache, b.key, b.value, slots)
+    after = decode()
+    assert torch.equal(after[keep], before[keep])
+    assert not torch.equal(after[diverge], before[diverge])   # their last block changed
+
+
 def test_deterministic_and_split_consistent():
     b = W.SMALL["long"]("cuda")
     o1 = run_step(b, write=True)
