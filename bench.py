@@ -25,6 +25,7 @@ import os
 import statistics
 import subprocess
 import sys
+import threading
 import time
 from pathlib import Path
 
@@ -143,27 +144,69 @@ def config_of(b, name, l2_note):
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
+    """SM clock and clock-event reasons sampled every ~0.5 ms by a background
+    thread through NVML (read-only queries; nothing on the GPU is changed),
+    or through `nvidia-smi -lms 100` where NVML is not available. summary()
+    keeps the samples taken inside the timed window when there are any."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+            "hw_thermal_slowdown": 0x40}
 
     def __init__(self, gpu_index):
         self.idx = gpu_index
+        self.samples = []          # (wall time, sm MHz, reason names)
+        self.sm_max = None
+        self.window = None
         self.proc = None
         self.out = None
+        self._stop = None
+        self._thread = None
+
+    def _nvml_loop(self, nv, h):
+        while not self._stop.is_set():
+            try:
+                mhz = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                bits = int(fn(h))
+            except Exception:  # noqa: BLE001 - sampling is best effort
+                break
+            names = [n for n, b in self.BITS.items() if bits & b]
+            self.samples.append((time.perf_counter(), mhz, names))
+            time.sleep(0.0005)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
-        time.sleep(0.15)
+            import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByIndex(self.idx)
+            self.sm_max = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            self._stop = threading.Event()
+            self._thread = threading.Thread(target=self._nvml_loop, args=(nv, h), daemon=True)
+            self._thread.start()
+        except Exception:  # noqa: BLE001 - fall back to nvidia-smi
+            self._thread = None
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                     "--format=csv,noheader,nounits", "-lms", "100"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except OSError:
+                self.proc = None
+            time.sleep(0.15)
         return self
 
+    def mark(self, t0, t1):
+        """Wall-clock bounds of the timed region."""
+        self.window = (t0, t1)
+
     def __exit__(self, *a):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
         if self.proc is not None:
             time.sleep(0.15)
             self.proc.terminate()
@@ -174,6 +217,14 @@ class ClockSampler:
                 self.out = ""
 
     def summary(self):
+        if self.samples:
+            inside = [x for x in self.samples
+                      if self.window and self.window[0] <= x[0] <= self.window[1]]
+            use = inside or self.samples
+            reasons = sorted({n for _, _, ns in use for n in ns})
+            return {"sm_mhz": statistics.median(x[1] for x in use), "sm_max_mhz": self.sm_max,
+                    "reasons": reasons, "samples": len(use),
+                    "samples_in_timed_region": len(inside), "source": "nvml"}
         if not self.out:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
         sm, smax, reasons = [], None, set()
@@ -191,7 +242,7 @@ class ClockSampler:
                 if v.lower().startswith("active"):
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvidia-smi"}
 
 
 # ---------------------------------------------------------------------------
@@ -213,7 +264,7 @@ def step_fn(b, ops, out, ws, split, path, stream):
     return step
 
 
-def time_device(step, K, W, stream, use_graph, world):
+def time_device(step, K, W, stream, use_graph, world, clock=None):
     """Device time of K steps (CUDA events on the launching stream)."""
     launches = 0
     with torch.cuda.stream(stream):
@@ -231,6 +282,7 @@ def time_device(step, K, W, stream, use_graph, world):
         barrier(world)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        w0 = time.perf_counter()
         e0.record(stream)
         for _ in range(K):
             if graph is not None:
@@ -239,9 +291,12 @@ def time_device(step, K, W, stream, use_graph, world):
                 step()
         e1.record(stream)
         torch.cuda.synchronize()
+        w1 = time.perf_counter()
         barrier(world)
     ms = e0.elapsed_time(e1)
     del graph
+    if clock is not None:
+        clock.mark(w0, w1)
     return ms / K, launches
 
 
@@ -515,7 +570,7 @@ def run_ours(args, rank, world, local):
     W = max(args.warmup, 3)
 
     with ClockSampler(local) as clk:
-        ms, per_step = time_device(step, args.steps, W, stream, not args.no_graph, world)
+        ms, per_step = time_device(step, args.steps, W, stream, not args.no_graph, world, clk)
     ms = max_over_ranks(ms, world)
     torch.cuda.synchronize()
     status = ops.pa_decode_status(ws, stream)
