@@ -485,12 +485,22 @@ def next_rows(ops, stream, rank):
     return res
 
 
-def kernel_source_hash():
-    """Hash of the decode kernels' sources (the traffic figure is only reported
-    while it was measured on these exact sources)."""
+def uses_tensor_cores(b, path):
+    """The decode kernel pa_decode picks for this batch (mirrors its dispatch:
+    16-bit KV, head_dim 128, 4..16 query heads per KV head, >= 16 query rows)."""
+    G = b.num_q_heads // b.num_kv_heads
+    fits = (b.dtype != torch.float32 and b.head_dim == 128 and 4 <= G <= 16
+            and b.num_seqs * b.num_q_heads >= 16)
+    return path == "tc" or (path == "auto" and fits)
+
+
+def kernel_source_hash(tensor_cores):
+    """Hash of the sources of the decode kernel that runs (the traffic figure
+    is only reported while it was measured on these exact sources)."""
     h = hashlib.sha256()
     csrc = ROOT / "paged_kv_cache_339_b200" / "csrc"
-    for name in ("pa_common.cuh", "pa_decode_simt.cu", "pa_decode_tc.cu", "pa_plan_reduce.cu"):
+    main = "pa_decode_tc.cu" if tensor_cores else "pa_decode_simt.cu"
+    for name in ("pa_common.cuh", main, "pa_plan_reduce.cu"):
         h.update((csrc / name).read_bytes())
     return h.hexdigest()[:16]
 
@@ -584,7 +594,7 @@ def run_ours(args, rank, world, local):
     seqs_all = sum_over_ranks(B, world)
     gbps = weak_scaling_value(kv_bytes_all, ms) / 1e9
     dec_gbps = kv_bytes / (dec_ms * 1e-3) / 1e9
-    khash = kernel_source_hash()
+    khash = kernel_source_hash(uses_tensor_cores(b, args.path))
     res = {
         "metric": METRIC, "value": round(gbps, 1), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": W, "ms_per_step": round(ms, 5),

@@ -166,6 +166,45 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* f) {
   for (int i = 0; i < 16; ++i) f[i] = __uint_as_float(v[i]);
 }
 
+// 16 columns of this warp's 32 TMEM lanes, without waiting for them; the
+// values are valid only after tmem_wait16 on the same array.
+__device__ __forceinline__ void tmem_ld16_async(uint32_t taddr, uint32_t* v) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+}
+// Wait for every outstanding tcgen05.ld of the thread; v is tied to the wait
+// so no use of it can be scheduled before it.
+__device__ __forceinline__ void tmem_wait16(uint32_t* v) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
+                 "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
+                 "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15])
+               :
+               : "memory");
+}
+// Orders later uses of v after an earlier tmem_wait16 (no instruction).
+__device__ __forceinline__ void tmem_after_wait16(uint32_t* v) {
+  asm volatile(""
+               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
+                 "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
+                 "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15])
+               :
+               : "memory");
+}
+
+// 2^x with the hardware approximation (ex2.approx.ftz: relative error below
+// 2^-22; -inf gives +0), for the probabilities of 16-bit caches.
+__device__ __forceinline__ float exp2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Round p to 16 bits (hi) and the remainder p - hi to 16 bits (lo): raw bits.
 template <typename T>
 __device__ __forceinline__ void split16(float p, uint16_t& hi, uint16_t& lo) {
@@ -701,9 +740,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!__all_sync(kFull, mbar_wait(&s_full[t], par, abrt, status))) break;
       tc_fence_after();
       float sv0[Ly::NS], sv1[Ly::NS];
-      tmem_ld16(lane_addr + s_col, sv0);
-      tmem_ld16(lane_addr + s_col + Ly::NS, sv1);
-      if constexpr (Ly::NS == 32) {
+      if constexpr (Ly::NS == 16) {
+        // both score tiles requested at once, one wait
+        uint32_t su0[16], su1[16];
+        tmem_ld16_async(lane_addr + s_col, su0);
+        tmem_ld16_async(lane_addr + s_col + Ly::NS, su1);
+        tmem_wait16(su0);
+        tmem_after_wait16(su1);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          sv0[i] = __uint_as_float(su0[i]);
+          sv1[i] = __uint_as_float(su1[i]);
+        }
+      } else {   // 64 columns: one wait per load keeps the registers in bounds
+        tmem_ld16(lane_addr + s_col, sv0);
+        tmem_ld16(lane_addr + s_col + Ly::NS, sv1);
         tmem_ld16(lane_addr + s_col + 16, sv0 + 16);
         tmem_ld16(lane_addr + s_col + Ly::NS + 16, sv1 + 16);
       }
@@ -711,6 +762,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[t]);
       const bool ok0 = tk0 < mt.valid, ok1 = tk0 + 64 < mt.valid;
+      // hardware 2^x (ex2.approx) where the registers allow it; the 16-head
+      // tile keeps exp2f, with which its registers fit without spilling
+      auto ex2 = [](float x) { return GT <= 8 ? exp2_approx(x) : exp2f(x); };
       float sa[GT], sb[GT];
 #pragma unroll
       for (int g = 0; g < GT; ++g) {
@@ -740,9 +794,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float cm = fmaxf(fmaxf(rb[g], rb[16 + g]), fmaxf(rb[32 + g], rb[48 + g]));
         const float mn = fmaxf(m_run[g], cm);
         // heads g >= G never see a finite score; keep them inert (alpha 0, p 0)
-        alpha[g] = (mn == -INFINITY) ? 0.f : exp2f(m_run[g] - mn);
+        alpha[g] = (mn == -INFINITY) ? 0.f : ex2(m_run[g] - mn);
         const float own_s = hh ? sb[g] : sa[g];
-        const float pr = (mn == -INFINITY) ? 0.f : exp2f(own_s - mn);
+        const float pr = (mn == -INFINITY) ? 0.f : ex2(own_s - mn);
         m_run[g] = mn;
         l_thr[g] = fmaf(l_thr[g], alpha[g], pr);
         uint16_t hi, lo;
