@@ -3,8 +3,9 @@
 One step = the whole hot path over one batch: copy-on-write block copies (when
 the workload has them), the new-token KV write, and paged decode attention for
 every sequence and query head. Inputs are resident in HBM before timing
-starts; every workload's KV bytes exceed the 126 MB L2, so no flush is needed
-between steps.
+starts; every workload's KV bytes exceed the 126 MB L2, so the mean step time
+is taken without a flush between steps. The line also gives p10 / p50 / p90 of
+per-step times, both as they come and with the L2 evicted before every step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mha|gqa|prefix_cow|long|tiny]
                     [--impl ours|reference] [--block-size BS] [--path auto|simt|tc]
@@ -300,6 +301,61 @@ def time_device(step, K, W, stream, use_graph, world, clock=None):
     return ms / K, launches
 
 
+def device_facts():
+    """Name, SM count and L2 size of the GPU the bench ran on."""
+    p = torch.cuda.get_device_properties(torch.cuda.current_device())
+    return {"name": p.name, "sm_count": p.multi_processor_count,
+            "l2_bytes": getattr(p, "L2_cache_size", None),
+            "hbm_bytes": p.total_memory}
+
+
+def l2_flusher():
+    """Evicts the L2 by reading a buffer of twice its size (a read leaves no
+    dirty lines to write back during the next step)."""
+    l2 = getattr(torch.cuda.get_device_properties(torch.cuda.current_device()),
+                 "L2_cache_size", 126 << 20) or (126 << 20)
+    buf = torch.ones((2 * l2) // 4, dtype=torch.float32, device="cuda")
+    sink = torch.empty((), dtype=torch.float32, device="cuda")
+    return lambda: torch.sum(buf, 0, out=sink)
+
+
+def step_times(step, K, stream, use_graph, flush=None):
+    """Device time of each of K steps, from a pair of CUDA events around every
+    step on the launching stream; `flush`, when given, runs between steps
+    outside the events. The step is idempotent (same write, same copies), so
+    every repetition does the same work."""
+    with torch.cuda.stream(stream):
+        graph = None
+        if use_graph:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=stream):
+                step()
+            graph.replay()
+        else:
+            step()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+        for e_a, e_z in ev:
+            if flush is not None:
+                flush()
+            e_a.record(stream)
+            if graph is not None:
+                graph.replay()
+            else:
+                step()
+            e_z.record(stream)
+        torch.cuda.synchronize()
+    del graph
+    return [e_a.elapsed_time(e_z) for e_a, e_z in ev]
+
+
+def percentiles(ms_list, world):
+    """p10 / p50 / p90 of per-step times, each the max over ranks."""
+    q = np.percentile(np.asarray(ms_list, dtype=np.float64), [10, 50, 90])
+    return {k: round(max_over_ranks(float(v), world), 5) for k, v in zip(("p10", "p50", "p90"), q)}
+
+
 def time_decode_only(b, ops, out, ws, split, path, stream, K, use_graph=True):
     """Average duration of the decode call alone (plan + main kernels):
     K calls back to back between two events on the launching stream, replayed
@@ -426,26 +482,30 @@ def time_graph(fn, stream, K):
 
 def next_rows(ops, stream, rank):
     """Measurements beyond the decode step: the paged-vs-contiguous cost of the
-    block table (same kernel, same lengths, blocks adjacent instead of
-    shuffled), a prefill-sized KV write, and block swap-out / swap-in between
-    the device pools and pinned host memory."""
+    block table at block sizes 8, 16 and 32 (same kernel, same lengths, blocks
+    adjacent instead of shuffled), a prefill-sized KV write, and block
+    swap-out / swap-in between the device pools and pinned host memory."""
     from paged_kv_cache_339_b200 import workloads as W
     res = {}
     for name, mk in (("mha", W.mha), ("gqa", W.gqa)):
-        row = {}
-        for placement in ("shuffled", "contiguous"):
-            b = mk("cuda", seed={"mha": 1002, "gqa": 1003}[name] + 100 * rank,
-                   contiguous=placement == "contiguous")
-            B, Hq, D = b.q.shape
-            ws = ops.decode_workspace(B, Hq, D, b.max_context_len, b.block_size, 0)
-            out = torch.empty((B, Hq, D), dtype=torch.float32, device="cuda")
-            ms = time_decode_only(b, ops, out, ws, 0, ops.PA_PATH_AUTO, stream, 20)
-            row[placement + "_decode_gbps"] = round(b.kv_bytes_logical() / (ms * 1e-3) / 1e9, 1)
-            del b, ws, out
-            torch.cuda.empty_cache()
-        row["table_cost_pct"] = round(
-            100.0 * (1.0 - row["shuffled_decode_gbps"] / row["contiguous_decode_gbps"]), 2)
-        res["paged_vs_contiguous_" + name] = row
+        per_bs = {}
+        for bs in (8, 16, 32):
+            row = {}
+            for placement in ("shuffled", "contiguous"):
+                b = mk("cuda", seed={"mha": 1002, "gqa": 1003}[name] + 100 * rank,
+                       block_size=bs, contiguous=placement == "contiguous")
+                B, Hq, D = b.q.shape
+                ws = ops.decode_workspace(B, Hq, D, b.max_context_len, b.block_size, 0)
+                out = torch.empty((B, Hq, D), dtype=torch.float32, device="cuda")
+                ms = time_decode_only(b, ops, out, ws, 0, ops.PA_PATH_AUTO, stream, 20)
+                row[placement + "_decode_gbps"] = round(
+                    b.kv_bytes_logical() / (ms * 1e-3) / 1e9, 1)
+                del b, ws, out
+                torch.cuda.empty_cache()
+            row["table_cost_pct"] = round(
+                100.0 * (1.0 - row["shuffled_decode_gbps"] / row["contiguous_decode_gbps"]), 2)
+            per_bs[f"bs{bs}"] = row
+        res["paged_vs_contiguous_" + name] = per_bs
     # prefill-sized write: T tokens of the MHA shape into distinct slots
     T, H, D, BS, NB = 16384, 32, 128, 16, 2048
     kc = torch.zeros((NB, H, BS, D), dtype=torch.bfloat16, device="cuda")
@@ -588,6 +648,10 @@ def run_ours(args, rank, world, local):
                                  not args.no_graph)
     e2e_ms, h2d, d2h = time_e2e(b, ops, ws, args.split, path, stream, max(5, args.steps // 2), 3)
     e2e_ms = max_over_ranks(e2e_ms, world)
+    use_graph = not args.no_graph
+    hot = percentiles(step_times(step, args.steps, stream, use_graph), world)
+    flushed = percentiles(step_times(step, args.steps, stream, use_graph, l2_flusher()), world)
+    torch.cuda.empty_cache()
 
     peak, peak_kind = measured_peak()
     kv_bytes_all = sum_over_ranks(kv_bytes, world)
@@ -602,7 +666,9 @@ def run_ours(args, rank, world, local):
         "dtype": {torch.bfloat16: "bf16", torch.float16: "f16", torch.float32: "f32"}[b.dtype],
         "data": "synthetic (seeded N(0,1) K/V/Q, shuffled block placement)",
         "config": config_of(b, args.workload,
-                            f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of KV read per step"),
+                            f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of KV read "
+                            "per step, not flushed; l2_flushed has per-step times with the "
+                            "L2 evicted before every step"),
         "seq_steps_per_s": round(weak_scaling_value(seqs_all, ms), 1),
         "pct_of_peak": round(100.0 * gbps / world / peak, 2),
         "pct_of_nominal_8tbs": round(100.0 * gbps / world / 8000.0, 2),
@@ -621,8 +687,24 @@ def run_ours(args, rank, world, local):
                 "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h)},
         "clocks": clk.summary(),
+        "device": device_facts(),
         "graph": not args.no_graph,
+        "step_ms": dict(mean=round(ms, 5), **hot),
+        "l2_flushed": dict(
+            note="L2 evicted (a read of 2x its size) before every step, outside the events",
+            gbps_at_p50=round(weak_scaling_value(kv_bytes_all, flushed["p50"]) / 1e9, 1),
+            **flushed),
     }
+    if b.cow_pairs.numel():
+        # the shared prefix is read by every sibling but crosses HBM once per step
+        ub = b.kv_bytes_unique()
+        ub_all = sum_over_ranks(ub, world)
+        res["unique_bytes"] = {
+            "kv_bytes_unique_per_step": ub,
+            "gbps_unique": round(weak_scaling_value(ub_all, ms) / 1e9, 1),
+            "pct_of_peak_unique": round(100.0 * ub_all / world / (ms * 1e-3) / 1e9 / peak, 2),
+            "gbps_unique_l2_flushed": round(weak_scaling_value(ub_all, flushed["p50"]) / 1e9, 1),
+        }
     if not args.no_secondary and world == 1 and args.workload == "mha":
         sec = {}
         for name in ("gqa", "long"):

@@ -39,7 +39,9 @@ def _worker(rank, world, port, q):
         ms = bench.max_over_ranks(my_ms, world)
         total = bench.sum_over_ranks(b.kv_bytes_logical(), world)
         value = bench.weak_scaling_value(total, ms)
-        q.put((rank, ms, value, float(out.sum()), b.kv_bytes_logical()))
+        # per-step times: rank 1's are uniformly 10x rank 0's
+        pct = bench.percentiles([(1 + 9 * rank) * x for x in range(1, 11)], world)
+        q.put((rank, ms, value, float(out.sum()), b.kv_bytes_logical(), pct))
     finally:
         dist.destroy_process_group()
 
@@ -51,12 +53,14 @@ def test_two_ranks_weak_scaling_control_path():
     procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
     for p in procs:
         p.start()
-    res = sorted(q.get(timeout=120) for _ in procs)
+    res = sorted((q.get(timeout=120) for _ in procs), key=lambda r: r[0])
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    (r0, ms0, v0, s0, b0), (r1, ms1, v1, s1, b1) = res
+    (r0, ms0, v0, s0, b0, p0), (r1, ms1, v1, s1, b1, p1) = res
     assert ms0 == ms1 == 2.0                         # max over ranks, on every rank
     assert v0 == v1                                  # every rank reports the same job value
     assert v0 == pytest.approx((b0 + b1) / 2.0e-3)   # units of both ranks / slowest time
     assert s0 != s1                                  # independent batches (different seeds)
+    # percentiles of 10x(1..10): linear interpolation gives 19, 55, 91 on both ranks
+    assert p0 == p1 == {"p10": 19.0, "p50": 55.0, "p90": 91.0}
