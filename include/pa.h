@@ -219,7 +219,9 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
  * Accumulation and softmax are fp32; the tensor-core path keeps the
  * probabilities at ~16 significant bits (two 16-bit terms).
  * PA_ERR_UNSUPPORTED also for more than 56,320 sequences in one call (the
- * planning kernel keeps the lengths in one CTA's shared memory).
+ * planning kernel keeps the lengths in one CTA's shared memory), and for
+ * num_seqs * num_q_heads of 2^31 or more (query rows are 32-bit copy
+ * coordinates).
  * Enqueues two kernels: a planning kernel, then the decode kernel. The
  * planning kernel is launched with programmatic stream serialisation: it may
  * start while the kernel before it in the stream is finishing, reads

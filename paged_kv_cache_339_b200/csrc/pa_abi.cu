@@ -213,6 +213,8 @@ pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
   if (workspace_bytes < lay.total) return PA_ERR_WORKSPACE_TOO_SMALL;
   // the planning kernel keeps the lengths in shared memory
   if (static_cast<int64_t>(num_seqs) * 4 > 220 * 1024) return PA_ERR_UNSUPPORTED;
+  // query rows are 32-bit coordinates of the copies
+  if (static_cast<int64_t>(num_seqs) * num_q_heads > INT32_MAX) return PA_ERR_UNSUPPORTED;
 
   // the tensor-core kernel loads query tiles of 16 rows: it needs >= 16 query rows
   const bool tc_ok = tc_supported(cache->dtype, cache->head_dim, group) &&

@@ -81,6 +81,11 @@ def test_host_side_rejections(lib):
     assert _decode(lib, ops, c, out=0x30004) == ops.PA_ERR_MISALIGNED
     assert _decode(lib, ops, c, ws_bytes=100) == ops.PA_ERR_WORKSPACE_TOO_SMALL
     assert _decode(lib, ops, c, B=0) == ops.PA_OK                          # nothing to do
+    # the plan keeps one length per sequence in shared memory: 56,320 at most
+    assert _decode(lib, ops, c, B=56321) == ops.PA_ERR_UNSUPPORTED
+    # 40,000 sequences x 53,688 query heads (26,844 KV heads, group 2) is past 2^31 query rows
+    big = _cache(ops, num_kv_heads=26844)
+    assert _decode(lib, ops, big, B=40000, Hq=53688, max_ctx=16, ws_bytes=1 << 62) == ops.PA_ERR_UNSUPPORTED
     assert lib.pa_write_kv(ctypes.byref(c), 0x1000, 0x2000, 0x3000, 0, None) == ops.PA_OK
     assert lib.pa_write_kv(ctypes.byref(c), 0x1000, 0x2000, 0x3000, -1, None) == ops.PA_ERR_INVALID_ARG
     assert lib.pa_write_kv(ctypes.byref(c), 0x1004, 0x2000, 0x3000, 3, None) == ops.PA_ERR_MISALIGNED

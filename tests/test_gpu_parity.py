@@ -335,3 +335,31 @@ def test_full_size_sampled(name):
         vblk = pool_bits(b.v_cache[s // BS:s // BS + 1])[0]
         assert np.array_equal(kblk[:, s % BS], bits(b.key[i]))
         assert np.array_equal(vblk[:, s % BS], bits(b.value[i]))
+
+
+@pytest.mark.parametrize("kind", ["tc_bf16_g4", "simt_f32_g1"])
+def test_maximum_sequence_count(kind):
+    """56,320 sequences, the most one call takes, with short log-normal /
+    uniform contexts: every row finite, sampled rows (first, last, longest,
+    shortest and a spread between) within tolerance of the oracle."""
+    B = 56320
+    if kind == "tc_bf16_g4":
+        b = W.gqa("cuda", seed=77, num_seqs=B, num_q_heads=4, num_kv_heads=1, mean_len=24,
+                  min_len=1, max_len=200)
+    else:
+        b = W.mha("cuda", seed=78, num_seqs=B, num_heads=1, head_dim=64, min_len=1,
+                  max_len=64, num_blocks=1, dtype=torch.float32)
+    out = run_step(b)
+    assert torch.isfinite(out).all()
+    lens = b.context_lens.cpu()
+    rng = np.random.default_rng(5)
+    seqs = sorted({0, B - 1, int(lens.argmax()), int(lens.argmin())}
+                  | {int(x) for x in rng.integers(0, B, 24)})
+    worst = 0.0
+    for i in seqs:
+        for h in sorted({0, b.num_q_heads - 1}):
+            ref = sampled_reference(b, i, h)
+            got = out[i, h].cpu().numpy().astype(np.float64)
+            worst = max(worst, float(np.max(np.abs(got - ref))))
+    assert worst <= TOL[b.dtype], (kind, worst)
+
