@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--pool-blocks", type=int, default=0,
                     help="mha only: pool size in blocks (0 = the workload's 16384)")
+    ap.add_argument("--num-seqs", type=int, default=0,
+                    help="mha / gqa / long: fewer sequences, for profiling a smaller case")
     return ap.parse_args()
 
 
@@ -115,7 +117,7 @@ def weak_scaling_value(units_all_ranks: float, ms_max: float) -> float:
 # workload
 # ---------------------------------------------------------------------------
 
-def make_batch(name, device, rank, block_size, pool_blocks=0):
+def make_batch(name, device, rank, block_size, pool_blocks=0, num_seqs=0):
     from paged_kv_cache_339_b200 import workloads as W
     fn = W.FULL[name]
     seed = {"tiny": 1001, "mha": 1002, "gqa": 1003, "prefix_cow": 1004, "long": 1005}[name]
@@ -124,6 +126,8 @@ def make_batch(name, device, rank, block_size, pool_blocks=0):
         kw["block_size"] = block_size
     if pool_blocks and name == "mha":
         kw["num_blocks"] = pool_blocks
+    if num_seqs and name in ("mha", "gqa", "long"):
+        kw["num_seqs"] = num_seqs
     return fn(device, **kw)
 
 
@@ -391,36 +395,59 @@ def time_decode_only(b, ops, out, ws, split, path, stream, K, use_graph=True):
 
 
 def time_e2e(b, ops, ws, split, path, stream, K, W):
-    """Same metric through the public API from pinned host buffers: every step
-    copies its inputs host->device and reads its result back. Two buffer sets
-    and a copy stream pipeline it the way a serving loop would: step i+1's
-    inputs go up while step i computes, step i's result comes back as soon as
-    it is done. All copies are inside the timed region."""
-    host = {k: getattr(b, k).cpu().pin_memory() for k in
-            ("q", "key", "value", "slot_mapping", "block_tables", "context_lens", "cow_pairs")}
-    dev = [{k: torch.empty_like(v, device="cuda") for k, v in host.items()} for _ in range(2)]
+    """Same metric through the public API from pinned host memory: every step
+    copies its inputs host->device and reads its result back, all inside the
+    timed region. The inputs travel as one packed buffer (every tensor at a
+    256-byte aligned offset), one copy per step. Two device buffer sets and
+    separate upload and download streams pipeline it the way a serving loop
+    would: step i+1's inputs go up while step i computes, and step i's result
+    comes back while step i+1 computes, both directions of the host link at
+    once."""
+    names = ("q", "key", "value", "slot_mapping", "block_tables", "context_lens", "cow_pairs")
+    src = {k: getattr(b, k) for k in names}
+    offs, n = {}, 0
+    for k in names:
+        offs[k] = n
+        n += (src[k].numel() * src[k].element_size() + 255) // 256 * 256
+    host = torch.zeros(max(n, 256), dtype=torch.uint8).pin_memory()
+    for k in names:
+        nb = src[k].numel() * src[k].element_size()
+        if nb:
+            host[offs[k]:offs[k] + nb] = src[k].contiguous().view(-1).cpu().view(torch.uint8)
+    raw = [torch.empty_like(host, device="cuda") for _ in range(2)]
+
+    def views(buf):
+        out = {}
+        for k in names:
+            t = src[k]
+            nb = t.numel() * t.element_size()
+            out[k] = buf[offs[k]:offs[k] + nb].view(t.dtype).view(t.shape)
+        return out
+
+    dev = [views(r) for r in raw]
     out = [torch.empty(b.q.shape, dtype=torch.float32, device="cuda") for _ in range(2)]
     out_h = [torch.empty(b.q.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
-    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    h2d = host.numel()
     d2h = out_h[0].numel() * 4
     max_ctx = b.max_context_len
-    cs = torch.cuda.Stream()
+    cu, cd = torch.cuda.Stream(), torch.cuda.Stream()
     ev = lambda: torch.cuda.Event()
     up = [ev(), ev()]      # inputs of a slot are on the device
     done = [ev(), ev()]    # the step that used a slot has finished
+    back = [ev(), ev()]    # the result of a slot has been read back
 
     def upload(i):
         sl = i & 1
-        with torch.cuda.stream(cs):
-            cs.wait_event(done[sl])          # the step two back has released the slot
-            for k in host:
-                dev[sl][k].copy_(host[k], non_blocking=True)
-            up[sl].record(cs)
+        with torch.cuda.stream(cu):
+            cu.wait_event(done[sl])          # the step two back has released the inputs
+            raw[sl].copy_(host, non_blocking=True)
+            up[sl].record(cu)
 
     def compute(i):
         sl, d = i & 1, dev[i & 1]
         with torch.cuda.stream(stream):
             stream.wait_event(up[sl])
+            stream.wait_event(back[sl])      # the step two back's result is out
             if d["cow_pairs"].numel():
                 ops.pa_copy_blocks(b.k_cache, b.v_cache, d["cow_pairs"], stream=stream)
             ops.pa_write_kv(b.k_cache, b.v_cache, d["key"], d["value"], d["slot_mapping"],
@@ -432,9 +459,10 @@ def time_e2e(b, ops, ws, split, path, stream, K, W):
 
     def download(i):
         sl = i & 1
-        with torch.cuda.stream(cs):
-            cs.wait_event(done[sl])
+        with torch.cuda.stream(cd):
+            cd.wait_event(done[sl])
             out_h[sl].copy_(out[sl], non_blocking=True)
+            back[sl].record(cd)
 
     def run(n):
         upload(0)
@@ -444,15 +472,17 @@ def time_e2e(b, ops, ws, split, path, stream, K, W):
                 upload(i + 1)
             download(i)
 
-    for e in done:
+    for e in done + back:
         e.record(stream)
     run(W)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    cs.wait_event(e0)
+    cu.wait_event(e0)
+    cd.wait_event(e0)
     run(K)
-    stream.wait_stream(cs)
+    stream.wait_stream(cu)
+    stream.wait_stream(cd)
     e1.record(stream)
     torch.cuda.synchronize()
     return e0.elapsed_time(e1) / K, h2d, d2h
@@ -630,7 +660,7 @@ def run_ours(args, rank, world, local):
     pa_build.build()
     from paged_kv_cache_339_b200 import ops
     path = {"auto": ops.PA_PATH_AUTO, "simt": ops.PA_PATH_SIMT, "tc": ops.PA_PATH_TCGEN05}[args.path]
-    b = make_batch(args.workload, "cuda", rank, args.block_size, args.pool_blocks)
+    b = make_batch(args.workload, "cuda", rank, args.block_size, args.pool_blocks, args.num_seqs)
     kv_bytes = b.kv_bytes_logical()
     B, Hq, D = b.q.shape
     ws = ops.decode_workspace(B, Hq, D, b.max_context_len, b.block_size, args.split)
@@ -729,7 +759,8 @@ def run_ours(args, rank, world, local):
         res["next"] = next_rows(ops, stream, rank)
         del b
         torch.cuda.empty_cache()
-        b = make_batch(args.workload, "cuda", rank, args.block_size)
+        b = make_batch(args.workload, "cuda", rank, args.block_size, args.pool_blocks,
+                       args.num_seqs)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         nbytes, secs, nseq, threads = oracle_sample(b, args.cpu_seconds)
         res["cpu_baseline"] = {

@@ -169,7 +169,8 @@ typedef enum {
 typedef struct {
   /* Tokens per work item (context split). 0 = chosen on the device from the
      actual context lengths: pieces of up to one item stream's share of the
-     whole batch (a multiple of 128, at least 256 and at least
+     whole batch (half a share when the batch has fewer (sequence, KV head)
+     units than item streams; a multiple of 128, at least 256 and at least
      max_context_len / 64), listed longest first, with the ends of the
      sequences cut finer when the batch has too little short work to even out
      the finish. Otherwise a positive multiple of block_size with

@@ -7,9 +7,11 @@
 // pieces and finish together. Pieces: as many whole S-token pieces as fit,
 // then the rest of the sequence. The automatic S is one stream's fair share
 // of the work (splits cost partial results and a merge, so only sequences
-// longer than that are cut); when the rests hold too little work to even
-// out the streams' finishing times (a few long sequences), each sequence's
-// last S-token pieces are cut into tail pieces of about an eighth of a share.
+// longer than that are cut), or half a share when there are fewer
+// (sequence, KV head) units than streams; when the rests hold too little
+// work to even out the streams' finishing times (a few long sequences), each
+// sequence's last S-token pieces are cut into tail pieces of about an eighth
+// of a share.
 //
 // The partial results of a split sequence are merged inside the decode
 // kernels by the last piece to finish (pa_common.cuh, merge_split_rows); the
@@ -122,7 +124,15 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
         // Whole pieces of up to one share: every split costs partial results
         // and a merge, so only sequences longer than a share are cut; the
         // longest-first order evens the CTAs out with the short sequences.
-        long long want = (share + kAutoSplitQuantum - 1) / kAutoSplitQuantum * kAutoSplitQuantum;
+        // With fewer (sequence, KV head) units than streams there are no
+        // short sequences to do that: every stream works on pieces of the
+        // few long ones, and a stream whose CTA partner has run dry slows
+        // down. Pieces of half a share then give each stream two or more,
+        // so the claiming order can even them out.
+        long long base = share;
+        if (static_cast<long long>(p.num_seqs) * p.num_kv_heads < p.num_ctas)
+          base = (share + 1) / 2;
+        long long want = (base + kAutoSplitQuantum - 1) / kAutoSplitQuantum * kAutoSplitQuantum;
         if (want < p.min_split) want = p.min_split;
         if (want > (1 << 30)) want = 1 << 30;
         S = static_cast<int>(want);

@@ -96,3 +96,26 @@ def test_plan_cuts_tails_when_sequences_are_few_and_long():
     S = plan["split_tokens"]
     assert sizes[0] == S
     assert np.sum(sizes <= S // 2) >= 64, "no short pieces at the end of the list"
+
+
+@pytest.mark.parametrize("name", ["gqa", "long"])
+def test_automatic_split_is_a_share_or_half_a_share(name):
+    """The automatic split on the tensor-core path (one CTA per SM, two item
+    streams each): one stream's share of the token-heads, rounded up to 128
+    tokens, or half a share when the (sequence, KV head) units are fewer than
+    the streams; never below the smallest split the workspace allows."""
+    b = W.FULL[name]("cuda")
+    B, Hq, D = b.q.shape
+    ws = ops.decode_workspace(B, Hq, D, b.max_context_len, b.block_size)
+    run_step(b, workspace=ws, write=False)
+    plan = read_plan(ws, B)
+    lens = b.context_lens.cpu().tolist()
+    streams = 2 * torch.cuda.get_device_properties(0).multi_processor_count
+    share = -(-sum(lens) * b.num_kv_heads // streams)
+    base = share if B * b.num_kv_heads >= streams else (share + 1) // 2
+    up128 = lambda x: -(-x // 128) * 128
+    min_split = max(256, up128(-(-max(lens) // 64)))
+    assert plan["split_tokens"] == max(up128(base), min_split)
+    # gqa has more units than streams, the long workload fewer
+    assert (B * b.num_kv_heads < streams) == (name == "long")
+
