@@ -117,6 +117,27 @@ def test_step_matches_oracle(name, split):
         assert err <= TOL[b.dtype], (name, path, st, err)
 
 
+# Split sequences of many pieces: counts around the merge's batches of 8
+# loads, up to 200 pieces, and a batch of sequences with different counts.
+PIECES = [7, 8, 9, 16, 17, 64, 65, 200, "mixed"]
+
+
+@pytest.mark.parametrize("pieces", PIECES)
+def test_many_pieces_merge(pieces):
+    if pieces == "mixed":
+        gen = np.random.default_rng(3)
+        lens = [int(x) for x in gen.integers(900, 9000, 5)] + [128 * 8, 128 * 8 + 1]
+    else:
+        lens = [128 * pieces - 5, 128 * pieces, 128 * (pieces - 1) + 1]
+    proto = _custom_batch(lens, device="cpu")
+    for path in paths_for(proto):
+        b = _custom_batch(lens)
+        bc = b.to("cpu")
+        out = run_step(b, split_tokens=128, path=path)
+        err = max_abs_err(out, oracle_step(bc))
+        assert err <= TOL[b.dtype], (pieces, path, err)
+
+
 def _custom_batch(lens, dtype=torch.bfloat16, Hq=8, Hkv=2, D=128, BS=16, seed=11,
                   device="cuda"):
     gen = torch.Generator().manual_seed(seed)
