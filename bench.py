@@ -271,6 +271,7 @@ def step_fn(b, ops, out, ws, split, path, stream):
 
 def time_device(step, K, W, stream, use_graph, world, clock=None):
     """Device time of K steps (CUDA events on the launching stream)."""
+    torch.cuda.synchronize()   # inputs drawn on the default stream are complete
     launches = 0
     with torch.cuda.stream(stream):
         for _ in range(W):
@@ -328,6 +329,7 @@ def step_times(step, K, stream, use_graph, flush=None):
     step on the launching stream; `flush`, when given, runs between steps
     outside the events. The step is idempotent (same write, same copies), so
     every repetition does the same work."""
+    torch.cuda.synchronize()   # inputs drawn on the default stream are complete
     with torch.cuda.stream(stream):
         graph = None
         if use_graph:
@@ -370,6 +372,7 @@ def time_decode_only(b, ops, out, ws, split, path, stream, K, use_graph=True):
         ops.pa_decode(out, b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens,
                       max_ctx, b.scale, ws, split_tokens=split, path=path, stream=stream)
 
+    torch.cuda.synchronize()   # inputs drawn on the default stream are complete
     with torch.cuda.stream(stream):
         for _ in range(3):
             call()
@@ -472,6 +475,7 @@ def time_e2e(b, ops, ws, split, path, stream, K, W):
                 upload(i + 1)
             download(i)
 
+    torch.cuda.synchronize()   # inputs drawn on the default stream are complete
     for e in done + back:
         e.record(stream)
     run(W)
@@ -491,6 +495,7 @@ def time_e2e(b, ops, ws, split, path, stream, K, W):
 def time_graph(fn, stream, K):
     """Average device time of fn (captured once in a CUDA graph), K replays
     back to back between two events."""
+    torch.cuda.synchronize()   # inputs drawn on the default stream are complete
     with torch.cuda.stream(stream):
         for _ in range(3):
             fn()
@@ -624,14 +629,16 @@ def measured_peak():
 # CPU oracle baseline (bounded sample)
 # ---------------------------------------------------------------------------
 
-def oracle_sample(b, seconds):
+def oracle_sample(b, seconds, out=None):
     """Run the fp64 oracle on the first sequences of the batch (all heads) until
-    about `seconds` of CPU work; returns (KV bytes covered, seconds, seqs)."""
+    about `seconds` of CPU work; returns (KV bytes covered, seconds, seqs,
+    threads, max-abs error of `out` on those rows or None)."""
     from oracle import ORACLE
     from threadpoolctl import threadpool_info
     BS = b.block_size
-    G = b.num_q_heads // b.num_kv_heads
     done_bytes, spent, nseq = 0, 0.0, 0
+    err = 0.0 if out is not None else None
+    scale = float(np.float32(b.scale))   # the fp32 value the kernels receive
     e = b.elem_bytes
     for i in range(b.num_seqs):
         L = int(b.context_lens[i])
@@ -642,15 +649,18 @@ def oracle_sample(b, seconds):
         q = b.q[i].to(torch.float32).cpu().numpy().astype(np.float64)
         t0 = time.perf_counter()
         tab = np.arange(nb)
-        for h in range(b.num_q_heads):
-            ORACLE.decode_one(q[h], kc, vc, tab, L, h, b.num_q_heads, b.scale)
+        ref = [ORACLE.decode_one(q[h], kc, vc, tab, L, h, b.num_q_heads, scale)
+               for h in range(b.num_q_heads)]
         spent += time.perf_counter() - t0
+        if out is not None:
+            got = out[i].cpu().numpy().astype(np.float64)
+            err = max(err, float(np.max(np.abs(got - np.stack(ref)))))
         done_bytes += 2 * L * b.num_kv_heads * b.head_dim * e
         nseq += 1
         if spent >= seconds:
             break
     threads = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
-    return done_bytes, spent, nseq, threads
+    return done_bytes, spent, nseq, threads, err
 
 
 # ---------------------------------------------------------------------------
@@ -762,13 +772,23 @@ def run_ours(args, rank, world, local):
         b = make_batch(args.workload, "cuda", rank, args.block_size, args.pool_blocks,
                        args.num_seqs)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        nbytes, secs, nseq, threads = oracle_sample(b, args.cpu_seconds)
+        # one untimed step on the batch as it is now (it may have been rebuilt
+        # after the secondary workloads), so `out` and the oracle see one cache;
+        # the pool was drawn on the default stream
+        torch.cuda.synchronize()
+        step_fn(b, ops, out, ws, args.split, path, stream)()
+        torch.cuda.synchronize()
+        nbytes, secs, nseq, threads, err = oracle_sample(b, args.cpu_seconds, out)
         res["cpu_baseline"] = {
             "value": round(nbytes / secs / 1e9, 4), "unit": "GB/s", "cores": threads,
             "kind": "oracle",
             "sample": f"fp64 NumPy oracle, decode of the first {nseq} of {b.num_seqs} "
                       f"sequences (all {b.num_q_heads} heads), {secs:.1f} s",
         }
+        tol = 1e-5 if b.dtype == torch.float32 else 2e-3
+        res["parity"] = {"max_abs_err": err, "tol": tol, "ok": err <= tol,
+                         "rows": nseq * b.num_q_heads,
+                         "against": "the fp64 oracle, on the cpu_baseline sample's rows"}
     return res
 
 
@@ -783,7 +803,7 @@ def run_reference(args, rank, world):
         oracle_sample(b, 0.1)
     tot_b, tot_s, seqs, threads = 0, 0.0, 0, 1
     for _ in range(args.steps):
-        nb, s, n, threads = oracle_sample(b, per)
+        nb, s, n, threads, _ = oracle_sample(b, per)
         tot_b += nb
         tot_s += s
         seqs = n

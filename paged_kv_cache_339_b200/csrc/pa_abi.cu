@@ -5,6 +5,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "pa.h"
 #include "pa_internal.h"
 
@@ -92,6 +94,16 @@ int num_sms() {
   return cached[dev];
 }
 
+// An NVTX range over one host call, named after the call, so a timeline
+// profiler shows where each call's work was enqueued; without a tool
+// attached, push and pop cost a call each.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 }  // namespace pa
 
 using namespace pa;
@@ -100,6 +112,7 @@ extern "C" {
 
 pa_status pa_write_kv(const pa_kv_cache* cache, const void* key, const void* value,
                       const int64_t* slot_mapping, int32_t num_tokens, pa_stream_t stream) {
+  NvtxRange range("pa_write_kv");
   pa_status st = check_cache(cache);
   if (st != PA_OK) return st;
   if (num_tokens < 0) return PA_ERR_INVALID_ARG;
@@ -118,6 +131,7 @@ pa_status pa_write_kv(const pa_kv_cache* cache, const void* key, const void* val
 
 pa_status pa_copy_blocks(const pa_kv_cache* cache, const int64_t* block_pairs, int32_t num_pairs,
                          pa_stream_t stream) {
+  NvtxRange range("pa_copy_blocks");
   pa_status st = check_cache(cache);
   if (st != PA_OK) return st;
   if (num_pairs < 0) return PA_ERR_INVALID_ARG;
@@ -147,6 +161,7 @@ static void* device_view_of_host(void* p) {
 pa_status pa_swap_blocks(const pa_kv_cache* cache, void* host_k, void* host_v,
                          int32_t host_num_blocks, const int64_t* block_pairs, int32_t num_pairs,
                          int32_t direction, pa_stream_t stream) {
+  NvtxRange range("pa_swap_blocks");
   pa_status st = check_cache(cache);
   if (st != PA_OK) return st;
   if (num_pairs < 0 || host_num_blocks < 0) return PA_ERR_INVALID_ARG;
@@ -183,6 +198,7 @@ pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
                     int32_t num_seqs, int32_t num_q_heads, int32_t max_context_len, float scale,
                     const pa_decode_options* opts, void* workspace, size_t workspace_bytes,
                     pa_stream_t stream) {
+  NvtxRange range("pa_decode");
   pa_status st = check_cache(cache);
   if (st != PA_OK) return st;
   if (num_seqs < 0 || num_q_heads <= 0 || max_context_len < 0) return PA_ERR_INVALID_ARG;
