@@ -397,6 +397,36 @@ def time_decode_only(b, ops, out, ws, split, path, stream, K, use_graph=True):
     return e0.elapsed_time(e1) / K
 
 
+STEP_INPUTS = ("q", "key", "value", "slot_mapping", "block_tables", "context_lens", "cow_pairs")
+
+
+def pack_step_inputs(b):
+    """One step's inputs as one host byte buffer, every tensor at a 256-byte
+    aligned offset (so one copy moves them all); returns (buffer, offsets)."""
+    offs, n = {}, 0
+    for k in STEP_INPUTS:
+        t = getattr(b, k)
+        offs[k] = n
+        n += (t.numel() * t.element_size() + 255) // 256 * 256
+    host = torch.zeros(max(n, 256), dtype=torch.uint8)
+    for k in STEP_INPUTS:
+        t = getattr(b, k)
+        nb = t.numel() * t.element_size()
+        if nb:
+            host[offs[k]:offs[k] + nb] = t.contiguous().view(-1).cpu().view(torch.uint8)
+    return host, offs
+
+
+def step_input_views(buf, b, offs):
+    """Typed views of a packed buffer (host or device), shaped like b's inputs."""
+    out = {}
+    for k in STEP_INPUTS:
+        t = getattr(b, k)
+        nb = t.numel() * t.element_size()
+        out[k] = buf[offs[k]:offs[k] + nb].view(t.dtype).view(t.shape)
+    return out
+
+
 def time_e2e(b, ops, ws, split, path, stream, K, W):
     """Same metric through the public API from pinned host memory: every step
     copies its inputs host->device and reads its result back, all inside the
@@ -406,28 +436,10 @@ def time_e2e(b, ops, ws, split, path, stream, K, W):
     would: step i+1's inputs go up while step i computes, and step i's result
     comes back while step i+1 computes, both directions of the host link at
     once."""
-    names = ("q", "key", "value", "slot_mapping", "block_tables", "context_lens", "cow_pairs")
-    src = {k: getattr(b, k) for k in names}
-    offs, n = {}, 0
-    for k in names:
-        offs[k] = n
-        n += (src[k].numel() * src[k].element_size() + 255) // 256 * 256
-    host = torch.zeros(max(n, 256), dtype=torch.uint8).pin_memory()
-    for k in names:
-        nb = src[k].numel() * src[k].element_size()
-        if nb:
-            host[offs[k]:offs[k] + nb] = src[k].contiguous().view(-1).cpu().view(torch.uint8)
+    host, offs = pack_step_inputs(b)
+    host = host.pin_memory()
     raw = [torch.empty_like(host, device="cuda") for _ in range(2)]
-
-    def views(buf):
-        out = {}
-        for k in names:
-            t = src[k]
-            nb = t.numel() * t.element_size()
-            out[k] = buf[offs[k]:offs[k] + nb].view(t.dtype).view(t.shape)
-        return out
-
-    dev = [views(r) for r in raw]
+    dev = [step_input_views(r, b, offs) for r in raw]
     out = [torch.empty(b.q.shape, dtype=torch.float32, device="cuda") for _ in range(2)]
     out_h = [torch.empty(b.q.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
     h2d = host.numel()
