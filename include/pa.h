@@ -34,6 +34,8 @@
  *     the CUDA error string of the most recent such failure on this thread.
  *   - Every array must be 16-byte aligned and densely packed in the layout
  *     given (row-major, innermost index last).
+ *   - Each call is wrapped in an NVTX range named after it, for timeline
+ *     profilers; without one attached, that costs two function calls.
  */
 #ifndef PAGED_KV_CACHE_PA_H
 #define PAGED_KV_CACHE_PA_H
@@ -267,7 +269,10 @@ pa_status pa_decode_noalloc(const pa_kv_cache* cache, float* out, const void* q,
 
 /*
  * pa_decode_status - read back (synchronously, on `stream`) the device status
- * word the last pa_decode using `workspace` left: PA_OK, or
+ * word the last pa_decode using `workspace` left: PA_OK;
+ * PA_ERR_INVALID_ARG if a table entry was outside the pool (block 0 was read
+ * in its place) or a length was negative or above max_context_len or its
+ * table (that sequence's rows were written as zero); or
  * PA_ERR_DEVICE_TIMEOUT if one of its kernels stopped waiting on a barrier
  * after its time limit and returned early (its output is then invalid).
  * The word is cleared on every pa_decode. Returns PA_ERR_CUDA if the copy fails.
