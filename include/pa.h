@@ -227,10 +227,13 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
  * coordinates).
  * Enqueues two kernels: a planning kernel, then the decode kernel. The
  * planning kernel is launched with programmatic stream serialisation: it may
- * start while the kernel before it in the stream is finishing, reads
- * context_lens at once and waits for that kernel before it completes. A
- * kernel right before pa_decode that lets its dependents launch early
- * (griddepcontrol.launch_dependents) must have written context_lens by then.
+ * start while the kernel before it in the stream is finishing: it reads
+ * context_lens and rewrites the workspace at once, then waits for that
+ * kernel before it writes the zero rows of empty sequences into `out` and
+ * completes. A kernel right before pa_decode that lets its dependents launch
+ * early (griddepcontrol.launch_dependents) must by then have written
+ * context_lens and be done with the workspace; it may still use `out`, q,
+ * the tables and the pools.
  */
 pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
                     const int32_t* block_tables, int32_t bt_stride,
@@ -254,11 +257,16 @@ pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
  * PA_ERR_WORKSPACE_TOO_SMALL before anything is enqueued. The call allocates
  * nothing.
  *   - The first call on a device looks up the array's device address (with
- *     that device current); make that first call before any stream capture.
+ *     that device current) and keeps it for the life of the process; make
+ *     that first call before any stream capture. cudaDeviceReset destroys the
+ *     array with the context, so no call may follow a reset in the same
+ *     process.
  *   - All calls share the one array and it keeps the last call's contents;
  *     each call re-initialises everything it reads, so nothing has to be
  *     cleared by the caller. Calls that overlap on the GPU (other streams, or
  *     other threads) race on the array and must not overlap.
+ *   - The status word the kernels raise (see pa_decode_status) lives in the
+ *     array too: read it with pa_decode_noalloc_status.
  */
 pa_status pa_decode_noalloc(const pa_kv_cache* cache, float* out, const void* q,
                             const int32_t* block_tables, int32_t bt_stride,
@@ -266,6 +274,17 @@ pa_status pa_decode_noalloc(const pa_kv_cache* cache, float* out, const void* q,
                             int32_t num_q_heads, int32_t max_context_len,
                             float scale, const pa_decode_options* opts,
                             pa_stream_t stream);
+
+/*
+ * pa_decode_noalloc_status - pa_decode_status for pa_decode_noalloc: reads
+ * back (synchronously, on `stream`) the status word that the last
+ * pa_decode_noalloc on the current device left in the library's fixed
+ * scratch, with the meanings given under pa_decode_status. The pages have no
+ * counterpart to this call either; it exists because a pa_decode_noalloc
+ * caller has no workspace pointer to hand to pa_decode_status. Returns
+ * PA_ERR_CUDA if the scratch cannot be reached or the copy fails.
+ */
+pa_status pa_decode_noalloc_status(pa_stream_t stream);
 
 /*
  * pa_decode_status - read back (synchronously, on `stream`) the device status

@@ -94,6 +94,61 @@ int num_sms() {
   return cached[dev];
 }
 
+// Every host check of a pa_decode call that does not involve the workspace,
+// and the kernel it will run. ch->empty: nothing to enqueue (no sequences).
+pa_status check_decode_args(const pa_kv_cache* cache, const float* out, const void* q,
+                            const int32_t* block_tables, int32_t bt_stride,
+                            const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                            int32_t max_context_len, float scale, const pa_decode_options* opts,
+                            DecodeChoice* ch) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (num_seqs < 0 || num_q_heads <= 0 || max_context_len < 0) return PA_ERR_INVALID_ARG;
+  if (num_q_heads % cache->num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+  const int group = num_q_heads / cache->num_kv_heads;
+  if (group > 16) return PA_ERR_UNSUPPORTED;
+  if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+  const int32_t split = opts ? opts->split_tokens : 0;
+  const int32_t path = opts ? opts->path : PA_PATH_AUTO;
+  if (split < 0 || path < PA_PATH_AUTO || path > PA_PATH_TCGEN05) return PA_ERR_INVALID_ARG;
+  if (split > 0) {
+    if (split % cache->block_size != 0) return PA_ERR_INVALID_ARG;
+    if (max_context_len > 0 && ceil_div(max_context_len, split) > kMaxSplits)
+      return PA_ERR_INVALID_ARG;
+  }
+  ch->group = group;
+  ch->split = split;
+  ch->use_tc = false;
+  ch->empty = num_seqs == 0;
+  if (ch->empty) return PA_OK;
+  if (out == nullptr || q == nullptr || block_tables == nullptr || context_lens == nullptr)
+    return PA_ERR_INVALID_ARG;
+  if (bt_stride <= 0) return PA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(max_context_len) > static_cast<int64_t>(bt_stride) * cache->block_size)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(q) || (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
+      (reinterpret_cast<uintptr_t>(context_lens) & 3u))
+    return PA_ERR_MISALIGNED;
+  // the planning kernel keeps the lengths in shared memory
+  if (static_cast<int64_t>(num_seqs) * 4 > 220 * 1024) return PA_ERR_UNSUPPORTED;
+  // query rows are 32-bit coordinates of the copies
+  if (static_cast<int64_t>(num_seqs) * num_q_heads > INT32_MAX) return PA_ERR_UNSUPPORTED;
+
+  // the tensor-core kernel loads query tiles of 16 rows: it needs >= 16 query rows
+  const bool tc_ok = tc_supported(cache->dtype, cache->head_dim, group) &&
+                     static_cast<int64_t>(num_seqs) * num_q_heads >= 16;
+  bool use_tc = false;
+  if (path == PA_PATH_TCGEN05) {
+    if (!tc_ok) return PA_ERR_UNSUPPORTED;
+    use_tc = true;
+  } else if (path == PA_PATH_AUTO) {
+    use_tc = tc_ok;
+  }
+  if (!use_tc && !simt_supported(cache->dtype, cache->head_dim, group)) return PA_ERR_UNSUPPORTED;
+  ch->use_tc = use_tc;
+  return PA_OK;
+}
+
 // An NVTX range over one host call, named after the call, so a timeline
 // profiler shows where each call's work was enqueued; without a tool
 // attached, push and pop cost a call each.
@@ -199,50 +254,19 @@ pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
                     const pa_decode_options* opts, void* workspace, size_t workspace_bytes,
                     pa_stream_t stream) {
   NvtxRange range("pa_decode");
-  pa_status st = check_cache(cache);
+  DecodeChoice ch;
+  pa_status st = check_decode_args(cache, out, q, block_tables, bt_stride, context_lens, num_seqs,
+                                   num_q_heads, max_context_len, scale, opts, &ch);
   if (st != PA_OK) return st;
-  if (num_seqs < 0 || num_q_heads <= 0 || max_context_len < 0) return PA_ERR_INVALID_ARG;
-  if (num_q_heads % cache->num_kv_heads != 0) return PA_ERR_INVALID_ARG;
-  const int group = num_q_heads / cache->num_kv_heads;
-  if (group > 16) return PA_ERR_UNSUPPORTED;
-  if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
-  const int32_t split = opts ? opts->split_tokens : 0;
-  const int32_t path = opts ? opts->path : PA_PATH_AUTO;
-  if (split < 0 || path < PA_PATH_AUTO || path > PA_PATH_TCGEN05) return PA_ERR_INVALID_ARG;
-  if (split > 0) {
-    if (split % cache->block_size != 0) return PA_ERR_INVALID_ARG;
-    if (max_context_len > 0 && ceil_div(max_context_len, split) > kMaxSplits)
-      return PA_ERR_INVALID_ARG;
-  }
-  if (num_seqs == 0) return PA_OK;
-  if (out == nullptr || q == nullptr || block_tables == nullptr || context_lens == nullptr ||
-      workspace == nullptr)
-    return PA_ERR_INVALID_ARG;
-  if (bt_stride <= 0) return PA_ERR_INVALID_ARG;
-  if (static_cast<int64_t>(max_context_len) > static_cast<int64_t>(bt_stride) * cache->block_size)
-    return PA_ERR_INVALID_ARG;
-  if (!aligned16(out) || !aligned16(q) || !aligned16(workspace) ||
-      (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
-      (reinterpret_cast<uintptr_t>(context_lens) & 3u))
-    return PA_ERR_MISALIGNED;
+  if (ch.empty) return PA_OK;
+  if (workspace == nullptr) return PA_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return PA_ERR_MISALIGNED;
+  const int group = ch.group;
+  const int32_t split = ch.split;
+  const bool use_tc = ch.use_tc;
+  // the workspace size is the last check
   const WsLayout lay = ws_layout(num_seqs, num_q_heads, cache->head_dim, max_context_len, split);
   if (workspace_bytes < lay.total) return PA_ERR_WORKSPACE_TOO_SMALL;
-  // the planning kernel keeps the lengths in shared memory
-  if (static_cast<int64_t>(num_seqs) * 4 > 220 * 1024) return PA_ERR_UNSUPPORTED;
-  // query rows are 32-bit coordinates of the copies
-  if (static_cast<int64_t>(num_seqs) * num_q_heads > INT32_MAX) return PA_ERR_UNSUPPORTED;
-
-  // the tensor-core kernel loads query tiles of 16 rows: it needs >= 16 query rows
-  const bool tc_ok = tc_supported(cache->dtype, cache->head_dim, group) &&
-                     static_cast<int64_t>(num_seqs) * num_q_heads >= 16;
-  bool use_tc = false;
-  if (path == PA_PATH_TCGEN05) {
-    if (!tc_ok) return PA_ERR_UNSUPPORTED;
-    use_tc = true;
-  } else if (path == PA_PATH_AUTO) {
-    use_tc = tc_ok;
-  }
-  if (!use_tc && !simt_supported(cache->dtype, cache->head_dim, group)) return PA_ERR_UNSUPPORTED;
 
   int ctas = 0;
   cudaError_t e = cached_ctas(use_tc, cache->dtype, cache->head_dim, group, &ctas);

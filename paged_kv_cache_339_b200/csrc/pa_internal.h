@@ -5,6 +5,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "pa.h"
 #include "pa_workspace.h"
 
 namespace pa {
@@ -87,6 +88,23 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
 }
+
+// What check_decode_args decided for a valid pa_decode call.
+struct DecodeChoice {
+  int group;       // query heads per KV head
+  int32_t split;   // explicit split (0 = automatic)
+  bool use_tc;     // tensor-core kernel (else CUDA cores)
+  bool empty;      // no sequences: nothing to enqueue
+};
+
+// Every host-side check of pa_decode's arguments except those of the
+// workspace (pointer, alignment, size), in pa_decode's order; PA_OK and the
+// choice, or the status pa_decode would return.
+pa_status check_decode_args(const pa_kv_cache* cache, const float* out, const void* q,
+                            const int32_t* block_tables, int32_t bt_stride,
+                            const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                            int32_t max_context_len, float scale, const pa_decode_options* opts,
+                            DecodeChoice* ch);
 
 // Store a CUDA error for pa_last_cuda_error() on this thread.
 void record_cuda_error(cudaError_t e);

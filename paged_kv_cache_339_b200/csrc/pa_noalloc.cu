@@ -54,15 +54,28 @@ extern "C" pa_status pa_decode_noalloc(const pa_kv_cache* cache, float* out, con
                                        int32_t num_q_heads, int32_t max_context_len,
                                        float scale, const pa_decode_options* opts,
                                        pa_stream_t stream) {
-  if (cache == nullptr || num_seqs < 0 || num_q_heads <= 0 || max_context_len < 0)
-    return PA_ERR_INVALID_ARG;
-  const int32_t split = opts ? opts->split_tokens : 0;
+  // pa_decode's own checks first, so a bad argument is reported as such and
+  // not as a scratch that is too small; the size of the scratch is the last
+  pa::DecodeChoice ch;
+  const pa_status chk = pa::check_decode_args(cache, out, q, block_tables, bt_stride,
+                                              context_lens, num_seqs, num_q_heads,
+                                              max_context_len, scale, opts, &ch);
+  if (chk != PA_OK) return chk;
+  if (ch.empty) return PA_OK;
   const size_t need = pa_decode_workspace_size(num_seqs, num_q_heads, cache->head_dim,
-                                               max_context_len, cache->block_size, split);
+                                               max_context_len, cache->block_size, ch.split);
   if (need > pa::kNoAllocScratchBytes) return PA_ERR_WORKSPACE_TOO_SMALL;
   void* scratch = nullptr;
   const pa_status st = pa::scratch_address(&scratch);
   if (st != PA_OK) return st;
   return pa_decode(cache, out, q, block_tables, bt_stride, context_lens, num_seqs, num_q_heads,
                    max_context_len, scale, opts, scratch, pa::kNoAllocScratchBytes, stream);
+}
+
+extern "C" pa_status pa_decode_noalloc_status(pa_stream_t stream) {
+  void* scratch = nullptr;
+  const pa_status st = pa::scratch_address(&scratch);
+  if (st != PA_OK) return st;
+  // the status word sits at the start of the scratch, as in a workspace
+  return pa_decode_status(scratch, stream);
 }

@@ -18,9 +18,10 @@
 // plan zeroes the merge counters they count on.
 //
 // Launched with programmatic stream serialisation: it may start while the KV
-// write before it is still running (it reads only the lengths), and waits for
-// that kernel before it exits, so the decode kernel that waits on the plan
-// also sees the new tokens.
+// write before it is still running (it reads only the lengths and rewrites
+// the workspace), and waits for that kernel before it writes the zero rows of
+// empty sequences into `out` and exits, so the decode kernel that waits on
+// the plan also sees the new tokens.
 #include "pa_common.cuh"
 #include "pa_internal.h"
 
@@ -203,12 +204,6 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
     if (nA > 0) atomicAdd(&s_hist[piece_key(S)], nA);
     if (k > 1) atomicAdd(&s_hist[piece_key(sb)], k - 1);
     if (k > 0) atomicAdd(&s_hist[piece_key(L - nA * S - (k - 1) * sb)], 1);
-    if (n == 0) {
-      float4* row = reinterpret_cast<float4*>(
-          p.out + static_cast<size_t>(i) * p.num_q_heads * p.head_dim);
-      const int n4 = p.num_q_heads * p.head_dim / 4;
-      for (int e = 0; e < n4; ++e) row[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
   }
   __syncthreads();
   // 4. longest first: bucket bases in descending length order (warp 0 scans
@@ -271,6 +266,17 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
   }
   // complete only after the kernel before this one (the KV write) has
   pdl_wait();
+  // Sequences with nothing to attend to get zero rows. These stores come
+  // after the wait: the kernel before this one may still read or write `out`
+  // until it has completed.
+  for (int i = tid; i < p.num_seqs; i += nthreads) {
+    const int L = s_len[i];
+    if (valid_len(L) && L > 0) continue;
+    float4* row = reinterpret_cast<float4*>(
+        p.out + static_cast<size_t>(i) * p.num_q_heads * p.head_dim);
+    const int n4 = p.num_q_heads * p.head_dim / 4;
+    for (int e = 0; e < n4; ++e) row[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 }
 
 }  // namespace

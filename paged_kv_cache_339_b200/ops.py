@@ -47,8 +47,8 @@ _lib = None
 
 EXPORTS = ("pa_write_kv", "pa_copy_blocks", "pa_swap_blocks", "pa_decode_workspace_size",
            "pa_decode",
-           "pa_decode_noalloc", "pa_decode_status", "pa_status_string", "pa_last_cuda_error",
-           "pa_version")
+           "pa_decode_noalloc", "pa_decode_noalloc_status", "pa_decode_status",
+           "pa_status_string", "pa_last_cuda_error", "pa_version")
 
 
 def _load():
@@ -78,6 +78,8 @@ def _load():
     lib.pa_decode_noalloc.restype = ctypes.c_int
     lib.pa_decode_status.argtypes = [vp, vp]
     lib.pa_decode_status.restype = ctypes.c_int
+    lib.pa_decode_noalloc_status.argtypes = [vp]
+    lib.pa_decode_noalloc_status.restype = ctypes.c_int
     lib.pa_status_string.argtypes = [ctypes.c_int]
     lib.pa_status_string.restype = ctypes.c_char_p
     lib.pa_last_cuda_error.argtypes = []
@@ -244,6 +246,12 @@ def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, max_
 def pa_decode_status(workspace, stream=None) -> int:
     """Device status word of the last pa_decode on this workspace (synchronises)."""
     return int(_load().pa_decode_status(_dev_tensor(workspace, "workspace"), _stream(stream)))
+
+
+def pa_decode_noalloc_status(stream=None) -> int:
+    """Device status word of the last pa_decode_noalloc on the current device
+    (synchronises)."""
+    return int(_load().pa_decode_noalloc_status(_stream(stream)))
 
 
 def pa_version() -> str:

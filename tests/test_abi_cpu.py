@@ -121,3 +121,36 @@ def test_workspace_size_layout(lib):
                  (4, 1, 64, 33, 16), (3, 8, 128, 1000, 32)):
         got = ops.pa_decode_workspace_size(args[0], args[1], args[2], args[3], 16, args[4])
         assert got == expect(*args), args
+
+
+def test_noalloc_checks_arguments_before_its_scratch_size(lib):
+    """pa_decode_noalloc runs pa_decode's argument checks first and compares
+    the fixed scratch size last; neither touches CUDA."""
+    from paged_kv_cache_339_b200 import ops
+    c = _cache(ops)
+
+    def noalloc(cache, B=2, Hq=4, max_ctx=64, bt_stride=4, split=0):
+        opts = ops.PaDecodeOptions(split, 0)
+        return lib.pa_decode_noalloc(ctypes.byref(cache), 0x30000, 0x40000, 0x50000, bt_stride,
+                                     0x60000, B, Hq, max_ctx, 0.1, ctypes.byref(opts), None)
+
+    assert noalloc(c, Hq=3) == ops.PA_ERR_INVALID_ARG                  # 3 % 2 != 0
+    assert noalloc(_cache(ops, head_dim=96)) == ops.PA_ERR_UNSUPPORTED
+    assert noalloc(c, split=24) == ops.PA_ERR_INVALID_ARG              # not k * 16
+    assert noalloc(c, B=0) == ops.PA_OK
+    # 4096 sequences x 64 heads (group 32 is refused first) ...
+    assert noalloc(_cache(ops, num_kv_heads=2), B=4096, Hq=64, max_ctx=65536,
+                   bt_stride=4096) == ops.PA_ERR_UNSUPPORTED
+    # ... while a valid shape that needs more than the 32 MiB scratch is refused as such
+    big = _cache(ops, num_kv_heads=8)
+    assert noalloc(big, B=4096, Hq=64, max_ctx=65536, bt_stride=4096) == \
+        ops.PA_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_device_timeout_status_is_reported(lib):
+    """A kernel that gave up waiting is reported by name, through the status
+    string and the binding's exception."""
+    from paged_kv_cache_339_b200 import ops
+    assert b"PA_ERR_DEVICE_TIMEOUT" in lib.pa_status_string(ops.PA_ERR_DEVICE_TIMEOUT)
+    e = ops.PagedAttnError("pa_decode", ops.PA_ERR_DEVICE_TIMEOUT)
+    assert e.status == ops.PA_ERR_DEVICE_TIMEOUT and "gave up waiting" in str(e)
