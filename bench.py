@@ -7,8 +7,16 @@ starts; every workload's KV bytes exceed the 126 MB L2, so the mean step time
 is taken without a flush between steps. The line also gives p10 / p50 / p90 of
 per-step times, both as they come and with the L2 evicted before every step.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mha|gqa|prefix_cow|long|tiny]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload long|gqa|mha|prefix_cow|tiny]
                     [--impl ours|reference] [--block-size BS] [--path auto|simt|tc]
+
+The default workload (the headline line) is long-context decode, the largest
+single-GPU configuration (8 sequences of 32K-128K tokens, 64/8 heads, bf16,
+block size 32). A default single-GPU run then measures the GQA, MHA and
+prefix-sharing configurations with the same keys (`configs`), and the rows
+beyond the decode step (`next`): paged vs contiguous placement, the
+long-context block-size sweep, a prefill-sized write, block swap, and the
+allocator waste simulation.
 
 Under torchrun (N > 1) every rank runs its own independent batch (different
 seed) on its own GPU: decode of different sequences needs no exchange, so the
@@ -45,7 +53,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="mha")
+    ap.add_argument("--workload", default="long")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--block-size", type=int, default=0)
     ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
@@ -562,8 +570,12 @@ def next_rows(ops, stream, rank):
     slots = torch.randperm(NB * BS, device="cuda")[:T].to(torch.int64)
     ms = time_graph(lambda: ops.pa_write_kv(kc, vc, key, val, slots, stream=stream), stream, 20)
     nbytes = 2 * T * H * D * 2
+    peak, _ = measured_peak()
     res["prefill_write"] = {"tokens": T, "bytes_written": nbytes,
                             "gbps_written": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                            "gbps_read_plus_written": round(2 * nbytes / (ms * 1e-3) / 1e9, 1),
+                            "frac_of_measured_peak": round(2 * nbytes / (ms * 1e-3) / 1e9 / peak,
+                                                           4),
                             "ms": round(ms, 4)}
     # swap: P blocks of that pool out to pinned host memory and back
     P = 1024
@@ -641,68 +653,92 @@ def measured_peak():
 # CPU oracle baseline (bounded sample)
 # ---------------------------------------------------------------------------
 
-def oracle_sample(b, seconds, out=None):
-    """Run the fp64 oracle on the first sequences of the batch (all heads) until
-    about `seconds` of CPU work; returns (KV bytes covered, seconds, seqs,
-    threads, max-abs error of `out` on those rows or None)."""
+def oracle_sample(b, seconds, out=None, cache=None):
+    """Run the fp64 oracle on (sequence, query head) rows of the batch, in
+    order, until about `seconds` of CPU work. Each (sequence, KV head) is
+    first copied back and widened to fp64 (not timed; `cache` keeps those
+    copies across calls). A row is credited with its share of the KV bytes,
+    2 * L * D * e / G, so a whole batch adds up to kv_bytes_logical().
+    Returns (KV bytes covered, seconds, rows, sequences touched, threads,
+    max-abs error of `out` on those rows or None)."""
     from oracle import ORACLE
     from threadpoolctl import threadpool_info
-    BS = b.block_size
-    done_bytes, spent, nseq = 0, 0.0, 0
-    err = 0.0 if out is not None else None
+    BS, D, e = b.block_size, b.head_dim, b.elem_bytes
+    G = b.num_q_heads // b.num_kv_heads
     scale = float(np.float32(b.scale))   # the fp32 value the kernels receive
-    e = b.elem_bytes
+    cache = {} if cache is None else cache
+    done_bytes, spent, rows, seqs = 0.0, 0.0, 0, 0
+    err = 0.0 if out is not None else None
+    stop = False
     for i in range(b.num_seqs):
         L = int(b.context_lens[i])
         nb = (L + BS - 1) // BS
-        rows = b.block_tables[i, :nb].long()
-        kc = ORACLE.logical_pool(b.k_cache[rows].to(torch.float32).cpu().numpy().astype(np.float64))
-        vc = ORACLE.logical_pool(b.v_cache[rows].to(torch.float32).cpu().numpy().astype(np.float64))
-        q = b.q[i].to(torch.float32).cpu().numpy().astype(np.float64)
-        t0 = time.perf_counter()
-        tab = np.arange(nb)
-        ref = [ORACLE.decode_one(q[h], kc, vc, tab, L, h, b.num_q_heads, scale)
-               for h in range(b.num_q_heads)]
-        spent += time.perf_counter() - t0
-        if out is not None:
-            got = out[i].cpu().numpy().astype(np.float64)
-            err = max(err, float(np.max(np.abs(got - np.stack(ref)))))
-        done_bytes += 2 * L * b.num_kv_heads * b.head_dim * e
-        nseq += 1
-        if spent >= seconds:
+        seqs += 1
+        for kv in range(b.num_kv_heads):
+            key = (i, kv)
+            if key not in cache:
+                blk = b.block_tables[i, :nb].long()
+                ks = b.k_cache[blk][:, kv:kv + 1].to(torch.float32).cpu().numpy()
+                vs = b.v_cache[blk][:, kv:kv + 1].to(torch.float32).cpu().numpy()
+                cache[key] = (ORACLE.logical_pool(ks.astype(np.float64)),
+                              ORACLE.logical_pool(vs.astype(np.float64)))
+            ksub, vsub = cache[key]
+            for h in range(kv * G, (kv + 1) * G):
+                q = b.q[i, h].to(torch.float32).cpu().numpy().astype(np.float64)
+                t0 = time.perf_counter()
+                ref = ORACLE.decode_one(q, ksub, vsub, np.arange(nb), L, 0, 1, scale)
+                spent += time.perf_counter() - t0
+                if out is not None:
+                    got = out[i, h].cpu().numpy().astype(np.float64)
+                    err = max(err, float(np.max(np.abs(got - ref))))
+                done_bytes += 2.0 * L * D * e / G
+                rows += 1
+                if spent >= seconds:
+                    stop = True
+                    break
+            if stop:
+                break
+        if stop:
             break
     threads = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
-    return done_bytes, spent, nseq, threads, err
+    return done_bytes, spent, rows, seqs, threads, err
 
 
 # ---------------------------------------------------------------------------
 
-def run_ours(args, rank, world, local):
-    from paged_kv_cache_339_b200 import build as pa_build
-    pa_build.build()
-    from paged_kv_cache_339_b200 import ops
-    path = {"auto": ops.PA_PATH_AUTO, "simt": ops.PA_PATH_SIMT, "tc": ops.PA_PATH_TCGEN05}[args.path]
-    b = make_batch(args.workload, "cuda", rank, args.block_size, args.pool_blocks, args.num_seqs)
+DTYPE_NAME = {torch.bfloat16: "bf16", torch.float16: "f16", torch.float32: "f32"}
+# the other configurations measured, with every key of the headline, in a
+# default single-GPU run
+OTHER_WORKLOADS = ("gqa", "mha", "prefix_cow")
+
+
+def measure(name, args, ops, rank, world, local, stream, path, split, steps, cpu_seconds,
+            block_size=0, pool_blocks=0, num_seqs=0):
+    """One configuration, every figure of the line: the step (copy-on-write
+    copies, KV write, decode) timed over `steps` graph replays, the decode
+    call alone (roofline), the end-to-end pipeline through pinned host
+    memory, per-step percentiles with and without an L2 flush, the clocks
+    during the timed region, and, at N = 1 on rank 0, the oracle on a
+    bounded sample of the same batch (cpu_baseline and parity)."""
+    b = make_batch(name, "cuda", rank, block_size, pool_blocks, num_seqs)
     kv_bytes = b.kv_bytes_logical()
     B, Hq, D = b.q.shape
-    ws = ops.decode_workspace(B, Hq, D, b.max_context_len, b.block_size, args.split)
+    ws = ops.decode_workspace(B, Hq, D, b.max_context_len, b.block_size, split)
     out = torch.empty((B, Hq, D), dtype=torch.float32, device="cuda")
-    stream = torch.cuda.Stream()
-    step = step_fn(b, ops, out, ws, args.split, path, stream)
+    step = step_fn(b, ops, out, ws, split, path, stream)
     W = max(args.warmup, 3)
+    use_graph = not args.no_graph
 
     with ClockSampler(local) as clk:
-        ms, per_step = time_device(step, args.steps, W, stream, not args.no_graph, world, clk)
+        ms, per_step = time_device(step, steps, W, stream, use_graph, world, clk)
     ms = max_over_ranks(ms, world)
     torch.cuda.synchronize()
     status = ops.pa_decode_status(ws, stream)
-    dec_ms = time_decode_only(b, ops, out, ws, args.split, path, stream, max(10, args.steps),
-                                 not args.no_graph)
-    e2e_ms, h2d, d2h = time_e2e(b, ops, ws, args.split, path, stream, max(5, args.steps // 2), 3)
+    dec_ms = time_decode_only(b, ops, out, ws, split, path, stream, max(10, steps), use_graph)
+    e2e_ms, h2d, d2h = time_e2e(b, ops, ws, split, path, stream, max(5, steps // 2), 3)
     e2e_ms = max_over_ranks(e2e_ms, world)
-    use_graph = not args.no_graph
-    hot = percentiles(step_times(step, args.steps, stream, use_graph), world)
-    flushed = percentiles(step_times(step, args.steps, stream, use_graph, l2_flusher()), world)
+    hot = percentiles(step_times(step, steps, stream, use_graph), world)
+    flushed = percentiles(step_times(step, steps, stream, use_graph, l2_flusher()), world)
     torch.cuda.empty_cache()
 
     peak, peak_kind = measured_peak()
@@ -710,24 +746,29 @@ def run_ours(args, rank, world, local):
     seqs_all = sum_over_ranks(B, world)
     gbps = weak_scaling_value(kv_bytes_all, ms) / 1e9
     dec_gbps = kv_bytes / (dec_ms * 1e-3) / 1e9
-    khash = kernel_source_hash(uses_tensor_cores(b, args.path))
+    tc = uses_tensor_cores(b, {ops.PA_PATH_AUTO: "auto", ops.PA_PATH_SIMT: "simt",
+                               ops.PA_PATH_TCGEN05: "tc"}[path])
+    khash = kernel_source_hash(tc)
+    l2_note = (f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of KV read per step, not "
+               "flushed; l2_flushed has per-step times with the L2 evicted before every step")
+    if b.cow_pairs.numel():
+        l2_note = (f"{kv_bytes / 1e9:.2f} GB of KV read per step (logical), "
+                   f"{b.kv_bytes_unique() / 1e9:.2f} GB of distinct slots: the shared prefix "
+                   "stays in L2 between siblings; not flushed, l2_flushed has per-step times "
+                   "with the L2 evicted before every step")
     res = {
-        "metric": METRIC, "value": round(gbps, 1), "unit": "GB/s", "n_gpus": world,
-        "steps": args.steps, "warmup": W, "ms_per_step": round(ms, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": {torch.bfloat16: "bf16", torch.float16: "f16", torch.float32: "f32"}[b.dtype],
-        "data": "synthetic (seeded N(0,1) K/V/Q, shuffled block placement)",
-        "config": config_of(b, args.workload,
-                            f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of KV read "
-                            "per step, not flushed; l2_flushed has per-step times with the "
-                            "L2 evicted before every step"),
+        "metric": METRIC, "value": round(gbps, 1), "unit": "GB/s",
+        "ms_per_step": round(ms, 5),
+        "dtype": DTYPE_NAME[b.dtype],
+        "config": config_of(b, name, l2_note),
         "seq_steps_per_s": round(weak_scaling_value(seqs_all, ms), 1),
         "pct_of_peak": round(100.0 * gbps / world / peak, 2),
         "pct_of_nominal_8tbs": round(100.0 * gbps / world / 8000.0, 2),
         "decode_status": int(status),
-        "gpu_launches": per_step * args.steps,
+        "gpu_launches": per_step * steps,
         "roofline": {
             "bound": "hbm", "kernel": "pa_decode (plan + decode main, merge fused)",
+            "decode_kernel": "tc_decode_kernel (tcgen05)" if tc else "simt_decode_kernel",
             "achieved": round(dec_gbps, 1), "peak": peak, "unit": "GB/s",
             "frac": round(dec_gbps / peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
             "algorithmic_bytes_per_launch": kv_bytes,
@@ -739,8 +780,6 @@ def run_ours(args, rank, world, local):
                 "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h)},
         "clocks": clk.summary(),
-        "device": device_facts(),
-        "graph": not args.no_graph,
         "step_ms": dict(mean=round(ms, 5), **hot),
         "l2_flushed": dict(
             note="L2 evicted (a read of 2x its size) before every step, outside the events",
@@ -756,51 +795,106 @@ def run_ours(args, rank, world, local):
             "gbps_unique": round(weak_scaling_value(ub_all, ms) / 1e9, 1),
             "pct_of_peak_unique": round(100.0 * ub_all / world / (ms * 1e-3) / 1e9 / peak, 2),
             "gbps_unique_l2_flushed": round(weak_scaling_value(ub_all, flushed["p50"]) / 1e9, 1),
+            "pct_of_peak_unique_l2_flushed": round(
+                100.0 * ub_all / world / (flushed["p50"] * 1e-3) / 1e9 / peak, 2),
         }
-    if not args.no_secondary and world == 1 and args.workload == "mha":
-        sec = {}
-        for name in ("gqa", "long"):
-            del b
-            torch.cuda.empty_cache()
-            b = make_batch(name, "cuda", rank, 0)
-            B2, Hq2, D2 = b.q.shape
-            ws2 = ops.decode_workspace(B2, Hq2, D2, b.max_context_len, b.block_size, 0)
-            out2 = torch.empty((B2, Hq2, D2), dtype=torch.float32, device="cuda")
-            st2 = step_fn(b, ops, out2, ws2, 0, ops.PA_PATH_AUTO, stream)
-            ms2, _ = time_device(st2, max(10, args.steps // 2), 3, stream, not args.no_graph, 1)
-            d2 = time_decode_only(b, ops, out2, ws2, 0, ops.PA_PATH_AUTO, stream, 10,
-                                     not args.no_graph)
-            kb = b.kv_bytes_logical()
-            sec[b.name] = {"step_gbps": round(kb / (ms2 * 1e-3) / 1e9, 1),
-                           "decode_gbps": round(kb / (d2 * 1e-3) / 1e9, 1),
-                           "frac_of_measured_peak": round(kb / (d2 * 1e-3) / 1e9 / peak, 4),
-                           "ms_per_step": round(ms2, 5),
-                           "status": ops.pa_decode_status(ws2, stream)}
-            del ws2, out2
-        res["secondary"] = sec
-        res["next"] = next_rows(ops, stream, rank)
-        del b
-        torch.cuda.empty_cache()
-        b = make_batch(args.workload, "cuda", rank, args.block_size, args.pool_blocks,
-                       args.num_seqs)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        # one untimed step on the batch as it is now (it may have been rebuilt
-        # after the secondary workloads), so `out` and the oracle see one cache;
-        # the pool was drawn on the default stream
+        # one untimed step on the batch as it is now, so `out` and the oracle
+        # see one cache; the pool was drawn on the default stream
         torch.cuda.synchronize()
-        step_fn(b, ops, out, ws, args.split, path, stream)()
+        step()
         torch.cuda.synchronize()
-        nbytes, secs, nseq, threads, err = oracle_sample(b, args.cpu_seconds, out)
+        nbytes, secs, rows, nseq, threads, err = oracle_sample(b, cpu_seconds, out)
         res["cpu_baseline"] = {
             "value": round(nbytes / secs / 1e9, 4), "unit": "GB/s", "cores": threads,
             "kind": "oracle",
-            "sample": f"fp64 NumPy oracle, decode of the first {nseq} of {b.num_seqs} "
-                      f"sequences (all {b.num_q_heads} heads), {secs:.1f} s",
+            "sample": f"fp64 NumPy oracle, decode of the first {rows} of "
+                      f"{b.num_seqs * b.num_q_heads} (sequence, query head) rows, in order "
+                      f"(first {nseq} sequences), {secs:.1f} s",
         }
         tol = 1e-5 if b.dtype == torch.float32 else 2e-3
-        res["parity"] = {"max_abs_err": err, "tol": tol, "ok": err <= tol,
-                         "rows": nseq * b.num_q_heads,
+        res["parity"] = {"max_abs_err": err, "tol": tol, "ok": err <= tol, "rows": rows,
                          "against": "the fp64 oracle, on the cpu_baseline sample's rows"}
+    del b, ws, out
+    torch.cuda.empty_cache()
+    return res
+
+
+def long_block_size_sweep(ops, stream, rank, steps, use_graph):
+    """The long-context workload at block sizes 8, 16 and 32 (same lengths,
+    shuffled pool): the step and the decode call alone."""
+    from paged_kv_cache_339_b200 import workloads as W
+    peak, _ = measured_peak()
+    res = {}
+    for bs in (8, 16, 32):
+        b = W.long_context("cuda", seed=1005 + 100 * rank, block_size=bs)
+        B, Hq, D = b.q.shape
+        ws = ops.decode_workspace(B, Hq, D, b.max_context_len, b.block_size, 0)
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device="cuda")
+        st = step_fn(b, ops, out, ws, 0, ops.PA_PATH_AUTO, stream)
+        ms, _ = time_device(st, steps, 3, stream, use_graph, 1)
+        d = time_decode_only(b, ops, out, ws, 0, ops.PA_PATH_AUTO, stream, steps, use_graph)
+        kb = b.kv_bytes_logical()
+        res[f"bs{bs}"] = {"step_gbps": round(kb / (ms * 1e-3) / 1e9, 1),
+                          "decode_gbps": round(kb / (d * 1e-3) / 1e9, 1),
+                          "frac_of_measured_peak": round(kb / (d * 1e-3) / 1e9 / peak, 4),
+                          "pct_of_nominal_8tbs": round(100.0 * kb / (d * 1e-3) / 1e9 / 8000.0, 2),
+                          "status": ops.pa_decode_status(ws, stream)}
+        del b, ws, out, st
+        torch.cuda.empty_cache()
+    return res
+
+
+def allocator_waste():
+    """Reserved-but-unused fraction of the KV cache under max-length
+    contiguous reservation and under paging at block sizes 8 / 16 / 32, over
+    one seeded trace of request arrivals and completions (host-side
+    bookkeeping only)."""
+    from paged_kv_cache_339_b200.block_manager import lifetime_trace, simulate_lifetimes
+    trace = lifetime_trace(2000, 4096, seed=1339)
+    res = {"trace": "2000 requests, Poisson arrivals 0.5/step, log-normal prompts (mean 256) "
+                    "and completions (mean 512), max context 4096, 64 live at most"}
+    for bs in (8, 16, 32):
+        r = simulate_lifetimes(trace, 4096, bs, max_live=64)
+        res[f"bs{bs}"] = {k: (round(v, 5) if isinstance(v, float) else v) for k, v in r.items()
+                          if k not in ("requests", "max_context", "max_live", "block_size")}
+    return res
+
+
+def run_ours(args, rank, world, local):
+    from paged_kv_cache_339_b200 import build as pa_build
+    pa_build.build()
+    from paged_kv_cache_339_b200 import ops
+    path = {"auto": ops.PA_PATH_AUTO, "simt": ops.PA_PATH_SIMT, "tc": ops.PA_PATH_TCGEN05}[args.path]
+    stream = torch.cuda.Stream()
+    head = measure(args.workload, args, ops, rank, world, local, stream, path, args.split,
+                   args.steps, args.cpu_seconds, args.block_size, args.pool_blocks,
+                   args.num_seqs)
+    res = {
+        "metric": METRIC, "value": head["value"], "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": head["dtype"],
+        "data": "synthetic (seeded N(0,1) K/V/Q, shuffled block placement)",
+        "config": head["config"],
+    }
+    for k, v in head.items():
+        res.setdefault(k, v)
+    res["device"] = device_facts()
+    res["graph"] = not args.no_graph
+    if not args.no_secondary and world == 1:
+        # the other configurations, each with the headline's keys
+        res["configs"] = {}
+        for name in OTHER_WORKLOADS:
+            if name == args.workload:
+                continue
+            r = measure(name, args, ops, rank, world, local, stream, ops.PA_PATH_AUTO, 0,
+                        max(10, args.steps // 2), args.cpu_seconds / 4)
+            res["configs"][r["config"]["workload"]] = r
+        res["next"] = next_rows(ops, stream, rank)
+        res["next"]["long_block_size_sweep"] = long_block_size_sweep(
+            ops, stream, rank, max(10, args.steps // 2), not args.no_graph)
+        res["next"]["allocator_waste"] = allocator_waste()
     return res
 
 
@@ -811,14 +905,14 @@ def run_reference(args, rank, world):
     b = make_batch(args.workload, "cuda" if torch.cuda.is_available() else "cpu", 0,
                    args.block_size)
     per = max(args.cpu_seconds / max(args.steps, 1), 0.5)
+    cache = {}
     for _ in range(min(args.warmup, 1)):
-        oracle_sample(b, 0.1)
-    tot_b, tot_s, seqs, threads = 0, 0.0, 0, 1
+        oracle_sample(b, 0.1, cache=cache)
+    tot_b, tot_s, rows, seqs, threads = 0.0, 0.0, 0, 0, 1
     for _ in range(args.steps):
-        nb, s, n, threads, _ = oracle_sample(b, per)
+        nb, sec, rows, seqs, threads, _ = oracle_sample(b, per, cache=cache)
         tot_b += nb
-        tot_s += s
-        seqs = n
+        tot_s += sec
     v = tot_b / tot_s / 1e9
     return {
         "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world,
@@ -829,7 +923,9 @@ def run_reference(args, rank, world):
         "config": config_of(b, args.workload, "host memory"),
         "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": threads,
                          "kind": "oracle",
-                         "sample": f"each step: decode of the first {seqs} sequences, all heads"},
+                         "sample": f"each step: decode of the first {rows} (sequence, query "
+                                   f"head) rows (first {seqs} sequences), the fp64 copies of "
+                                   "their KV prepared once before timing"},
         "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }

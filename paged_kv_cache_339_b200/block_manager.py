@@ -162,3 +162,96 @@ def paged_waste(block_size: int, lengths) -> float:
     lengths = list(lengths)
     reserved = sum(-(-L // block_size) * block_size for L in lengths)
     return 1.0 - sum(lengths) / reserved if reserved else 0.0
+
+
+def lifetime_trace(num_requests: int, max_context: int, seed: int, mean_prompt: int = 256,
+                   mean_completion: int = 512, sigma: float = 1.0, arrivals_per_step: float = 0.5):
+    """A seeded request trace: (arrival step, prompt tokens, completion tokens)
+    per request. Prompt and completion lengths are log-normal with the given
+    means (mu = ln(mean) - sigma^2 / 2), prompts clipped to [1, max_context / 2]
+    and completions to [1, max_context - prompt], so every request fits one
+    maximum-length reservation; arrivals are Poisson with the given rate.
+    The pages give only the maximum context (4096) and the average completion
+    (512) of their worked example; the distributions are a plain choice."""
+    import math
+    import random
+    rnd = random.Random(seed)
+
+    def lognormal(mean):
+        return math.exp(math.log(mean) - sigma * sigma / 2.0 + sigma * rnd.gauss(0.0, 1.0))
+
+    trace, t = [], 0.0
+    for _ in range(num_requests):
+        t += rnd.expovariate(arrivals_per_step)
+        p = min(max(1, round(lognormal(mean_prompt))), max_context // 2)
+        c = min(max(1, round(lognormal(mean_completion))), max_context - p)
+        trace.append((int(t), p, c))
+    return trace
+
+
+def simulate_lifetimes(trace, max_context: int, block_size: int, max_live: int):
+    """Run a request trace through both allocation schemes, step by step.
+
+    A request is admitted (first come, first served) once it has arrived and
+    fewer than `max_live` requests are live; it is prefilled with its prompt,
+    then generates one token per step until its completion length is reached,
+    and is freed. Both schemes see the same admissions, so they hold the same
+    tokens at every step and differ only in what they reserve:
+      * contiguous: a slab of `max_context` slots per live request, reserved
+        at admission ("Paged Attention as a Memory Manager", "The KV-Cache
+        Fragmentation Problem"; "Paged Attention: Virtual Memory for the KV
+        Cache", first section);
+      * paged: this module's BlockManager, a block at a time as tokens arrive
+        ("The fix borrowed from operating systems").
+    Returns the reserved-but-unused fraction of each scheme, summed over all
+    steps (time-averaged) and at each request's completion, the largest
+    number of unused slots one live paged request ever held, and whether the
+    pool got every block back."""
+    import math
+    total_tokens = sum(p + c for _, p, c in trace)
+    bm = BlockManager(num_blocks=max(1, min(max_live, len(trace)) *
+                                     math.ceil(max_context / block_size)),
+                      block_size=block_size)
+    pending = sorted(range(len(trace)), key=lambda i: (trace[i][0], i))
+    live = {}            # request -> tokens still to generate
+    nxt, step = 0, 0
+    used_sum = contig_sum = paged_sum = 0
+    fin_used = fin_contig = fin_paged = 0
+    max_unused = 0
+    while nxt < len(pending) or live:
+        while nxt < len(pending) and len(live) < max_live and trace[pending[nxt]][0] <= step:
+            r = pending[nxt]
+            bm.add_sequence(r, trace[r][1])
+            live[r] = trace[r][2]
+            nxt += 1
+        done = []
+        for r in live:
+            bm.append_token(r)
+            live[r] -= 1
+            if live[r] == 0:
+                done.append(r)
+        used = sum(bm.lengths[r] for r in live)
+        held = sum(len(bm.tables[r]) for r in live) * block_size
+        used_sum += used
+        contig_sum += len(live) * max_context
+        paged_sum += held
+        max_unused = max([max_unused] + [bm.reserved_unused_tokens(r) for r in live])
+        for r in done:
+            fin_used += bm.lengths[r]
+            fin_contig += max_context
+            fin_paged += len(bm.tables[r]) * block_size
+            bm.free(r)
+            del live[r]
+        step += 1
+    bm.check_invariants()
+    assert fin_used == total_tokens
+    return {
+        "requests": len(trace), "steps": step, "max_context": max_context,
+        "block_size": block_size, "max_live": max_live,
+        "contiguous_waste": 1.0 - used_sum / contig_sum if contig_sum else 0.0,
+        "paged_waste": 1.0 - used_sum / paged_sum if paged_sum else 0.0,
+        "contiguous_waste_at_completion": 1.0 - fin_used / fin_contig if fin_contig else 0.0,
+        "paged_waste_at_completion": 1.0 - fin_used / fin_paged if fin_paged else 0.0,
+        "paged_max_unused_slots_per_request": max_unused,
+        "all_blocks_returned": bm.num_free_blocks == bm.num_blocks,
+    }

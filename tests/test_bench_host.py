@@ -35,10 +35,26 @@ def test_parity_bookkeeping_catches_a_planted_error():
                         ORACLE.logical_pool(f(b.v_cache)), b.block_tables.numpy(),
                         b.context_lens.numpy(), float(np.float32(b.scale)))
     out = torch.from_numpy(ref.astype(np.float32))
-    _, _, nseq, _, err = bench.oracle_sample(b, 5.0, out)
-    assert nseq == b.num_seqs
+    nbytes, _, rows, nseq, _, err = bench.oracle_sample(b, 5.0, out)
+    assert nseq == b.num_seqs and rows == b.num_seqs * b.num_q_heads
+    assert nbytes == b.kv_bytes_logical()                  # a whole batch: every KV byte once
     assert err < 1e-6                                      # fp32 rounding of the oracle only
     planted = out.clone()
     planted[2, 0, 5] += 0.01
-    _, _, _, _, err2 = bench.oracle_sample(b, 5.0, planted)
+    _, _, _, _, _, err2 = bench.oracle_sample(b, 5.0, planted)
     assert err2 == pytest.approx(0.01, rel=1e-3)
+
+
+def test_oracle_sample_credits_kv_bytes_per_query_head_row():
+    """With query groups, each (sequence, query head) row carries 1 / G of its
+    KV head's bytes, so rows of a whole batch add up to its KV bytes."""
+    b = W.SMALL["gqa8"]("cpu")
+    G = b.num_q_heads // b.num_kv_heads
+    nbytes, _, rows, _, _, _ = bench.oracle_sample(b, 60.0)
+    assert rows == b.num_seqs * b.num_q_heads and G > 1
+    assert nbytes == pytest.approx(b.kv_bytes_logical(), rel=1e-12)
+    # a tiny budget stops after the first row: 2 * L_0 * D * e / G bytes
+    nb1, _, r1, s1, _, _ = bench.oracle_sample(b, 0.0)
+    L0 = int(b.context_lens[0])
+    assert (r1, s1) == (1, 1)
+    assert nb1 == pytest.approx(2 * L0 * b.head_dim * b.elem_bytes / G)

@@ -8,7 +8,8 @@ import pytest
 
 from paged_kv_cache_339_b200.block_manager import (BlockManager, OutOfBlocks,
                                                    contiguous_reservation_waste,
-                                                   paged_waste)
+                                                   lifetime_trace, paged_waste,
+                                                   simulate_lifetimes)
 
 GOLDEN = Path(__file__).parent / "golden"
 
@@ -137,3 +138,49 @@ def test_worked_example_internal_fragmentation():
     assert abs(w - g["page_says_untouched_fraction_approx"]) <= 0.0051   # "roughly 87%"
     assert paged_waste(16, lens) == 0.0
     assert paged_waste(16, [513]) == pytest.approx(1 - 513 / 528)
+
+
+def test_lifetime_simulation_reproduces_the_worked_example():
+    """Requests that all end at 512 tokens under a 4096-token maximum: each
+    contiguous reservation is 87.5 % untouched at completion ('Paged
+    Attention as a Memory Manager', 'The KV-Cache Fragmentation Problem'),
+    while 512 = 32 whole blocks of 16 leaves paging nothing unused."""
+    g = json.loads((GOLDEN / "fragmentation_worked_example.json").read_text())
+    M, L = g["max_context"], g["average_len"]
+    # prompt L - 1, one generated token: a single step at length L
+    r = simulate_lifetimes([(0, L - 1, 1)] * 10, M, 16, max_live=4)
+    assert r["contiguous_waste"] == g["exact_untouched_fraction"]
+    assert r["contiguous_waste_at_completion"] == g["exact_untouched_fraction"]
+    assert r["paged_waste"] == 0.0 and r["paged_max_unused_slots_per_request"] == 0
+    # prompt 1, 511 generated tokens: lengths 2..512 over the lifetime
+    r = simulate_lifetimes([(0, 1, L - 1)] * 10, M, 16, max_live=4)
+    assert r["contiguous_waste_at_completion"] == g["exact_untouched_fraction"]
+    lens = range(2, L + 1)
+    assert r["contiguous_waste"] == pytest.approx(1 - sum(lens) / (len(lens) * M), abs=1e-15)
+    held = sum(-(-n // 16) * 16 for n in lens)
+    assert r["paged_waste"] == pytest.approx(1 - sum(lens) / held, abs=1e-15)
+    assert r["paged_waste_at_completion"] == 0.0
+
+
+@pytest.mark.parametrize("bs", [8, 16, 32])
+def test_lifetime_simulation_paged_waste_below_one_block_per_request(bs):
+    """A seeded trace of arrivals and completions: every live paged request
+    holds fewer than one block of unused slots at every step ('The fix
+    borrowed from operating systems'), every block comes back, and paging
+    wastes a small fraction of what max-length contiguous slabs do."""
+    trace = lifetime_trace(400, 4096, seed=11)
+    r = simulate_lifetimes(trace, 4096, bs, max_live=32)
+    assert r["all_blocks_returned"]
+    assert r["paged_max_unused_slots_per_request"] < bs
+    assert r["paged_waste"] < bs / 2 / 256          # mean prompt alone is 256 tokens
+    assert r["contiguous_waste"] > 0.6
+    assert r["paged_waste"] < r["contiguous_waste"] / 20
+    # the two schemes hold the same tokens; only reservations differ
+    assert 0.0 <= r["paged_waste_at_completion"] < 1.0
+
+
+def test_lifetime_trace_is_seeded_and_fits_the_maximum():
+    a, b = lifetime_trace(200, 4096, seed=3), lifetime_trace(200, 4096, seed=3)
+    assert a == b and a != lifetime_trace(200, 4096, seed=4)
+    assert all(1 <= p and 1 <= c and p + c <= 4096 for _, p, c in a)
+    assert all(a[i][0] <= a[i + 1][0] for i in range(len(a) - 1))
