@@ -561,22 +561,31 @@ def next_rows(ops, stream, rank):
                 100.0 * (1.0 - row["shuffled_decode_gbps"] / row["contiguous_decode_gbps"]), 2)
             per_bs[f"bs{bs}"] = row
         res["paged_vs_contiguous_" + name] = per_bs
-    # prefill-sized write: T tokens of the MHA shape into distinct slots
+    # prefill-sized write: T tokens of the MHA shape. "prompt": 16 prompts of
+    # 1024 tokens, each filling its blocks in order (consecutive slots inside
+    # a block), blocks taken from a shuffled pool, as the block manager hands
+    # them out; "scattered": every token to a random slot of the pool.
     T, H, D, BS, NB = 16384, 32, 128, 16, 2048
     kc = torch.zeros((NB, H, BS, D), dtype=torch.bfloat16, device="cuda")
     vc = torch.zeros_like(kc)
     key = torch.randn((T, H, D), device="cuda").to(torch.bfloat16)
     val = torch.randn((T, H, D), device="cuda").to(torch.bfloat16)
-    slots = torch.randperm(NB * BS, device="cuda")[:T].to(torch.int64)
-    ms = time_graph(lambda: ops.pa_write_kv(kc, vc, key, val, slots, stream=stream), stream, 20)
+    g = torch.Generator().manual_seed(1339 + 100 * rank)
+    blocks = torch.randperm(NB, generator=g)[:T // BS]
+    prompt_slots = (blocks[:, None] * BS + torch.arange(BS)[None, :]).reshape(-1)
+    scattered = torch.randperm(NB * BS, generator=g)[:T]
     nbytes = 2 * T * H * D * 2
     peak, _ = measured_peak()
-    res["prefill_write"] = {"tokens": T, "bytes_written": nbytes,
-                            "gbps_written": round(nbytes / (ms * 1e-3) / 1e9, 1),
-                            "gbps_read_plus_written": round(2 * nbytes / (ms * 1e-3) / 1e9, 1),
-                            "frac_of_measured_peak": round(2 * nbytes / (ms * 1e-3) / 1e9 / peak,
-                                                           4),
-                            "ms": round(ms, 4)}
+    pw = {"tokens": T, "bytes_written": nbytes}
+    for label, sl in (("prompt", prompt_slots), ("scattered", scattered)):
+        slots = sl.to(torch.int64).cuda()
+        ms = time_graph(lambda: ops.pa_write_kv(kc, vc, key, val, slots, stream=stream),
+                        stream, 20)
+        pw[label] = {"gbps_written": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                     "gbps_read_plus_written": round(2 * nbytes / (ms * 1e-3) / 1e9, 1),
+                     "frac_of_measured_peak": round(2 * nbytes / (ms * 1e-3) / 1e9 / peak, 4),
+                     "ms": round(ms, 4)}
+    res["prefill_write"] = pw
     # swap: P blocks of that pool out to pinned host memory and back
     P = 1024
     hk = torch.empty((P, H, BS, D), dtype=torch.bfloat16, pin_memory=True)
@@ -709,7 +718,7 @@ def oracle_sample(b, seconds, out=None, cache=None):
 DTYPE_NAME = {torch.bfloat16: "bf16", torch.float16: "f16", torch.float32: "f32"}
 # the other configurations measured, with every key of the headline, in a
 # default single-GPU run
-OTHER_WORKLOADS = ("gqa", "mha", "prefix_cow")
+OTHER_WORKLOADS = ("long", "gqa", "mha", "prefix_cow")
 
 
 def measure(name, args, ops, rank, world, local, stream, path, split, steps, cpu_seconds,
