@@ -83,3 +83,23 @@ def sampled_reference(batch, seq, h):
     vsub = pool_f64(batch.v_cache[rows][:, kv:kv + 1])
     return ORACLE.decode_one(f64(batch.q[seq, h]), ksub, vsub, np.arange(nb), L, 0, 1,
                              float(np.float32(batch.scale)))
+
+
+def reference_rows(batch, seq, heads):
+    """Oracle output rows {h: row} for the given query heads of one sequence,
+    copying each KV head's blocks back once for all its query heads."""
+    L = int(batch.context_lens[seq].item())
+    BS = batch.block_size
+    nb = (L + BS - 1) // BS
+    G = batch.num_q_heads // batch.num_kv_heads
+    rows = batch.block_tables[seq, :nb].long()
+    scale = float(np.float32(batch.scale))
+    res = {}
+    for kv in sorted({h // G for h in heads}):
+        ksub = pool_f64(batch.k_cache[rows][:, kv:kv + 1])
+        vsub = pool_f64(batch.v_cache[rows][:, kv:kv + 1])
+        for h in heads:
+            if h // G == kv:
+                res[h] = ORACLE.decode_one(f64(batch.q[seq, h]), ksub, vsub, np.arange(nb),
+                                           L, 0, 1, scale)
+    return res

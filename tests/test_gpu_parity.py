@@ -15,7 +15,7 @@ from paged_kv_cache_339_b200 import build as pa_build
 from paged_kv_cache_339_b200 import ops
 from paged_kv_cache_339_b200 import workloads as W
 from tests.gpu_helpers import (TOL, bits, f64, max_abs_err, oracle_step, pool_bits,
-                               pool_f64, run_step, sampled_reference)
+                               pool_f64, reference_rows, run_step, sampled_reference)
 
 pytestmark = pytest.mark.gpu
 
@@ -345,6 +345,14 @@ def test_full_size_sampled(name):
             ref = sampled_reference(b, i, h)
             got = out[i, h].cpu().numpy().astype(np.float64)
             worst = max(worst, float(np.max(np.abs(got - ref))))
+    if name == "long":
+        # every query head of the longest and the shortest sequence: the rows
+        # that go through the tail cut of the plan and the merge of the most
+        # pieces
+        for i in sorted({int(lens.argmax()), int(lens.argmin())}):
+            for h, ref in reference_rows(b, i, list(range(Hq))).items():
+                got = out[i, h].cpu().numpy().astype(np.float64)
+                worst = max(worst, float(np.max(np.abs(got - ref))))
     assert worst <= TOL[b.dtype], (name, worst)
     # every row is finite, and rows of one KV-head group share the same keys
     assert torch.isfinite(out).all()
