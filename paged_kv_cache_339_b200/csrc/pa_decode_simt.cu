@@ -147,9 +147,10 @@ __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
     const WorkPair* pairs = reinterpret_cast<const WorkPair*>(p.ws + p.pairs_off);
     uint32_t c = 0;
     bool ok = true;
-    int kraw = 0;
-    if (lane == 0) kraw = atomicAdd(&hdr->work_counter, 1);
-    int k = __shfl_sync(kFull, kraw, 0);
+    // the first item is this CTA's own (the plan starts the claim counter
+    // after one item per CTA)
+    int kraw = blockIdx.x;
+    int k = static_cast<int>(blockIdx.x);
     while (k < num_items) {
       const int pi = k / Hkv, kvh = k - pi * Hkv;
       const WorkPair wp = pairs[pi];

@@ -480,12 +480,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         cur.nst = 3;
       }
     };
+    // Each stream's first item is its own, unclaimed: stream 2b + t of CTA b
+    // takes item 2b + t (the plan starts the claim counter after one item per
+    // stream), so the start-up path has no atomic.
     Stream st0 = {};
-    st0.nkraw = claim();   // both streams' first claims in flight at once
+    st0.nkraw = 2 * static_cast<int>(blockIdx.x);
     st0.nst = 1;
     Stream st1 = {};
-    st1.nkraw = claim();
+    st1.nkraw = 2 * static_cast<int>(blockIdx.x) + 1;
     st1.nst = 1;
+    // the two first items' work pairs, then their first table windows: each
+    // pair of loads is in flight together, two round trips in all
+    prefetch_step(st0);
+    prefetch_step(st1);
+    prefetch_step(st0);
+    prefetch_step(st1);
     int stops = 0;
     uint32_t c = 0;
     // describe position c for stream `cur` (a chunk, or an END / bubble /

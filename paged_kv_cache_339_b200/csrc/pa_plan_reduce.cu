@@ -223,7 +223,9 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
     if (lane == 31) {
       hdr->num_pairs = inc;
       hdr->num_items = inc * p.num_kv_heads;
-      hdr->work_counter = 0;
+      // every item stream takes item (its index) first without claiming it
+      // (no atomic on the start-up path); claims continue from here
+      hdr->work_counter = p.num_ctas;
     }
   }
   __syncthreads();

@@ -26,43 +26,69 @@ namespace {
 
 constexpr int kCopyThreads = 256;
 
-// A CTA takes whole tokens (one slot load per token) and its threads walk the
-// token's (head, 16-byte vector) pairs; every size that appears in the index
-// arithmetic (vectors per row, 64-column halves, the 16-token group) is a
-// power of two, so it is all shifts and masks.
+// A thread per 16-byte vector of the new K (and V) rows, four vectors apart by
+// the grid's width in flight at once: the four slot loads and eight row loads
+// are all issued before the first store, so neither the slot lookup nor the
+// load of one token waits for another's. Vector i of the input is row
+// i / row_vecs ((token, head) = divmod(row, num_kv_heads)), vector
+// i % row_vecs of it; consecutive threads read consecutive vectors, and each
+// run of 64 columns lands as one contiguous half-row of the tile. Sizes in the
+// index arithmetic other than the head count are powers of two (shifts).
+constexpr int kWriteUnroll = 4;
+
 __global__ void __launch_bounds__(kCopyThreads)
     write_kv_kernel(uint4* __restrict__ kc, uint4* __restrict__ vc,
                     const uint4* __restrict__ key,
                     const uint4* __restrict__ value,
-                    const int64_t* __restrict__ slots, int32_t num_tokens,
-                    int32_t num_kv_heads, int32_t block_size,
-                    int32_t row_vecs, int32_t head_dim, int64_t num_slots) {
+                    const int64_t* __restrict__ slots, int64_t total_vecs,
+                    int32_t num_kv_heads, int32_t bs_shift, int32_t rv_shift,
+                    int32_t head_dim, int64_t num_slots) {
   pdl_launch_dependents();   // the decode plan may start; it waits for us before it ends
-  const int per_token = num_kv_heads * row_vecs;
-  const int rv_shift = __ffs(row_vecs) - 1;
+  const int row_vecs = 1 << rv_shift;
   const int vec_elems = head_dim >> rv_shift;           // elements per 16-byte vector
   const int vh_shift = __ffs(64 / vec_elems) - 1;       // vectors per 64-column half
+  const int block_size = 1 << bs_shift;
   const int sh = tile_sub_height(block_size);
   const int sh_shift = __ffs(sh) - 1;
   const int nh = head_dim >> 6;
-  for (int t = blockIdx.x; t < num_tokens; t += gridDim.x) {
-    const int64_t slot = slots[t];
-    if (slot < 0 || slot >= num_slots) continue;
-    const int64_t blk = slot / block_size;
-    const int off = static_cast<int>(slot - blk * block_size);
-    // vector offset of (token off, half 0, column 0) inside a tile, and of
-    // the tile of head 0
-    const int row_base = (((off >> sh_shift) * nh) << sh_shift) * (64 / vec_elems) +
-                         (off & (sh - 1)) * (64 / vec_elems);
-    const int64_t tile0 = blk * num_kv_heads * (static_cast<int64_t>(block_size) << rv_shift);
-    const size_t src0 = static_cast<size_t>(t) * per_token;
-    for (int r = threadIdx.x; r < per_token; r += blockDim.x) {
-      const int h = r >> rv_shift, v = r & (row_vecs - 1);
-      const int half = v >> vh_shift, vin = v & ((1 << vh_shift) - 1);
-      const int64_t dst = tile0 + (static_cast<int64_t>(h) * block_size << rv_shift) + row_base +
-                          ((half << sh_shift) << vh_shift) + vin;
-      kc[dst] = key[src0 + r];
-      vc[dst] = value[src0 + r];
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+       base < total_vecs; base += kWriteUnroll * stride) {
+    uint4 a[kWriteUnroll], b[kWriteUnroll];
+    int64_t dst[kWriteUnroll];
+#pragma unroll
+    for (int k = 0; k < kWriteUnroll; ++k) {
+      const int64_t i = base + k * stride;
+      dst[k] = -1;
+      if (i < total_vecs) {
+        a[k] = key[i];
+        b[k] = value[i];
+        const int64_t row = i >> rv_shift;
+        // 32-bit division where the row index allows it (all realistic sizes)
+        const int64_t t = row <= 0x7fffffff
+                              ? static_cast<int64_t>(static_cast<uint32_t>(row) /
+                                                     static_cast<uint32_t>(num_kv_heads))
+                              : row / num_kv_heads;
+        const int h = static_cast<int>(row - t * num_kv_heads);
+        const int64_t slot = slots[t];
+        if (slot >= 0 && slot < num_slots) {
+          const int64_t blk = slot >> bs_shift;
+          const int off = static_cast<int>(slot & (block_size - 1));
+          const int v = static_cast<int>(i & (row_vecs - 1));
+          const int half = v >> vh_shift, vin = v & ((1 << vh_shift) - 1);
+          // tile (blk, h), then (token off, half, vector vin) inside it
+          dst[k] = ((blk * num_kv_heads + h) << (bs_shift + rv_shift)) +
+                   ((((off >> sh_shift) * nh + half) << sh_shift) << vh_shift) +
+                   ((off & (sh - 1)) << vh_shift) + vin;
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kWriteUnroll; ++k) {
+      if (dst[k] >= 0) {
+        kc[dst[k]] = a[k];
+        vc[dst[k]] = b[k];
+      }
     }
   }
 }
@@ -115,12 +141,16 @@ cudaError_t launch_write_kv(void* k_cache, void* v_cache, const void* key,
                             int32_t block_size, int32_t row_bytes, int32_t elem_bytes,
                             int64_t num_slots, cudaStream_t stream) {
   const int32_t row_vecs = row_bytes / 16;
+  const int64_t total = static_cast<int64_t>(num_tokens) * num_kv_heads * row_vecs;
+  const int64_t per_cta = static_cast<int64_t>(kCopyThreads) * kWriteUnroll;
   const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
-  const int grid = static_cast<int>(num_tokens < cap ? (num_tokens > 0 ? num_tokens : 1) : cap);
-  write_kv_kernel<<<grid, kCopyThreads, 0, stream>>>(
+  int64_t grid = (total + per_cta - 1) / per_cta;
+  grid = grid < 1 ? 1 : (grid > cap ? cap : grid);
+  write_kv_kernel<<<static_cast<int>(grid), kCopyThreads, 0, stream>>>(
       static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
-      static_cast<const uint4*>(key), static_cast<const uint4*>(value), slots,
-      num_tokens, num_kv_heads, block_size, row_vecs, row_vecs * 16 / elem_bytes, num_slots);
+      static_cast<const uint4*>(key), static_cast<const uint4*>(value), slots, total,
+      num_kv_heads, __builtin_ctz(static_cast<unsigned>(block_size)),
+      __builtin_ctz(static_cast<unsigned>(row_vecs)), row_vecs * 16 / elem_bytes, num_slots);
   return cudaGetLastError();
 }
 
