@@ -280,6 +280,7 @@ pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
   pp.ws = ws;
   pp.pairs_off = lay.pairs_off;
   pp.nsplit_off = lay.nsplit_off;
+  pp.split_off = lay.split_off;
   pp.cnt_off = lay.cnt_off;
   pp.num_seqs = num_seqs;
   pp.num_q_heads = num_q_heads;
@@ -304,6 +305,8 @@ pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
   dp.block_tables = block_tables;
   dp.ws = ws;
   dp.pairs_off = lay.pairs_off;
+  dp.nsplit_off = lay.nsplit_off;
+  dp.split_off = lay.split_off;
   dp.cnt_off = lay.cnt_off;
   dp.ml_off = lay.ml_off;
   dp.o_off = lay.o_off;

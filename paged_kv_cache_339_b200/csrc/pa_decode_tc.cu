@@ -710,13 +710,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (nsp == 1) return true;
       __threadfence();   // this piece's partial result, before it is counted
       if (!group_sync(gbar, gphase, abrt, status)) return false;
-      if (wq == 0 && lane == 0)
-        s_last[t] = atomicAdd(cnt + static_cast<size_t>(seq) * Hkv + kvh, 1) == nsp - 1;
-      if (!group_sync(gbar, gphase, abrt, status)) return false;
-      if (s_last[t]) {
-        __threadfence();   // every other piece counted before us is visible
-        merge_split_rows(p.out, ml, po, row0, G, kD, nsp, p.max_splits, r, 128);
-      }
+      // counted; the merge runs after the main loop (merge tasks below)
+      if (wq == 0 && lane == 0) atomicAdd(cnt + static_cast<size_t>(seq) * Hkv + kvh, 1);
       return true;
     };
 
@@ -883,6 +878,79 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!group_sync(gbar, gphase, abrt, status)) break;
           if (!finish(lr, mt.seq, mt.kvh, mt.split_raw, o, m_run)) break;
         }
+      }
+    }
+    // ---- merges of the split sequences, one output row per task. After its
+    // last item the group claims tasks, waits until every piece of the row's
+    // (sequence, KV head) has been counted, and merges the row: thread r
+    // takes column r over all pieces, 16 pieces' loads in flight. Outside the
+    // main loop, so the merge neither stalls the ring nor adds to the loop's
+    // registers; the groups that finish first share the merges out. A group
+    // waits only on pieces that streams of running CTAs have claimed (every
+    // item was claimed before any stream saw END), so every wait ends.
+    if (!*abrt) {
+      const int32_t* split_list = reinterpret_cast<const int32_t*>(p.ws + p.split_off);
+      const int32_t* nsplit_of = reinterpret_cast<const int32_t*>(p.ws + p.nsplit_off);
+      const int Hq = p.num_q_heads;
+      const int ntasks = hdr->num_split_seqs * Hq;
+      for (;;) {
+        if (wq == 0 && lane == 0) {
+          int k = atomicAdd(&hdr->merge_counter, 1);
+          if (k < ntasks) {
+            const int j = k / Hq;
+            const int sq = split_list[j];
+            const int kv = (k - j * Hq) / G;
+            const int nsp = nsplit_of[sq];
+            volatile int* c = cnt + static_cast<size_t>(sq) * Hkv + kv;
+            const unsigned long long t0 = global_timer_ns();
+            while (*c < nsp) {
+              if (*abrt || global_timer_ns() - t0 > kWaitLimitNs) {
+                if (!*abrt) atomicExch(status, 6 /* PA_ERR_DEVICE_TIMEOUT */);
+                *abrt = 1;
+                k = ntasks;
+                break;
+              }
+            }
+          }
+          s_last[t] = k;
+        }
+        if (!group_sync(gbar, gphase, abrt, status)) break;
+        const int k = s_last[t];
+        if (k >= ntasks) break;
+        __threadfence();   // the counted pieces' partial results are visible
+        const int j = k / Hq;
+        const int sq = split_list[j];
+        const int nsp = nsplit_of[sq];
+        const size_t row = static_cast<size_t>(sq) * Hq + (k - j * Hq);
+        const float2* mr = ml + row * p.max_splits;
+        const float* pr = po + row * p.max_splits * kD + r;
+        float M = -INFINITY, L = 0.f, acc = 0.f;
+        for (int s0 = 0; s0 < nsp; s0 += 16) {
+          float2 e[16];
+          float v[16];
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const bool in = s0 + jj < nsp;
+            e[jj] = in ? __ldcg(mr + s0 + jj) : make_float2(-INFINITY, 0.f);
+            v[jj] = in ? __ldcg(pr + static_cast<size_t>(s0 + jj) * kD) : 0.f;
+          }
+          float mb = M;
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) mb = fmaxf(mb, e[jj].x);
+          const float sc = exp2f(M - mb);   // M = -inf on the first batch: 0
+          L *= sc;
+          acc *= sc;
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const float w = exp2f(e[jj].x - mb);   // 0 for the padding entries
+            L = fmaf(e[jj].y, w, L);
+            acc = fmaf(w, v[jj], acc);
+          }
+          M = mb;
+        }
+        p.out[row * kD + r] = acc / L;
+        // the task slot is rewritten only after every thread has read it
+        if (!group_sync(gbar, gphase, abrt, status)) break;
       }
     }
   }

@@ -14,7 +14,7 @@ struct PlanParams {
   const int32_t* context_lens;
   float* out;
   uint8_t* ws;
-  size_t pairs_off, nsplit_off, cnt_off;
+  size_t pairs_off, nsplit_off, split_off, cnt_off;
   int32_t num_seqs, num_q_heads, num_kv_heads, head_dim;
   int32_t bt_stride, block_size, max_context_len;
   int32_t split_tokens;   // explicit split, or 0 = choose on the device
@@ -31,7 +31,7 @@ struct DecodeParams {
   float* out;
   const int32_t* block_tables;
   uint8_t* ws;
-  size_t pairs_off, cnt_off, ml_off, o_off;
+  size_t pairs_off, nsplit_off, split_off, cnt_off, ml_off, o_off;
   int32_t bt_stride, num_blocks, num_kv_heads, num_q_heads, head_dim,
       block_size, num_seqs, max_splits;
   float scale_log2;  // scale * log2(e): scores kept in log2 units

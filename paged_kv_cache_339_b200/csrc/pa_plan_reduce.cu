@@ -74,13 +74,16 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
   __shared__ int s_hist[kKeys + 1];
   __shared__ int s_fill[kKeys + 1];
   __shared__ PieceRule s_rule;
+  __shared__ int s_nsplit_seqs;
   extern __shared__ int s_len[];   // [num_seqs]
 
   WsHeader* hdr = reinterpret_cast<WsHeader*>(p.ws);
   WorkPair* pairs = reinterpret_cast<WorkPair*>(p.ws + p.pairs_off);
   int32_t* nsplit = reinterpret_cast<int32_t*>(p.ws + p.nsplit_off);
   int32_t* cnt = reinterpret_cast<int32_t*>(p.ws + p.cnt_off);
+  int32_t* split_list = reinterpret_cast<int32_t*>(p.ws + p.split_off);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) s_nsplit_seqs = 0;
   const int nthreads = blockDim.x, nwarps = nthreads >> 5;
   const int64_t cap = static_cast<int64_t>(p.bt_stride) * p.block_size;
   auto valid_len = [&](int L) { return !(L < 0 || L > p.max_context_len || L > cap); };
@@ -199,8 +202,10 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
     if (valid_len(L) && L > 0) seq_pieces(L, rule, nA, sb, k);
     const int n = nA + k;
     nsplit[i] = n;
-    if (n > 1)
+    if (n > 1) {
       for (int h = 0; h < p.num_kv_heads; ++h) cnt[static_cast<size_t>(i) * p.num_kv_heads + h] = 0;
+      split_list[atomicAdd(&s_nsplit_seqs, 1)] = i;
+    }
     if (nA > 0) atomicAdd(&s_hist[piece_key(S)], nA);
     if (k > 1) atomicAdd(&s_hist[piece_key(sb)], k - 1);
     if (k > 0) atomicAdd(&s_hist[piece_key(L - nA * S - (k - 1) * sb)], 1);
@@ -226,6 +231,8 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
       // every item stream takes item (its index) first without claiming it
       // (no atomic on the start-up path); claims continue from here
       hdr->work_counter = p.num_ctas;
+      hdr->num_split_seqs = s_nsplit_seqs;
+      hdr->merge_counter = 0;
     }
   }
   __syncthreads();

@@ -1,8 +1,8 @@
 // Layout of the caller-provided decode workspace (shared by host and device
 // code). All offsets are multiples of 256 bytes from the workspace start.
 //
-//   [header 256 B][work pairs][splits per sequence][merge counters]
-//   [partial (m, l)][partial o]
+//   [header 256 B][work pairs][splits per sequence][split sequences]
+//   [merge counters][partial (m, l)][partial o]
 //
 // The header holds the device status word (first 4 bytes), the work counter
 // the persistent decode kernels claim items from, and the plan the planning
@@ -24,7 +24,9 @@ struct WsHeader {
   int32_t num_pairs;     // (sequence, split) pairs
   int32_t split_tokens;  // tokens per split chosen for this call
   int32_t max_splits;    // split capacity per sequence in this workspace
-  int32_t reserved[58];
+  int32_t num_split_seqs;  // sequences cut into more than one piece
+  int32_t merge_counter;   // next unclaimed merge task (tensor-core kernel)
+  int32_t reserved[56];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
@@ -52,7 +54,7 @@ inline int32_t auto_min_split(int32_t max_ctx) {
 
 struct WsLayout {
   int32_t max_splits;
-  size_t pairs_off, nsplit_off, cnt_off, ml_off, o_off, total;
+  size_t pairs_off, nsplit_off, split_off, cnt_off, ml_off, o_off, total;
 };
 
 inline WsLayout ws_layout(int32_t num_seqs, int32_t num_q_heads,
@@ -70,6 +72,8 @@ inline WsLayout ws_layout(int32_t num_seqs, int32_t num_q_heads,
   w.pairs_off = off;
   off += align256(B * ms * 16);
   w.nsplit_off = off;
+  off += align256(B * 4);
+  w.split_off = off;   // the sequences cut into more than one piece
   off += align256(B * 4);
   w.cnt_off = off;   // merge counters [sequence][KV head] (KV heads <= query heads)
   off += align256(B * H * 4);

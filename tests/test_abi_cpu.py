@@ -105,16 +105,16 @@ def test_host_side_rejections(lib):
 
 
 def test_workspace_size_layout(lib):
-    """Header 256 B, then pairs, splits per sequence, partial (m, l) and
-    partial o, each rounded up to 256 B (header, pairs, splits, merge counters,
-    m/l, partial o); split capacity from the split rule."""
+    """Header 256 B, then pairs, splits per sequence, the list of split
+    sequences, merge counters, partial (m, l) and partial o, each rounded up to
+    256 B; split capacity from the split rule."""
     from paged_kv_cache_339_b200 import ops
 
     def expect(B, H, D, max_ctx, split):
         s = split if split > 0 else max(256, -(-(-(-max_ctx // 64)) // 128) * 128)
         ms = max(1, -(-max_ctx // s))
         r = lambda x: -(-x // 256) * 256
-        return (256 + r(B * ms * 16) + r(B * 4) + r(B * H * 4) + r(B * H * ms * 8)
+        return (256 + r(B * ms * 16) + r(B * 4) + r(B * 4) + r(B * H * 4) + r(B * H * ms * 8)
                 + r(B * H * ms * D * 4))
 
     for args in ((64, 32, 128, 2048, 0), (256, 32, 128, 4096, 0), (8, 64, 128, 131072, 0),
