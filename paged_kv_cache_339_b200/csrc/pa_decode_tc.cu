@@ -433,8 +433,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Per-stream state (warp-uniform), plus a window of block-table entries:
     // lane j holds entries wbase + j and wbase + 32 + j of the current item.
     // The next item of each stream is prefetched one step per emission
-    // (claim -> work pair -> first table window), starting three chunks
-    // before the current item ends. The loop below is unrolled over the two
+    // (claim -> work pair -> first table window), starting with the current
+    // item's last chunk. The loop below is unrolled over the two
     // streams so each stream's state sits in its own registers.
     struct Stream {
       int seq, kvh, split_n, tb, te, cs;   // current item, next chunk start
@@ -540,9 +540,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           blk = 0;
         }
         // advance the next item's prefetch by one step; the claim itself waits
-        // until the current item has at most 3 chunks left, so a stream never
-        // holds an unstarted item for long (it would lengthen the tail)
-        if (cur.nst != 0 || cur.te - cur.cs <= 3 * kChunk) prefetch_step(cur);
+        // until the current item has its last chunk left, so a stream never
+        // holds an unstarted item for long (it would lengthen the tail); the
+        // scheduler runs far enough ahead of the copies to cover the claim,
+        // work pair and table window loads
+        if (cur.nst != 0 || cur.te - cur.cs <= kChunk) prefetch_step(cur);
       }
       const int qd = c % kQd;
       if (!mbar_wait(&desc_empty[qd], ((c / kQd) & 1u) ^ 1u, abrt, status)) return false;
