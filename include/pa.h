@@ -184,9 +184,10 @@ typedef struct {
 
 /*
  * pa_decode_workspace_size - bytes of device workspace pa_decode needs for the
- * given shapes (status word and plan, work list, piece counts, a merge counter
- * per (sequence, KV head), one partial result per (sequence, query head,
- * piece)). split_tokens as in pa_decode_options.
+ * given shapes (status word and plan, work list, piece counts, the list of
+ * sequences cut into pieces, a merge counter per (sequence, KV head), one
+ * partial result per (sequence, query head, piece)). split_tokens as in
+ * pa_decode_options.
  */
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
                                 int32_t head_dim, int32_t max_context_len,

@@ -1020,6 +1020,9 @@ cudaError_t launch_t(const DecodeParams& p, int num_ctas, cudaStream_t stream) {
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(Ly::SMEM));
   if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
   e = launch_pdl(kern, dim3(num_ctas), dim3(kThreads), Ly::SMEM, stream, p, mk, mv, mq);
   return e != cudaSuccess ? e : cudaGetLastError();
 }

@@ -193,9 +193,8 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
   const PieceRule rule = s_rule;
 
   // 3. pieces per sequence (a thread per sequence): split counts, zeroed merge
-  // counters of split sequences, and the length histogram (a sequence's
-  // pieces form at most three runs of equal length); sequences with nothing
-  // to attend to get zero rows
+  // counters and the list of split sequences, and the length histogram (a
+  // sequence's pieces form at most three runs of equal length)
   for (int i = tid; i < p.num_seqs; i += nthreads) {
     const int L = s_len[i];
     int nA = 0, sb = 0, k = 0;
@@ -311,6 +310,11 @@ cudaError_t launch_plan(const PlanParams& p, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  // the largest shared-memory carveout, as the decode kernels use: an SM that
+  // ran this kernel need not be reconfigured before it takes a decode CTA
+  cudaError_t e = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                       cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
   return cudaLaunchKernelEx(&cfg, plan_kernel, p);
 }
 
