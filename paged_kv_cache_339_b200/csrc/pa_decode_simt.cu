@@ -145,6 +145,7 @@ __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     const WorkPair* pairs = reinterpret_cast<const WorkPair*>(p.ws + p.pairs_off);
+    const uint64_t pol = l2_evict_first_policy();   // K and V tiles: read once per call
     uint32_t c = 0;
     bool ok = true;
     // the first item is this CTA's own (the plan starts the claim counter
@@ -200,8 +201,8 @@ __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
           const uint8_t* gv = static_cast<const uint8_t*>(p.v_cache) + src;
           uint8_t* dk = stages + static_cast<size_t>(stage) * Tr::STAGE + lane * BS * ROW;
           if (rows == BS || Tr::NH == 1) {
-            bulk_g2s(dk, gk, rows * ROW, &full[stage]);
-            bulk_g2s(dk + CHUNK * ROW, gv, rows * ROW, &full[stage]);
+            bulk_g2s_hint(dk, gk, rows * ROW, &full[stage], pol);
+            bulk_g2s_hint(dk + CHUNK * ROW, gv, rows * ROW, &full[stage], pol);
           } else {
             const int sh = tile_sub_height(BS);
             for (int sp = 0; sp * sh < rows; ++sp) {
@@ -209,8 +210,8 @@ __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
 #pragma unroll
               for (int h = 0; h < Tr::NH; ++h) {
                 const int seg = (sp * Tr::NH + h) * sh * Tr::HALF;
-                bulk_g2s(dk + seg, gk + seg, nb, &full[stage]);
-                bulk_g2s(dk + CHUNK * ROW + seg, gv + seg, nb, &full[stage]);
+                bulk_g2s_hint(dk + seg, gk + seg, nb, &full[stage], pol);
+                bulk_g2s_hint(dk + CHUNK * ROW + seg, gv + seg, nb, &full[stage], pol);
               }
             }
           }

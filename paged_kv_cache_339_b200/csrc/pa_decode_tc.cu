@@ -337,6 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_v);
     }
+    const uint64_t pol = l2_evict_first_policy();   // K and V tiles: read once per call
     int stops = 0;
     uint32_t ck = 0, cv = 0;   // positions whose K / V copies (or markers) were issued
     bool ok = true;
@@ -385,7 +386,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           __syncwarp();
           if (lane < npg)
-            tma_load_2d(st + lane * BS * 256, &tm_k, 0, (blk * Hkv + kvh) * BS * 2, &kfull[bi]);
+            tma_load_2d_hint(st + lane * BS * 256, &tm_k, 0, (blk * Hkv + kvh) * BS * 2,
+                             &kfull[bi], pol);
         } else {
           if (lane == 0) {
             meta[bi].flags = flags;
@@ -405,8 +407,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) mbar_arrive_expect_tx(&vfull[bi], static_cast<uint32_t>(npg * BS * 256));
           __syncwarp();
           if (lane < npg)
-            tma_load_2d(st + kTile + lane * BS * 256, &tm_v, 0, (blk * Hkv + kvh) * BS * 2,
-                        &vfull[bi]);
+            tma_load_2d_hint(st + kTile + lane * BS * 256, &tm_v, 0, (blk * Hkv + kvh) * BS * 2,
+                             &vfull[bi], pol);
         } else {
           if (lane == 0) mbar_arrive(&vfull[bi]);
           __syncwarp();
