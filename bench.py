@@ -854,6 +854,29 @@ def long_block_size_sweep(ops, stream, rank, steps, use_graph):
     return res
 
 
+def long_few_sequences(ops, stream, rank, steps, use_graph):
+    """The long-context workload with 1, 2, 4 and 8 sequences (block size 32,
+    lengths 32K-128K): the decode call alone. Few (sequence, KV head) units
+    leave the split plan to spread each sequence over the streams."""
+    from paged_kv_cache_339_b200 import workloads as W
+    peak, _ = measured_peak()
+    res = {}
+    for n in (1, 2, 4, 8):
+        b = W.long_context("cuda", seed=1005 + 100 * rank, num_seqs=n)
+        B, Hq, D = b.q.shape
+        ws = ops.decode_workspace(B, Hq, D, b.max_context_len, b.block_size, 0)
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device="cuda")
+        d = time_decode_only(b, ops, out, ws, 0, ops.PA_PATH_AUTO, stream, steps, use_graph)
+        kb = b.kv_bytes_logical()
+        res[f"seqs{n}"] = {"kv_bytes": kb,
+                           "decode_gbps": round(kb / (d * 1e-3) / 1e9, 1),
+                           "frac_of_measured_peak": round(kb / (d * 1e-3) / 1e9 / peak, 4),
+                           "status": ops.pa_decode_status(ws, stream)}
+        del b, ws, out
+        torch.cuda.empty_cache()
+    return res
+
+
 def allocator_waste():
     """Reserved-but-unused fraction of the KV cache under max-length
     contiguous reservation and under paging at block sizes 8 / 16 / 32, over
@@ -902,6 +925,8 @@ def run_ours(args, rank, world, local):
             res["configs"][r["config"]["workload"]] = r
         res["next"] = next_rows(ops, stream, rank)
         res["next"]["long_block_size_sweep"] = long_block_size_sweep(
+            ops, stream, rank, max(10, args.steps // 2), not args.no_graph)
+        res["next"]["long_few_sequences"] = long_few_sequences(
             ops, stream, rank, max(10, args.steps // 2), not args.no_graph)
         res["next"]["allocator_waste"] = allocator_waste()
     return res
