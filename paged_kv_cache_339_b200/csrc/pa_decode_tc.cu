@@ -20,8 +20,10 @@
 //               position c belongs to stream c & 1): metadata, query row and
 //               the physical blocks read from the block table. It runs up to
 //               8 positions ahead through a shared-memory descriptor queue.
-//               When a stream runs out of items its positions carry END, then
-//               empty "bubble" slots, and finally a STOP for each stream.
+//               When a stream runs out of items its position carries END and
+//               the other stream takes every later position (its first chunk
+//               after that is marked SOLO), so a stream left alone at the end
+//               has the whole ring; two STOPs end the producer.
 //   warp 0      producer: for each descriptor loads each page's K and V tile
 //               (two 64-column halves each) plus the Q tile with 2-D TMA
 //               (128-byte swizzle) into a 3-stage ring; completion by mbarrier
@@ -51,7 +53,7 @@ namespace pa {
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
-constexpr int kFirst = 1, kLast = 2, kEnd = 4, kBubble = 8, kStop = 16;
+constexpr int kFirst = 1, kLast = 2, kEnd = 4, kSolo = 8, kStop = 16;
 constexpr int kChunk = 128;   // tokens per stage (= MMA M)
 constexpr int kD = 128;       // head_dim
 constexpr int kNst = 3;       // pipeline stages
@@ -255,9 +257,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Ly::OFF_BAR);
   // A stage holds K and Q' (released once the score MMA has read them) and V
   // (released after the P.V MMA), each with its own full / empty barriers.
-  // kfull / vfull[2 * stage + group]: one barrier per (stage, stream) so a
-  // stream's consumers see every phase of the barriers they wait on (the two
-  // streams alternate over an odd number of stages).
+  // kfull / vfull[2 * stage + (c & 1)]: one barrier per (stage, position
+  // parity), so the consumers of ring position c see every phase of the
+  // barrier they wait on: it serves every 2 x kNst-th position, and its phase
+  // parity at c is (c / (2 kNst)) & 1, whichever stream c belongs to.
   uint64_t* kfull = bars;                // [kNst][2]
   uint64_t* vfull = bars + 2 * kNst;     // [kNst][2]
   uint64_t* kempty = bars + 4 * kNst;    // [kNst]
@@ -330,8 +333,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ producer
     // Takes ring position c's descriptor from the scheduler, waits for the
     // stage halves, and issues the chunk's copies: Q' (two boxes) and one K
-    // box per page, then one V box per page; or forwards an END / bubble /
-    // STOP marker.
+    // box per page, then one V box per page; or forwards an END / STOP
+    // marker.
     if (lane == 0) {
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_q);
@@ -364,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int stage = c % kNst;
       const uint32_t epar = ((c / kNst) & 1u) ^ 1u;
       const int bi = 2 * stage + (c & 1);
-      const bool data = !(flags & (kEnd | kBubble | kStop));
+      const bool data = !(flags & (kEnd | kStop));
       uint8_t* st = smem + static_cast<size_t>(stage) * kStage;
       {
         // K and Q' (and the chunk's metadata) once the score MMA of the
@@ -499,16 +502,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_step(st1);
     int stops = 0;
     uint32_t c = 0;
-    // describe position c for stream `cur` (a chunk, or an END / bubble /
-    // STOP marker); returns false when the scheduler should stop
-    auto emit = [&](Stream& cur, const Stream& other) -> bool {
-      int kind = 0;   // 0 data, 1 end, 2 bubble, 3 stop
+    int solo = -1;            // once one stream has ended: the stream (0 / 1) that takes every position
+    bool solo_mark = false;   // its next chunk carries kSolo
+    // describe position c for stream t = `cur` (a chunk, or an END / STOP
+    // marker); returns false when the scheduler should stop
+    auto emit = [&](Stream& cur, const Stream& other, int t) -> bool {
+      int kind = 0;   // 0 data, 1 end, 3 stop
       if (!cur.ended && cur.cs >= cur.te) {
         // current item done: finish the prefetch of the next one, then switch
         while (cur.nst < 3) prefetch_step(cur);
         if (cur.nst == 4) {
           cur.ended = true;
           kind = 1;
+          if (!other.ended) {
+            solo = t ^ 1;
+            solo_mark = true;
+          }
         } else {
           cur.seq = cur.nseq;
           cur.kvh = cur.nkvh;
@@ -522,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           cur.nst = 0;
         }
       } else if (cur.ended) {
-        kind = other.ended ? 3 : 2;
+        kind = 3;   // a stream is only described again once both have ended
       }
       int valid = 0, npg = 0, blk = 0;
       if (kind == 0) {
@@ -559,7 +568,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           m.split_raw = cur.split_n;
           m.t0 = cur.cs;
           m.valid = valid;
-          m.flags = (cur.cs == cur.tb ? kFirst : 0) | (cur.cs + kChunk >= cur.te ? kLast : 0);
+          m.flags = (cur.cs == cur.tb ? kFirst : 0) | (cur.cs + kChunk >= cur.te ? kLast : 0) |
+                    (solo_mark ? kSolo : 0);
           m.pad0 = m.pad1 = 0;
           d.meta = m;
           d.q_row = cur.seq * p.num_q_heads + cur.kvh * G;
@@ -567,16 +577,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (lane < kMaxPages) d.blk[lane] = lane < npg ? blk : 0;
         cur.cs += kChunk;
+        solo_mark = false;
       } else if (lane == 0) {
-        d.meta.flags = kind == 1 ? kEnd : (kind == 2 ? kBubble : kStop);
+        d.meta.flags = kind == 1 ? kEnd : kStop;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&desc_full[qd]);
       ++c;
       return !(kind == 3 && ++stops == 2);
     };
-    while (emit(st0, st1) && emit(st1, st0)) {
+    // alternate until a stream ends (the position after its END belongs to
+    // the other stream), then the other stream alone
+    bool run = true;
+    while (run && solo < 0) {
+      run = emit(st0, st1, 0);
+      if (run && solo < 0) run = emit(st1, st0, 1);
     }
+    if (solo == 0)
+      while (run) run = emit(st0, st1, 0);
+    if (solo == 1)
+      while (run) run = emit(st1, st0, 1);
   } else if (warp == 1 || warp == 2) {
     // ------------------------------------------------------------ MMA issuers
     const int t = warp - 1;   // group served
@@ -590,13 +610,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t pb = smem_u32(pbuf) + t * Ly::PBUF;
       const uint32_t s_tm = tmem + t * Ly::COLS_PER_STREAM;   // two NS-column score tiles
       const uint32_t o_tm = s_tm + 2 * Ly::NS;
-      uint32_t n = 0;   // data chunks of this group so far
-      for (uint32_t c = t;; c += 2) {
+      uint32_t n = 0;      // data chunks of this group so far
+      uint32_t step = 2;   // 1 once this stream takes every position
+      for (uint32_t c = t;; c += step) {
         const int stage = c % kNst;
         const uint32_t fpar = (c / (2 * kNst)) & 1u;
-        if (!mbar_wait(&kfull[2 * stage + t], fpar, abrt, status)) break;
-        const ChunkMeta mt = meta[2 * stage + t];
+        const int bi = 2 * stage + static_cast<int>(c & 1u);
+        if (!mbar_wait(&kfull[bi], fpar, abrt, status)) break;
+        const ChunkMeta mt = meta[bi];
         if (mt.flags & kStop) break;
+        if (mt.flags & kSolo) step = 1;
         const uint32_t par = n & 1u;
         if (mt.flags & kEnd) {
           // release only after the softmax group has seen END (it acknowledges
@@ -607,15 +630,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           // V's slot only after the producer has passed this position's V half
           // (its vfull arrival): an earlier release would complete two phases
           // of vempty[] before the producer waits on the first
-          if (!mbar_wait(&vfull[2 * stage + t], fpar, abrt, status)) break;
+          if (!mbar_wait(&vfull[bi], fpar, abrt, status)) break;
           mbar_arrive(&vempty[stage]);
-          continue;
-        }
-        if (mt.flags & kBubble) {   // only this warp looks at bubbles
-          mbar_arrive(&kempty[stage]);
-          if (!mbar_wait(&vfull[2 * stage + t], fpar, abrt, status)) break;
-          mbar_arrive(&vempty[stage]);
-          continue;
+          break;   // the stream's last position (later ones go to the other stream)
         }
         // Half-row scores: the K region holds 256 half-rows (token, half) of
         // 128 B; Q' holds the query rows' first halves then their second
@@ -638,7 +655,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // O^T = V^T . P^T once the softmax group has written P and V has landed
         if (!mbar_wait(&p_full[t], par, abrt, status)) break;
         if (!mbar_wait(&o_free[t], par ^ 1u, abrt, status)) break;
-        if (!mbar_wait(&vfull[2 * stage + t], fpar, abrt, status)) break;
+        if (!mbar_wait(&vfull[bi], fpar, abrt, status)) break;
         tc_fence_after();
         const int nks = (mt.valid + 15) >> 4;
         for (int ks = 0; ks < nks; ++ks) {
@@ -719,11 +736,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       return true;
     };
 
-    for (uint32_t c = t;; c += 2) {
+    uint32_t step = 2;   // 1 once this stream takes every position
+    for (uint32_t c = t;; c += step) {
       const int stage = c % kNst;
       const uint32_t fpar = (c / (2 * kNst)) & 1u;
-      if (!__all_sync(kFull, mbar_wait(&kfull[2 * stage + t], fpar, abrt, status))) break;
-      const ChunkMeta mt = meta[2 * stage + t];
+      const int bi = 2 * stage + static_cast<int>(c & 1u);
+      if (!__all_sync(kFull, mbar_wait(&kfull[bi], fpar, abrt, status))) break;
+      const ChunkMeta mt = meta[bi];
+      if (mt.flags & kSolo) step = 1;
       if (mt.flags & kEnd) {
         if (Ly::DEFER_END && pend) {
           if (!group_sync(gbar, gphase, abrt, status)) break;
@@ -823,7 +843,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (own_t >= mt.valid && own_t < ((mt.valid + 15) & ~15)) {
         // past the chunk's valid tokens but inside the last 16-token step of
         // the P.V MMA: make V finite (zero) once the stage's V has landed
-        vok = mbar_wait(&vfull[2 * stage + t], fpar, abrt, status);
+        vok = mbar_wait(&vfull[bi], fpar, abrt, status);
         if (vok) {
           uint8_t* vrow = smem + static_cast<size_t>(stage) * kStage + vrow_off;
 #pragma unroll
