@@ -66,7 +66,19 @@ def parse():
                     help="mha only: pool size in blocks (0 = the workload's 16384)")
     ap.add_argument("--num-seqs", type=int, default=0,
                     help="mha / gqa / long: fewer sequences, for profiling a smaller case")
+    ap.add_argument("--no-share-prefixes", action="store_true",
+                    help="prefix_cow: read the shared prefix per sequence (pa_decode's "
+                         "share_prefixes off)")
     return ap.parse_args()
+
+
+# pa_decode reads shared prefixes once per group of sequences on workloads
+# built with one (prefix_cow), unless --no-share-prefixes
+SHARE_PREFIXES = [True]
+
+
+def share_for(b):
+    return bool(SHARE_PREFIXES[0] and "prefix_blocks" in b.meta)
 
 
 # ---------------------------------------------------------------------------
@@ -149,6 +161,7 @@ def config_of(b, name, l2_note):
         "context_len_mean": round(float(lens.float().mean()), 1),
         "context_len_max": int(lens.max()), "cow_pairs": int(b.cow_pairs.shape[0]),
         "kv_bytes_per_step": b.kv_bytes_logical(), "l2": l2_note,
+        "share_prefixes": share_for(b),
     }
 
 
@@ -264,6 +277,7 @@ class ClockSampler:
 
 def step_fn(b, ops, out, ws, split, path, stream):
     max_ctx = b.max_context_len
+    share = share_for(b)
 
     def step():
         n = 0
@@ -272,8 +286,9 @@ def step_fn(b, ops, out, ws, split, path, stream):
             n += 1
         ops.pa_write_kv(b.k_cache, b.v_cache, b.key, b.value, b.slot_mapping, stream=stream)
         ops.pa_decode(out, b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, max_ctx,
-                      b.scale, ws, split_tokens=split, path=path, stream=stream)
-        return n + 1 + 2   # write, plan, decode
+                      b.scale, ws, split_tokens=split, path=path, stream=stream,
+                      share_prefixes=share)
+        return n + 1 + 2 + (1 if share else 0)   # write, plan, (groups,) decode
     return step
 
 
@@ -370,15 +385,17 @@ def percentiles(ms_list, world):
     return {k: round(max_over_ranks(float(v), world), 5) for k, v in zip(("p10", "p50", "p90"), q)}
 
 
-def time_decode_only(b, ops, out, ws, split, path, stream, K, use_graph=True):
+def time_decode_only(b, ops, out, ws, split, path, stream, K, use_graph=True, share=None):
     """Average duration of the decode call alone (plan + main kernels):
     K calls back to back between two events on the launching stream, replayed
     from a CUDA graph like the step, so the device never waits for the host."""
     max_ctx = b.max_context_len
+    share = share_for(b) if share is None else share
 
     def call():
         ops.pa_decode(out, b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens,
-                      max_ctx, b.scale, ws, split_tokens=split, path=path, stream=stream)
+                      max_ctx, b.scale, ws, split_tokens=split, path=path, stream=stream,
+                      share_prefixes=share)
 
     torch.cuda.synchronize()   # inputs drawn on the default stream are complete
     with torch.cuda.stream(stream):
@@ -477,7 +494,7 @@ def time_e2e(b, ops, ws, split, path, stream, K, W):
                             stream=stream)
             ops.pa_decode(out[sl], d["q"], b.k_cache, b.v_cache, d["block_tables"],
                           d["context_lens"], max_ctx, b.scale, ws, split_tokens=split,
-                          path=path, stream=stream)
+                          path=path, stream=stream, share_prefixes=share_for(b))
             done[sl].record(stream)
 
     def download(i):
@@ -622,13 +639,16 @@ def uses_tensor_cores(b, path):
     return path == "tc" or (path == "auto" and fits)
 
 
-def kernel_source_hash(tensor_cores):
-    """Hash of the sources of the decode kernel that runs (the traffic figure
-    is only reported while it was measured on these exact sources)."""
+def kernel_source_hash(tensor_cores, groups=False):
+    """Hash of the sources of the decode kernels that run (the traffic figure
+    is only reported while it was measured on these exact sources); groups:
+    the shared-prefix launch (tensor-core kernel) runs too."""
     h = hashlib.sha256()
     csrc = ROOT / "paged_kv_cache_339_b200" / "csrc"
-    main = "pa_decode_tc.cu" if tensor_cores else "pa_decode_simt.cu"
-    for name in ("pa_common.cuh", main, "pa_plan_reduce.cu"):
+    main = ["pa_decode_tc.cu" if tensor_cores else "pa_decode_simt.cu"]
+    if groups and not tensor_cores:
+        main.append("pa_decode_tc.cu")
+    for name in ["pa_common.cuh"] + main + ["pa_plan_reduce.cu"]:
         h.update((csrc / name).read_bytes())
     return h.hexdigest()[:16]
 
@@ -757,7 +777,7 @@ def measure(name, args, ops, rank, world, local, stream, path, split, steps, cpu
     dec_gbps = kv_bytes / (dec_ms * 1e-3) / 1e9
     tc = uses_tensor_cores(b, {ops.PA_PATH_AUTO: "auto", ops.PA_PATH_SIMT: "simt",
                                ops.PA_PATH_TCGEN05: "tc"}[path])
-    khash = kernel_source_hash(tc)
+    khash = kernel_source_hash(tc, share_for(b))
     l2_note = (f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of KV read per step, not "
                "flushed; l2_flushed has per-step times with the L2 evicted before every step")
     if b.cow_pairs.numel():
@@ -777,7 +797,9 @@ def measure(name, args, ops, rank, world, local, stream, path, split, steps, cpu
         "gpu_launches": per_step * steps,
         "roofline": {
             "bound": "hbm", "kernel": "pa_decode (plan + decode main, merge fused)",
-            "decode_kernel": "tc_decode_kernel (tcgen05)" if tc else "simt_decode_kernel",
+            "decode_kernel": ("tc_decode_kernel (tcgen05)" if tc else "simt_decode_kernel") +
+                             (" after the shared-prefix groups' tc_decode_kernel"
+                              if share_for(b) else ""),
             "achieved": round(dec_gbps, 1), "peak": peak, "unit": "GB/s",
             "frac": round(dec_gbps / peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
             "algorithmic_bytes_per_launch": kv_bytes,
@@ -795,6 +817,17 @@ def measure(name, args, ops, rank, world, local, stream, path, split, steps, cpu
             gbps_at_p50=round(weak_scaling_value(kv_bytes_all, flushed["p50"]) / 1e9, 1),
             **flushed),
     }
+    if share_for(b):
+        # the same decode call with every sequence reading the prefix itself
+        off_ms = time_decode_only(b, ops, out, ws, split, path, stream, max(10, steps),
+                                  use_graph, share=False)
+        res["prefix_sharing"] = {
+            "note": "pa_decode share_prefixes: the common prefix is read once per group of "
+                    "up to 16 sequences; decode_gbps_without is the same call with it off",
+            "decode_gbps": round(dec_gbps, 1),
+            "decode_gbps_without": round(kv_bytes / (off_ms * 1e-3) / 1e9, 1),
+            "speedup": round(off_ms / dec_ms, 3),
+        }
     if b.cow_pairs.numel():
         # the shared prefix is read by every sibling but crosses HBM once per step
         ub = b.kv_bytes_unique()
@@ -967,6 +1000,7 @@ def run_reference(args, rank, world):
 
 def main():
     args = parse()
+    SHARE_PREFIXES[0] = not args.no_share_prefixes
     rank, world, local = dist_setup(args.gpus)
     try:
         if args.impl == "reference":

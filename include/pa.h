@@ -180,14 +180,29 @@ typedef struct {
      long except each sequence's last. */
   int32_t split_tokens;
   int32_t path;        /* a pa_decode_path */
+  /* 1 = read shared prefixes once per group of sequences (0 = off). Sequences
+     forked from one another point at the same physical blocks for their
+     common prefix ("Paged Attention: Virtual Memory for the KV Cache",
+     "Sharing comes almost for free"). With this option the planning kernel
+     compares each sequence's block table with the previous sequence's; runs
+     of consecutive sequences sharing at least 256 tokens form groups of up
+     to 16 query rows (16 / G sequences), and the whole pieces of their
+     common prefix (pieces of at most 512 tokens unless split_tokens is set)
+     are computed once for the group, reading each shared block once for all
+     its members (on the tensor cores for 16-bit KV with head_dim 128 and G
+     dividing 16, else on the CUDA cores), then merged with each member's own
+     pieces. Results equal the per-sequence ones up to fp32 rounding. Applies
+     to batches of 2 to 1024 sequences with G <= 8; elsewhere the option
+     changes nothing. */
+  int32_t share_prefixes;
 } pa_decode_options;
 
 /*
  * pa_decode_workspace_size - bytes of device workspace pa_decode needs for the
  * given shapes (status word and plan, work list, piece counts, the list of
- * sequences cut into pieces, a merge counter per (sequence, KV head), one
- * partial result per (sequence, query head, piece)). split_tokens as in
- * pa_decode_options.
+ * sequences cut into pieces, a merge counter per (sequence, KV head), the
+ * list of pieces shared by groups of sequences, one partial result per
+ * (sequence, query head, piece)). split_tokens as in pa_decode_options.
  */
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
                                 int32_t head_dim, int32_t max_context_len,
@@ -226,7 +241,9 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
  * planning kernel keeps the lengths in one CTA's shared memory), and for
  * num_seqs * num_q_heads of 2^31 or more (query rows are 32-bit copy
  * coordinates).
- * Enqueues two kernels: a planning kernel, then the decode kernel. The
+ * Enqueues two kernels: a planning kernel, then the decode kernel (three
+ * with share_prefixes: the groups' shared pieces run as a decode launch of
+ * their own before the decode kernel). The
  * planning kernel is launched with programmatic stream serialisation: it may
  * start while the kernel before it in the stream is finishing: it reads
  * context_lens and rewrites the workspace at once, then waits for that

@@ -110,7 +110,9 @@ pa_status check_decode_args(const pa_kv_cache* cache, const float* out, const vo
   if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
   const int32_t split = opts ? opts->split_tokens : 0;
   const int32_t path = opts ? opts->path : PA_PATH_AUTO;
+  const int32_t share = opts ? opts->share_prefixes : 0;
   if (split < 0 || path < PA_PATH_AUTO || path > PA_PATH_TCGEN05) return PA_ERR_INVALID_ARG;
+  if (share != 0 && share != 1) return PA_ERR_INVALID_ARG;
   if (split > 0) {
     if (split % cache->block_size != 0) return PA_ERR_INVALID_ARG;
     if (max_context_len > 0 && ceil_div(max_context_len, split) > kMaxSplits)
@@ -119,6 +121,7 @@ pa_status check_decode_args(const pa_kv_cache* cache, const float* out, const vo
   ch->group = group;
   ch->split = split;
   ch->use_tc = false;
+  ch->share = false;
   ch->empty = num_seqs == 0;
   if (ch->empty) return PA_OK;
   if (out == nullptr || q == nullptr || block_tables == nullptr || context_lens == nullptr)
@@ -146,6 +149,9 @@ pa_status check_decode_args(const pa_kv_cache* cache, const float* out, const vo
   }
   if (!use_tc && !simt_supported(cache->dtype, cache->head_dim, group)) return PA_ERR_UNSUPPORTED;
   ch->use_tc = use_tc;
+  // shared prefixes are read once per group of at least two sequences (at
+  // most 16 query rows: G <= 8), for batches of up to kShareMaxSeqs
+  ch->share = share == 1 && group <= 8 && num_seqs >= 2 && num_seqs <= kShareMaxSeqs;
   return PA_OK;
 }
 
@@ -294,6 +300,19 @@ pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
   pp.max_splits = lay.max_splits;
   // the tensor-core kernel runs two independent item streams per CTA
   pp.num_ctas = use_tc ? 2 * ctas : ctas;
+  pp.block_tables = block_tables;
+  pp.share_prefixes = ch.share ? 1 : 0;
+  pp.share_members = 16 / group;
+  pp.gpairs_off = lay.gpairs_off;
+  // the group list runs on the tensor cores where its 16-row tiles fit
+  // (16-bit KV, head_dim 128, G dividing 16), else on the CUDA cores
+  const bool tc_groups = ch.share && tc_group_supported(cache->dtype, cache->head_dim, group);
+  int gctas = 0;
+  if (ch.share) {
+    e = cached_ctas(tc_groups, cache->dtype, cache->head_dim, 16, &gctas);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  pp.group_ctas = tc_groups ? 2 * gctas : gctas;   // item streams of that launch
   e = launch_plan(pp, s);
   if (e != cudaSuccess) return cuda_fail(e);
 
@@ -320,6 +339,15 @@ pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
   dp.max_splits = lay.max_splits;
   dp.scale_log2 = scale * 1.4426950408889634f;
   dp.dtype = cache->dtype;
+  dp.gpairs_off = lay.gpairs_off;
+  if (ch.share) {
+    // the groups' common pieces first (each member's piece is counted there),
+    // then every sequence's own pieces
+    dp.group_mode = 1;
+    e = tc_groups ? launch_decode_tc_groups(dp, gctas, s) : launch_decode_simt_groups(dp, gctas, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  dp.group_mode = 0;
   e = use_tc ? launch_decode_tc(dp, ctas, s) : launch_decode_simt(dp, ctas, s);
   if (e != cudaSuccess) return cuda_fail(e);
 

@@ -131,6 +131,17 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
   return pol;
 }
+// 3-D tiled TMA load of the box at (x, y, z) of `tmap` (x innermost, in
+// elements; x * element size a multiple of 16 bytes).
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* tmap, int32_t x,
+                                            int32_t y, int32_t z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::"
+      "complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // tma_load_2d with an L2 cache policy.
 __device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* tmap, int32_t x,
                                                  int32_t y, uint64_t* bar, uint64_t pol) {

@@ -106,10 +106,12 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-template <typename T, int D, int GPW>
+// GRP: the launch over the group list of shared prefixes (group items only).
+template <typename T, int D, int GPW, bool GRP>
 __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
     simt_decode_kernel(const DecodeParams p) {
   __shared__ volatile int s_last;   // this piece completed its sequence
+  __shared__ volatile int s_lastm[16];   // group items: this piece completed member m
   using Tr = SimtTraits<T, D, GPW>;
   constexpr int CHUNK = Tr::CHUNK, ROW = Tr::ROW, NST = Tr::NST;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -139,12 +141,15 @@ __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
   pdl_wait();   // the plan (and the KV write before it) are complete from here on
   // (no early launch of dependents: the next call's plan rewrites the workspace)
 
-  const int num_items = hdr->num_items;
+  // the group list (shared prefixes) or the work list
+  const int num_items = GRP ? hdr->num_group_items : hdr->num_items;
+  int* const work_counter = GRP ? &hdr->group_work_counter : &hdr->work_counter;
   const int Hkv = p.num_kv_heads, BS = p.block_size;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    const WorkPair* pairs = reinterpret_cast<const WorkPair*>(p.ws + p.pairs_off);
+    const WorkPair* pairs =
+        reinterpret_cast<const WorkPair*>(p.ws + (GRP ? p.gpairs_off : p.pairs_off));
     const uint64_t pol = l2_evict_first_policy();   // K and V tiles: read once per call
     uint32_t c = 0;
     bool ok = true;
@@ -161,7 +166,7 @@ __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
         // next claim in flight two chunks before this item ends (a claim held
         // for a whole item would lengthen the tail)
         if (!claimed && wp.t_end - cs <= 2 * CHUNK) {
-          if (lane == 0) kraw = atomicAdd(&hdr->work_counter, 1);
+          if (lane == 0) kraw = atomicAdd(work_counter, 1);
           claimed = true;
         }
         const int valid = min(CHUNK, wp.t_end - cs);
@@ -219,7 +224,7 @@ __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
         ++c;
       }
       if (!ok) break;
-      if (!claimed && lane == 0) kraw = atomicAdd(&hdr->work_counter, 1);
+      if (!claimed && lane == 0) kraw = atomicAdd(work_counter, 1);
       k = __shfl_sync(kFull, kraw, 0);
     }
     if (ok) {
@@ -242,7 +247,9 @@ __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
     // ------------------------------------------------------------ consumers
     const int cw = warp - 1;
     const int G = p.num_q_heads / Hkv;
-    const int HG = (G + GPW - 1) / GPW;
+    // query rows an item has at most: G, or 16 for group items (members x G)
+    const int GL = GRP ? 16 : G;
+    const int HG = (GL + GPW - 1) / GPW;
     const int HGp = HG <= 1 ? 1 : (HG <= 2 ? 2 : 4);
     const int WPG = Tr::NCW / HGp;
     const int hg = cw / WPG, wg = cw % WPG;
@@ -286,10 +293,18 @@ __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
           l[g] = 0.f;
 #pragma unroll
           for (int e = 0; e < Tr::EPL; ++e) o[g][e] = 0.f;
+          // query row of row slot hl (spare slots repeat the first row): head
+          // hl of the sequence, or for a group item head hl % G of member hl / G
           const int hl = hg * GPW + g;
-          const int hq = mt.kvh * G + (hl < G ? hl : 0);
-          const uint8_t* qrow = static_cast<const uint8_t*>(p.q) +
-                                (static_cast<size_t>(mt.seq) * p.num_q_heads + hq) * ROW;
+          size_t qr;
+          if constexpr (GRP) {
+            const int hr = hl < item_nsplit(mt.split_raw) * G ? hl : 0;
+            const int mb = hr / G;
+            qr = static_cast<size_t>(mt.seq + mb) * p.num_q_heads + mt.kvh * G + (hr - mb * G);
+          } else {
+            qr = static_cast<size_t>(mt.seq) * p.num_q_heads + mt.kvh * G + (hl < G ? hl : 0);
+          }
+          const uint8_t* qrow = static_cast<const uint8_t*>(p.q) + qr * ROW;
 #pragma unroll
           for (int v = 0; v < Tr::NV; ++v) {
             float f[Tr::EPV];
@@ -399,45 +414,90 @@ __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
         }
         if (!group_sync(&gbar[0], gphase, abrt, status)) break;
         const int tid = threadIdx.x - 32;
-        const int nsp = item_nsplit(mt.split_raw);
-        const bool single = nsp == 1;
-        const int split = item_split(mt.split_raw);
         float2* ml = reinterpret_cast<float2*>(p.ws + p.ml_off);
         float* po = reinterpret_cast<float*>(p.ws + p.o_off);
-        const size_t row0 = static_cast<size_t>(mt.seq) * p.num_q_heads + mt.kvh * G;
-        for (int idx = tid; idx < G * D; idx += Tr::NCW * 32) {
-          const int h = idx / D, d = idx - (idx / D) * D;
+        int* cnt = reinterpret_cast<int*>(p.ws + p.cnt_off);
+        // row h of the item, merged over the warps of its head group
+        auto combine = [&](int h, int d, float& M, float& L, float& O) {
           const int hgi = h / GPW, g = h - hgi * GPW;
-          float M = -INFINITY;
+          M = -INFINITY;
           for (int w = 0; w < WPG; ++w) M = fmaxf(M, cmb[(hgi * WPG + w) * Tr::CMB + GPW * D + g]);
-          float L = 0.f, O = 0.f;
+          L = 0.f;
+          O = 0.f;
           for (int w = 0; w < WPG; ++w) {
             const float* src = cmb + (hgi * WPG + w) * Tr::CMB;
             const float sc = exp2f(src[GPW * D + g] - M);
             L = fmaf(src[GPW * D + GPW + g], sc, L);
             O = fmaf(src[g * D + d], sc, O);
           }
-          const size_t row = row0 + h;
-          if (single) {
-            p.out[row * D + d] = O / L;
-          } else {
-            const size_t pr_ = row * p.max_splits + split;
-            po[pr_ * D + d] = O;
-            if (d == 0) ml[pr_] = make_float2(M, L);
+        };
+        const int split = item_split(mt.split_raw);
+        if (GRP) {
+          // A group item: whole pieces common to `members` consecutive
+          // sequences (the same physical blocks), rows h = member x G + head.
+          // Each member counts the piece on its own (sequence, KV head)
+          // counter; a member whose pieces are then all counted is merged
+          // here, as by the last piece of any split sequence.
+          const int members = item_nsplit(mt.split_raw);
+          const int32_t* nsplit_of = reinterpret_cast<const int32_t*>(p.ws + p.nsplit_off);
+          for (int idx = tid; idx < members * G * D; idx += Tr::NCW * 32) {
+            const int h = idx / D, d = idx - (idx / D) * D;
+            float M, L, O;
+            combine(h, d, M, L, O);
+            const int mb = h / G;
+            const size_t row = static_cast<size_t>(mt.seq + mb) * p.num_q_heads + mt.kvh * G + (h - mb * G);
+            if (nsplit_of[mt.seq + mb] == 1) {
+              p.out[row * D + d] = O / L;
+            } else {
+              const size_t pr_ = row * p.max_splits + split;
+              po[pr_ * D + d] = O;
+              if (d == 0) ml[pr_] = make_float2(M, L);
+            }
           }
-        }
-        if (!single) __threadfence();   // this piece's partial result, before it is counted
-        if (!group_sync(&gbar[0], gphase, abrt, status)) break;
-        if (!single) {
-          // the last piece of the (sequence, KV head) to finish merges them all
-          if (tid == 0)
-            s_last = atomicAdd(reinterpret_cast<int*>(p.ws + p.cnt_off) +
-                                   static_cast<size_t>(mt.seq) * Hkv + mt.kvh,
-                               1) == nsp - 1;
+          __threadfence();   // the partial results, before they are counted
           if (!group_sync(&gbar[0], gphase, abrt, status)) break;
-          if (s_last) {
+          if (tid < members) {
+            const int sq = mt.seq + tid;
+            const int nspm = nsplit_of[sq];
+            s_lastm[tid] = nspm > 1 &&
+                           atomicAdd(cnt + static_cast<size_t>(sq) * Hkv + mt.kvh, 1) == nspm - 1;
+          }
+          if (!group_sync(&gbar[0], gphase, abrt, status)) break;
+          for (int mb = 0; mb < members; ++mb) {
+            if (!s_lastm[mb]) continue;
             __threadfence();   // every other piece counted before us is visible
-            merge_split_rows(p.out, ml, po, row0, G, D, nsp, p.max_splits, tid, Tr::NCW * 32);
+            const int sq = mt.seq + mb;
+            merge_split_rows(p.out, ml, po, static_cast<size_t>(sq) * p.num_q_heads + mt.kvh * G, G,
+                             D, nsplit_of[sq], p.max_splits, tid, Tr::NCW * 32);
+          }
+        } else {
+          const int nsp = item_nsplit(mt.split_raw);
+          const bool single = nsp == 1;
+          const size_t row0 = static_cast<size_t>(mt.seq) * p.num_q_heads + mt.kvh * G;
+          for (int idx = tid; idx < G * D; idx += Tr::NCW * 32) {
+            const int h = idx / D, d = idx - (idx / D) * D;
+            float M, L, O;
+            combine(h, d, M, L, O);
+            const size_t row = row0 + h;
+            if (single) {
+              p.out[row * D + d] = O / L;
+            } else {
+              const size_t pr_ = row * p.max_splits + split;
+              po[pr_ * D + d] = O;
+              if (d == 0) ml[pr_] = make_float2(M, L);
+            }
+          }
+          if (!single) __threadfence();   // this piece's partial result, before it is counted
+          if (!group_sync(&gbar[0], gphase, abrt, status)) break;
+          if (!single) {
+            // the last piece of the (sequence, KV head) to finish merges them all
+            if (tid == 0)
+              s_last = atomicAdd(cnt + static_cast<size_t>(mt.seq) * Hkv + mt.kvh, 1) == nsp - 1;
+            if (!group_sync(&gbar[0], gphase, abrt, status)) break;
+            if (s_last) {
+              __threadfence();   // every other piece counted before us is visible
+              merge_split_rows(p.out, ml, po, row0, G, D, nsp, p.max_splits, tid, Tr::NCW * 32);
+            }
           }
         }
       }
@@ -447,10 +507,10 @@ __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
   __syncthreads();
 }
 
-template <typename T, int D, int GPW>
+template <typename T, int D, int GPW, bool GRP = false>
 cudaError_t launch_t(const DecodeParams& p, int num_ctas, cudaStream_t stream) {
   using Tr = SimtTraits<T, D, GPW>;
-  auto kern = simt_decode_kernel<T, D, GPW>;
+  auto kern = simt_decode_kernel<T, D, GPW, GRP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(Tr::SMEM));
   if (e != cudaSuccess) return e;
@@ -459,9 +519,14 @@ cudaError_t launch_t(const DecodeParams& p, int num_ctas, cudaStream_t stream) {
 }
 
 template <typename T, int D, int GPW>
+cudaError_t launch_groups_t(const DecodeParams& p, int num_ctas, cudaStream_t stream) {
+  return launch_t<T, D, GPW, true>(p, num_ctas, stream);
+}
+
+template <typename T, int D, int GPW>
 cudaError_t ctas_t(int* n) {
   using Tr = SimtTraits<T, D, GPW>;
-  auto kern = simt_decode_kernel<T, D, GPW>;
+  auto kern = simt_decode_kernel<T, D, GPW, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(Tr::SMEM));
   if (e != cudaSuccess) return e;
@@ -523,6 +588,13 @@ cudaError_t launch_decode_simt(const DecodeParams& p, int num_ctas, cudaStream_t
   const int dtype = p.dtype, head_dim = p.head_dim, group = p.num_q_heads / p.num_kv_heads;
   if (!simt_supported(dtype, head_dim, group)) return cudaErrorInvalidValue;
   PA_SIMT_DISPATCH(launch_t, p, num_ctas, stream);
+}
+
+cudaError_t launch_decode_simt_groups(const DecodeParams& p, int num_ctas, cudaStream_t stream) {
+  // 16 query rows per item: the 4-rows-per-warp flavour
+  const int dtype = p.dtype, head_dim = p.head_dim, group = 16;
+  if (!p.group_mode || !simt_supported(dtype, head_dim, group)) return cudaErrorInvalidValue;
+  PA_SIMT_DISPATCH(launch_groups_t, p, num_ctas, stream);
 }
 
 }  // namespace pa

@@ -241,7 +241,8 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-template <typename T, int GT>
+// GRP: the launch over the group list of shared prefixes (group items only).
+template <typename T, int GT, bool GRP>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v,
@@ -325,7 +326,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_wait();   // the plan (and the KV write before it) are complete from here on
   // (no early launch of dependents: the next call's plan rewrites the workspace)
 
-  const int num_items = hdr->num_items;
+  // the group list (shared prefixes) or the work list
+  const int num_items = GRP ? hdr->num_group_items : hdr->num_items;
   const int Hkv = p.num_kv_heads, BS = p.block_size;
   const int G = p.num_q_heads / Hkv;
 
@@ -356,11 +358,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int npg = d.npg;
       const int blk = d.blk[lane & (kMaxPages - 1)];
       uint4 m0 = make_uint4(0, 0, 0, 0), m1 = m0;
-      int q_row = 0;
+      int q_row = 0, q_y = 0;
       if (lane == 0) {
         m0 = reinterpret_cast<const uint4*>(&d.meta)[0];
         m1 = reinterpret_cast<const uint4*>(&d.meta)[1];
         q_row = d.q_row;
+        q_y = d.pad0;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&desc_empty[qd]);   // every lane has its copy of the descriptor
@@ -384,8 +387,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             // rows, first halves then second halves (NS/2 rows each)
             mbar_arrive_expect_tx(&kfull[bi],
                                   static_cast<uint32_t>(npg * BS * 256 + Ly::NS * 128));
-            tma_load_2d(st + 2 * kTile, &tm_q, 0, q_row, &kfull[bi]);
-            tma_load_2d(st + 2 * kTile + (Ly::NS / 2) * 128, &tm_q, 64, q_row, &kfull[bi]);
+            if (GRP) {
+              tma_load_3d(st + 2 * kTile, &tm_q, 0, q_y, q_row, &kfull[bi]);
+              tma_load_3d(st + 2 * kTile + (Ly::NS / 2) * 128, &tm_q, 64, q_y, q_row, &kfull[bi]);
+            } else {
+              tma_load_2d(st + 2 * kTile, &tm_q, 0, q_row, &kfull[bi]);
+              tma_load_2d(st + 2 * kTile + (Ly::NS / 2) * 128, &tm_q, 64, q_row, &kfull[bi]);
+            }
           }
           __syncwarp();
           if (lane < npg)
@@ -434,7 +442,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // table and writes one descriptor per position, up to kQd positions ahead
     // of the producer, so none of this global-memory latency sits on the copy
     // issue path.
-    const WorkPair* pairs = reinterpret_cast<const WorkPair*>(p.ws + p.pairs_off);
+    const WorkPair* pairs =
+        reinterpret_cast<const WorkPair*>(p.ws + (GRP ? p.gpairs_off : p.pairs_off));
+    int* const work_counter = GRP ? &hdr->group_work_counter : &hdr->work_counter;
     // Per-stream state (warp-uniform), plus a window of block-table entries:
     // lane j holds entries wbase + j and wbase + 32 + j of the current item.
     // The next item of each stream is prefetched one step per emission
@@ -458,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     auto claim = [&]() {
       int kr = 0;
-      if (lane == 0) kr = atomicAdd(&hdr->work_counter, 1);
+      if (lane == 0) kr = atomicAdd(work_counter, 1);
       return kr;
     };
     // one prefetch step for the next item of stream `cur`
@@ -572,7 +582,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     (solo_mark ? kSolo : 0);
           m.pad0 = m.pad1 = 0;
           d.meta = m;
-          d.q_row = cur.seq * p.num_q_heads + cur.kvh * G;
+          // the query rows: G heads of the sequence (a row of the [B * Hq,
+          // 128] map), or for a group item, from its first member on, G heads
+          // of each member (the [B, Hq, 128] map at (kvh * G, seq))
+          d.q_row = GRP ? cur.seq : cur.seq * p.num_q_heads + cur.kvh * G;
+          d.pad0 = cur.kvh * G;
           d.npg = npg;
         }
         if (lane < kMaxPages) d.blk[lane] = lane < npg ? blk : 0;
@@ -712,14 +726,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     // all of them; false when a barrier gave up
     auto finish = [&](const float* lr, int seq, int kvh, int split_raw, const float* ov_,
                       const float* mv_) -> bool {
-      const int nsp = item_nsplit(split_raw);
+      // a group item (shared prefix) is a piece of each of its members,
+      // never their only one (each keeps a piece of its own); its rows are
+      // member x G + head
+      const int members = GRP ? item_nsplit(split_raw) : 1;
+      const int nsp = GRP ? 0 : item_nsplit(split_raw);
+      const int rows = members * G;
       const int split = item_split(split_raw);
       const size_t row0 = static_cast<size_t>(seq) * p.num_q_heads + kvh * G;
 #pragma unroll
       for (int g = 0; g < GT; ++g) {
-        if (g >= G) break;
+        if (g >= rows) break;
         const float L = lr[g] + lr[16 + g] + lr[32 + g] + lr[48 + g];
-        const size_t row = row0 + g;
+        size_t row = row0 + g;
+        if constexpr (GRP) {
+          const int mb = g / G;
+          row = row0 + static_cast<size_t>(mb) * p.num_q_heads + (g - mb * G);
+        }
         if (nsp == 1) {
           p.out[row * kD + r] = ov_[g] / L;
         } else {
@@ -731,8 +754,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (nsp == 1) return true;
       __threadfence();   // this piece's partial result, before it is counted
       if (!group_sync(gbar, gphase, abrt, status)) return false;
-      // counted; the merge runs after the main loop (merge tasks below)
-      if (wq == 0 && lane == 0) atomicAdd(cnt + static_cast<size_t>(seq) * Hkv + kvh, 1);
+      // counted (for each member); the merge runs after the main loop (merge
+      // tasks below), in the launch of the members' own pieces for group items
+      if (wq == 0 && lane < members) atomicAdd(cnt + static_cast<size_t>(seq + lane) * Hkv + kvh, 1);
       return true;
     };
 
@@ -744,6 +768,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!__all_sync(kFull, mbar_wait(&kfull[bi], fpar, abrt, status))) break;
       const ChunkMeta mt = meta[bi];
       if (mt.flags & kSolo) step = 1;
+      // query rows of the chunk's item: G, or members x G for a group item
+      const int rows = GRP ? item_nsplit(mt.split_raw) * G : G;
       if (mt.flags & kEnd) {
         if (Ly::DEFER_END && pend) {
           if (!group_sync(gbar, gphase, abrt, status)) break;
@@ -800,8 +826,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         float b = hh ? sv1[Ly::NS / 2 + g] : sv1[g];
         a += __shfl_xor_sync(kFull, a, sh);
         b += __shfl_xor_sync(kFull, b, sh);
-        sa[g] = (ok0 && g < G) ? a * sl2 : -INFINITY;
-        sb[g] = (ok1 && g < G) ? b * sl2 : -INFINITY;
+        sa[g] = (ok0 && g < rows) ? a * sl2 : -INFINITY;
+        sb[g] = (ok1 && g < rows) ? b * sl2 : -INFINITY;
       }
       // ---- chunk max per head across the group's 128 threads
       float* rb = red_t + par * 64;
@@ -821,7 +847,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int g = 0; g < GT; ++g) {
         const float cm = fmaxf(fmaxf(rb[g], rb[16 + g]), fmaxf(rb[32 + g], rb[48 + g]));
         const float mn = fmaxf(m_run[g], cm);
-        // heads g >= G never see a finite score; keep them inert (alpha 0, p 0)
+        // rows g >= rows never see a finite score; keep them inert (alpha 0, p 0)
         alpha[g] = (mn == -INFINITY) ? 0.f : ex2(m_run[g] - mn);
         const float own_s = hh ? sb[g] : sa[g];
         const float pr = (mn == -INFINITY) ? 0.f : ex2(own_s - mn);
@@ -912,7 +938,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // registers; the groups that finish first share the merges out. A group
     // waits only on pieces that streams of running CTAs have claimed (every
     // item was claimed before any stream saw END), so every wait ends.
-    if (!*abrt) {
+    // (None in the launch over the group list: its pieces are merged by the
+    // launch of the members' own pieces, which runs after it.)
+    if (!GRP && !*abrt) {
       const int32_t* split_list = reinterpret_cast<const int32_t*>(p.ws + p.split_off);
       const int32_t* nsplit_of = reinterpret_cast<const int32_t*>(p.ws + p.nsplit_off);
       const int Hq = p.num_q_heads;
@@ -1022,7 +1050,28 @@ cudaError_t make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t r
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <typename T, int GT>
+// 3-D map over q as [num_seqs, num_q_heads, 128] 16-bit elements, box = 64
+// columns x G heads x 16 / G sequences (16 rows in the 2-D box's order),
+// 128-byte swizzle; sequences past the end read as zero.
+cudaError_t make_q_group_map(CUtensorMap* m, const void* q, int num_seqs, int num_q_heads, int G,
+                             bool bf16) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  if (G < 1 || 16 % G != 0) return cudaErrorInvalidValue;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(num_q_heads),
+                        static_cast<cuuint64_t>(num_seqs)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(kD) * 2,
+                           static_cast<cuuint64_t>(num_q_heads) * kD * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(16 / G)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                  const_cast<void*>(q), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <typename T, int GT, bool GRP = false>
 cudaError_t launch_t(const DecodeParams& p, int num_ctas, cudaStream_t stream) {
   using Ly = TcLayout<GT>;
   const bool bf16 = std::is_same<T, __nv_bfloat16>::value;
@@ -1033,12 +1082,20 @@ cudaError_t launch_t(const DecodeParams& p, int num_ctas, cudaStream_t stream) {
       static_cast<uint64_t>(p.num_blocks) * p.num_kv_heads * p.block_size * 2;
   cudaError_t e = make_map(&mk, p.k_cache, 64, half_rows, 128, 2 * p.block_size, bf16);
   if (e == cudaSuccess) e = make_map(&mv, p.v_cache, 64, half_rows, 128, 2 * p.block_size, bf16);
-  // q as [rows, 128]: one box per column half, NS/2 query rows
-  if (e == cudaSuccess)
-    e = make_map(&mq, p.q, kD, static_cast<uint64_t>(p.num_seqs) * p.num_q_heads, kD * 2,
-                 Ly::NS / 2, bf16);
+  // q as [rows, 128]: one box per column half, NS/2 query rows; for the
+  // group list, the rows of G heads of 16 / G consecutive sequences
+  if (e == cudaSuccess) {
+    if constexpr (GRP) {
+      static_assert(Ly::NS / 2 == 16, "group items fill a 16-row tile");
+      e = make_q_group_map(&mq, p.q, p.num_seqs, p.num_q_heads, p.num_q_heads / p.num_kv_heads,
+                           bf16);
+    } else {
+      e = make_map(&mq, p.q, kD, static_cast<uint64_t>(p.num_seqs) * p.num_q_heads, kD * 2,
+                   Ly::NS / 2, bf16);
+    }
+  }
   if (e != cudaSuccess) return e;
-  auto kern = tc_decode_kernel<T, GT>;
+  auto kern = tc_decode_kernel<T, GT, GRP>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(Ly::SMEM));
   if (e != cudaSuccess) return e;
@@ -1061,6 +1118,18 @@ cudaError_t tc_num_ctas(int dtype, int group, int* num_ctas) {
   (void)group;
   *num_ctas = num_sms();   // one CTA per SM (shared memory and TMEM sized for it)
   return cudaSuccess;
+}
+
+bool tc_group_supported(int dtype, int head_dim, int group) {
+  return (dtype == 1 || dtype == 2) && head_dim == kD && group >= 1 && group <= 8 &&
+         16 % group == 0 && encode_fn() != nullptr;
+}
+
+cudaError_t launch_decode_tc_groups(const DecodeParams& p, int num_ctas, cudaStream_t stream) {
+  const int group = p.num_q_heads / p.num_kv_heads;
+  if (!p.group_mode || !tc_group_supported(p.dtype, p.head_dim, group)) return cudaErrorInvalidValue;
+  if (p.dtype == 2) return launch_t<__nv_bfloat16, 16, true>(p, num_ctas, stream);
+  return launch_t<__half, 16, true>(p, num_ctas, stream);
 }
 
 cudaError_t launch_decode_tc(const DecodeParams& p, int num_ctas, cudaStream_t stream) {

@@ -21,6 +21,14 @@ struct PlanParams {
   int32_t min_split;      // lower bound of an automatic split
   int32_t max_splits;
   int32_t num_ctas;       // item streams of the decode kernel (CTAs x streams per CTA)
+  // shared prefixes (share_prefixes = 1): groups of consecutive sequences
+  // whose tables start with the same blocks; their common whole pieces go to
+  // a list of their own (gpairs_off), taken by a CUDA-core launch of
+  // group_ctas CTAs that reads each shared tile once for up to share_members
+  // sequences
+  const int32_t* block_tables;
+  int32_t share_prefixes, share_members, group_ctas;
+  size_t gpairs_off;
 };
 
 // Everything a decode main kernel needs; filled by the C-ABI shim.
@@ -36,7 +44,15 @@ struct DecodeParams {
       block_size, num_seqs, max_splits;
   float scale_log2;  // scale * log2(e): scores kept in log2 units
   int32_t dtype;     // pa_dtype
+  // 1: this launch takes the group list (shared prefixes): an item is a run
+  // of whole pieces common to `members` consecutive sequences, its query rows
+  // those sequences' rows of the KV head (CUDA-core kernel only)
+  int32_t group_mode;
+  size_t gpairs_off;
 };
+
+// Largest batch whose shared prefixes pa_decode looks for.
+constexpr int32_t kShareMaxSeqs = 1024;
 
 // Launched with programmatic stream serialisation (PDL): the plan may be
 // scheduled while its predecessor in the stream (the KV write) finishes.
@@ -47,12 +63,20 @@ bool simt_supported(int dtype, int head_dim, int group);
 cudaError_t simt_num_ctas(int dtype, int head_dim, int group, int* num_ctas);
 cudaError_t launch_decode_simt(const DecodeParams& p, int num_ctas,
                                cudaStream_t stream);
+// The CUDA-core kernel over the group list (16 query rows per item).
+cudaError_t launch_decode_simt_groups(const DecodeParams& p, int num_ctas,
+                                      cudaStream_t stream);
 
 // Tensor-core (tcgen05) decode for 16-bit KV, head_dim 128, 4 <= G <= 16.
 bool tc_supported(int dtype, int head_dim, int group);
 cudaError_t tc_num_ctas(int dtype, int group, int* num_ctas);
 cudaError_t launch_decode_tc(const DecodeParams& p, int num_ctas,
                              cudaStream_t stream);
+// The tensor-core kernel over the group list: 16-row tiles of 16 / G
+// sequences x G heads (16-bit KV, head_dim 128, G a divisor of 16 up to 8).
+bool tc_group_supported(int dtype, int head_dim, int group);
+cudaError_t launch_decode_tc_groups(const DecodeParams& p, int num_ctas,
+                                    cudaStream_t stream);
 
 // KV write and block copy.
 cudaError_t launch_write_kv(void* k_cache, void* v_cache, const void* key,
@@ -94,6 +118,7 @@ struct DecodeChoice {
   int group;       // query heads per KV head
   int32_t split;   // explicit split (0 = automatic)
   bool use_tc;     // tensor-core kernel (else CUDA cores)
+  bool share;      // look for shared prefixes (CUDA-core path, 2..1024 sequences)
   bool empty;      // no sequences: nothing to enqueue
 };
 

@@ -22,6 +22,8 @@
 // the workspace), and waits for that kernel before it writes the zero rows of
 // empty sequences into `out` and exits, so the decode kernel that waits on
 // the plan also sees the new tokens.
+#include <climits>
+
 #include "pa_common.cuh"
 #include "pa_internal.h"
 
@@ -31,6 +33,10 @@ namespace {
 
 constexpr int kPlanMaxThreads = 1024;
 constexpr int kKeys = 64;   // length buckets: 1..63 chunks of 128 tokens, and >= 64 chunks
+// Shared prefixes: a group needs at least this many common tokens, and its
+// common whole pieces are at most this long (automatic split).
+constexpr int kShareMinTokens = 256;
+constexpr int kShareSplit = 512;
 
 __device__ __forceinline__ int piece_key(int tokens) {
   const int k = (tokens + 127) >> 7;
@@ -67,6 +73,58 @@ __device__ __forceinline__ void seq_pieces(int L, const PieceRule& r, int& nA, i
   k = (rest + sb - 1) / sb;
 }
 
+// Inclusive scans over the CTA's threads in thread order (every thread
+// calls them; tmp: 32 shared ints).
+__device__ __forceinline__ int block_scan_max(int v, int* tmp) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v = max(v, n);
+  }
+  if (lane == 31) tmp[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    int t = lane < nw ? tmp[lane] : INT_MIN;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t = max(t, n);
+    }
+    if (lane < nw) tmp[lane] = t;
+  }
+  __syncthreads();
+  if (warp > 0) v = max(v, tmp[warp - 1]);
+  __syncthreads();
+  return v;
+}
+__device__ __forceinline__ int block_scan_sum(int v, int* tmp) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) tmp[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    int t = lane < nw ? tmp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += n;
+    }
+    if (lane < nw) tmp[lane] = t;
+  }
+  __syncthreads();
+  if (warp > 0) v += tmp[warp - 1];
+  __syncthreads();
+  return v;
+}
+
+// SHARE: also group sequences that share leading blocks (one thread per
+// sequence: launched with kPlanMaxThreads threads, num_seqs <= kShareMaxSeqs).
+template <bool SHARE>
 __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) {
   pdl_launch_dependents();
   __shared__ long long s_sum[32];
@@ -75,7 +133,18 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
   __shared__ int s_fill[kKeys + 1];
   __shared__ PieceRule s_rule;
   __shared__ int s_nsplit_seqs;
-  extern __shared__ int s_len[];   // [num_seqs]
+  __shared__ int s_ngroups, s_ngpairs;
+  __shared__ int s_scan[32];
+  extern __shared__ int s_len[];   // [num_seqs]; with shared prefixes 4 more arrays follow
+  // shared prefixes: per sequence, the leading full blocks it shares with the
+  // one before it, then (at a group's first member) the group's common whole
+  // pieces; the group's first member (or -1); at the first member, the common
+  // prefix in tokens, then the member count; at the first member, the group's
+  // first slot in the group list
+  int* s_aux = s_len + p.num_seqs;
+  int* s_lead = s_aux + p.num_seqs;
+  int* s_pre = s_lead + p.num_seqs;
+  int* s_goff = s_pre + p.num_seqs;
 
   WsHeader* hdr = reinterpret_cast<WsHeader*>(p.ws);
   WorkPair* pairs = reinterpret_cast<WorkPair*>(p.ws + p.pairs_off);
@@ -83,7 +152,11 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
   int32_t* cnt = reinterpret_cast<int32_t*>(p.ws + p.cnt_off);
   int32_t* split_list = reinterpret_cast<int32_t*>(p.ws + p.split_off);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid == 0) s_nsplit_seqs = 0;
+  if (tid == 0) {
+    s_nsplit_seqs = 0;
+    s_ngroups = 0;
+    s_ngpairs = 0;
+  }
   const int nthreads = blockDim.x, nwarps = nthreads >> 5;
   const int64_t cap = static_cast<int64_t>(p.bt_stride) * p.block_size;
   auto valid_len = [&](int L) { return !(L < 0 || L > p.max_context_len || L > cap); };
@@ -112,6 +185,80 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
     s_bad[warp] = bad;
   }
   __syncthreads();
+  if constexpr (SHARE) {
+    // 1b. Shared prefixes ("Paged Attention: Virtual Memory for the KV
+    // Cache", "Sharing comes almost for free": sequences forked from one
+    // another point at the same physical blocks). Each sequence counts the
+    // leading full blocks its table has in common with the previous
+    // sequence's: a thread per sequence checks the first entry, then a warp
+    // per sequence whose first entries match compares the rest, 256 entries
+    // per round (8 loads in flight per lane).
+    const int i = tid;   // num_seqs <= threads
+    int La = 0, nb = 0;
+    if (i < p.num_seqs) {
+      La = s_len[i];
+      const int Lb = i > 0 ? s_len[i - 1] : 0;
+      nb = i > 0 && valid_len(La) && valid_len(Lb) ? min(La, Lb) / p.block_size : 0;
+      if (nb > 0) {
+        const int32_t* ra = p.block_tables + static_cast<size_t>(i) * p.bt_stride;
+        if (ra[0] != ra[-p.bt_stride]) nb = 0;
+      }
+      s_aux[i] = nb;   // an upper bound, exact below
+      s_lead[i] = -1;
+    }
+    __syncthreads();
+    for (int w = warp; w < p.num_seqs; w += nwarps) {
+      const int n = s_aux[w];
+      if (n <= 1) continue;
+      const int32_t* ra = p.block_tables + static_cast<size_t>(w) * p.bt_stride;
+      const int32_t* rb = ra - p.bt_stride;
+      int common = n;
+      for (int j0 = 0; j0 < n; j0 += 256) {
+        bool diff[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int j = j0 + 32 * q + lane;
+          diff[q] = j < n && ra[j] != rb[j];
+        }
+        unsigned first = 0xffffffffu;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const unsigned m = __ballot_sync(0xffffffffu, diff[q]);
+          if (m != 0u && first == 0xffffffffu) first = 32 * q + __ffs(m) - 1;
+        }
+        if (first != 0xffffffffu) {
+          common = j0 + static_cast<int>(first);
+          break;
+        }
+      }
+      if (lane == 0) s_aux[w] = common;
+    }
+    __syncthreads();
+    // Groups: runs of consecutive sequences each sharing >= kShareMinTokens
+    // with the one before, cut into groups of at most share_members members
+    // (their query rows fill one 16-row tile). A run starts at the last
+    // sequence that does not share with its predecessor (a max scan); a
+    // member whose offset in its run is a multiple of share_members leads a
+    // group if the next sequence is in the run too. The group's common
+    // prefix is the smallest count among its members after the first.
+    auto shares = [&](int j) { return s_aux[j] * p.block_size >= kShareMinTokens; };
+    const bool in = i < p.num_seqs;
+    const int run_start = block_scan_max(in && !(i > 0 && shares(i)) ? i : -1, s_scan);
+    const bool leader = in && (i - run_start) % p.share_members == 0 && i + 1 < p.num_seqs &&
+                        shares(i + 1);
+    if (leader) {
+      int m = i + 1, P = 1 << 30;
+      for (; m < p.num_seqs && m - i < p.share_members && shares(m); ++m) P = min(P, s_aux[m]);
+      s_pre[i] = P * p.block_size;
+      s_goff[i] = m - i;   // members, until the offsets are known
+    }
+    const int any = __syncthreads_or(leader);
+    if (leader) {
+      for (int m = i; m < i + s_goff[i]; ++m) s_lead[m] = i;
+    }
+    if (tid == 0) s_ngroups = any;
+    __syncthreads();
+  }
   if (warp == 0) {
     long long t = lane < nwarps ? s_sum[lane] : 0;
     int b = lane < nwarps ? s_bad[lane] : 0;
@@ -139,6 +286,12 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
         long long want = (base + kAutoSplitQuantum - 1) / kAutoSplitQuantum * kAutoSplitQuantum;
         if (want < p.min_split) want = p.min_split;
         if (want > (1 << 30)) want = 1 << 30;
+        // groups share whole pieces: keep them short enough that a prefix
+        // holds several
+        if (s_ngroups > 0) {
+          const long long cap_s = p.min_split > kShareSplit ? p.min_split : kShareSplit;
+          if (want > cap_s) want = cap_s;
+        }
         S = static_cast<int>(want);
       }
       s_rule.S = S;
@@ -192,14 +345,56 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
   }
   const PieceRule rule = s_rule;
 
+  if constexpr (SHARE) {
+    // 2b. A group's common whole pieces: the S-token pieces inside its
+    // common prefix, short of every member's last token (so each member
+    // keeps a piece of its own, which completes and merges its result). The
+    // group list gets them once, with the members' query rows; each member's
+    // own part (the rest of its sequence) is cut by the usual rule, with that
+    // many pieces fewer of room. Group list offsets: a sum scan.
+    const int i = tid;
+    const bool leader = i < p.num_seqs && s_lead[i] == i;
+    int kg = 0, members = 0;
+    if (leader) {
+      members = s_goff[i];
+      kg = s_pre[i] / S;
+      for (int m = i; m < i + members; ++m) kg = min(kg, (s_len[m] - 1) / S);
+    }
+    const int incl = block_scan_sum(kg, s_scan);
+    if (leader) {
+      s_aux[i] = kg;
+      s_pre[i] = members;
+      s_goff[i] = incl - kg;
+    }
+    if (tid == nthreads - 1) {
+      s_ngpairs = incl;
+      hdr->num_group_items = incl * p.num_kv_heads;
+      hdr->group_work_counter = p.group_ctas;
+    }
+    __syncthreads();
+  }
+  // whole pieces of sequence i that a group lists for it
+  auto shared_pieces = [&](int i) { return SHARE && s_lead[i] >= 0 ? s_aux[s_lead[i]] : 0; };
+  auto s_lead_is = [&](int i) { return SHARE && s_lead[i] == i; };
+  WorkPair* gpairs = reinterpret_cast<WorkPair*>(p.ws + p.gpairs_off);
+  // pieces of sequence i (valid, L > 0): the kg whole pieces its group lists,
+  // then its own part [kg*S, L) as nA whole pieces of S tokens and k pieces
+  // of sb tokens (the last one shorter); n = kg + nA + k <= ms
+  auto pieces_of = [&](int i, int L, int& kg, int& nA, int& sb, int& k) {
+    kg = shared_pieces(i);
+    PieceRule r = rule;
+    r.ms -= kg;
+    seq_pieces(L - kg * S, r, nA, sb, k);
+  };
+
   // 3. pieces per sequence (a thread per sequence): split counts, zeroed merge
   // counters and the list of split sequences, and the length histogram (a
   // sequence's pieces form at most three runs of equal length)
   for (int i = tid; i < p.num_seqs; i += nthreads) {
     const int L = s_len[i];
-    int nA = 0, sb = 0, k = 0;
-    if (valid_len(L) && L > 0) seq_pieces(L, rule, nA, sb, k);
-    const int n = nA + k;
+    int kg = 0, nA = 0, sb = 0, k = 0;
+    if (valid_len(L) && L > 0) pieces_of(i, L, kg, nA, sb, k);
+    const int n = kg + nA + k;
     nsplit[i] = n;
     if (n > 1) {
       for (int h = 0; h < p.num_kv_heads; ++h) cnt[static_cast<size_t>(i) * p.num_kv_heads + h] = 0;
@@ -207,7 +402,7 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
     }
     if (nA > 0) atomicAdd(&s_hist[piece_key(S)], nA);
     if (k > 1) atomicAdd(&s_hist[piece_key(sb)], k - 1);
-    if (k > 0) atomicAdd(&s_hist[piece_key(L - nA * S - (k - 1) * sb)], 1);
+    if (k > 0) atomicAdd(&s_hist[piece_key(L - kg * S - nA * S - (k - 1) * sb)], 1);
   }
   __syncthreads();
   // 4. longest first: bucket bases in descending length order (warp 0 scans
@@ -227,6 +422,7 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
     if (lane == 31) {
       hdr->num_pairs = inc;
       hdr->num_items = inc * p.num_kv_heads;
+      if (!SHARE) hdr->num_group_items = 0;
       // every item stream takes item (its index) first without claiming it
       // (no atomic on the start-up path); claims continue from here
       hdr->work_counter = p.num_ctas;
@@ -242,16 +438,16 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
   for (int i = tid; i < p.num_seqs; i += nthreads) {
     const int L = s_len[i];
     if (!valid_len(L) || L == 0) continue;
-    int nA, sb, k;
-    seq_pieces(L, rule, nA, sb, k);
-    const int n = nA + k;
+    int kg, nA, sb, k;
+    pieces_of(i, L, kg, nA, sb, k);
+    const int n = kg + nA + k, base = kg * S;
     WorkPair w;
     w.seq = i;
     if (nA > 0) {
       const int pos = atomicAdd(&s_fill[piece_key(S)], nA);
       for (int j = 0; j < nA; ++j) {
-        w.split_n = j | (n << 16);
-        w.t_begin = j * S;
+        w.split_n = (kg + j) | (n << 16);
+        w.t_begin = base + j * S;
         w.t_end = w.t_begin + S;
         pairs[pos + j] = w;
       }
@@ -259,17 +455,29 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
     if (k > 1) {
       const int pos = atomicAdd(&s_fill[piece_key(sb)], k - 1);
       for (int q = 0; q < k - 1; ++q) {
-        w.split_n = (nA + q) | (n << 16);
-        w.t_begin = nA * S + q * sb;
+        w.split_n = (kg + nA + q) | (n << 16);
+        w.t_begin = base + nA * S + q * sb;
         w.t_end = w.t_begin + sb;
         pairs[pos + q] = w;
       }
     }
     if (k > 0) {
       w.split_n = (n - 1) | (n << 16);
-      w.t_begin = nA * S + (k - 1) * sb;
+      w.t_begin = base + nA * S + (k - 1) * sb;
       w.t_end = L;
       pairs[atomicAdd(&s_fill[piece_key(L - w.t_begin)], 1)] = w;
+    }
+    if (s_lead_is(i)) {
+      // the group list: the group's common whole pieces, each with the
+      // members' count in place of the split count
+      WorkPair g;
+      g.seq = i;
+      for (int j = 0; j < kg; ++j) {
+        g.split_n = j | (s_pre[i] << 16);
+        g.t_begin = j * S;
+        g.t_end = g.t_begin + S;
+        gpairs[s_goff[i] + j] = g;
+      }
     }
   }
   // complete only after the kernel before this one (the KV write) has
@@ -290,13 +498,17 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
 }  // namespace
 
 cudaError_t launch_plan(const PlanParams& p, cudaStream_t stream) {
-  // a thread per sequence
+  // a thread per sequence (all threads for the table comparison of shared
+  // prefixes)
   int threads = (p.num_seqs + 31) / 32 * 32;
   threads = threads < 128 ? 128 : (threads > kPlanMaxThreads ? kPlanMaxThreads : threads);
-  const size_t smem = static_cast<size_t>(p.num_seqs) * sizeof(int);
+  if (p.share_prefixes) threads = kPlanMaxThreads;
+  auto kern = p.share_prefixes ? plan_kernel<true> : plan_kernel<false>;
+  // the lengths, and with shared prefixes four more arrays per sequence
+  const size_t smem = static_cast<size_t>(p.num_seqs) * sizeof(int) * (p.share_prefixes ? 5 : 1);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
@@ -312,10 +524,10 @@ cudaError_t launch_plan(const PlanParams& p, cudaStream_t stream) {
   cfg.numAttrs = 1;
   // the largest shared-memory carveout, as the decode kernels use: an SM that
   // ran this kernel need not be reconfigured before it takes a decode CTA
-  cudaError_t e = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                                        cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
-  return cudaLaunchKernelEx(&cfg, plan_kernel, p);
+  return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
 }  // namespace pa

@@ -2,7 +2,7 @@
 // code). All offsets are multiples of 256 bytes from the workspace start.
 //
 //   [header 256 B][work pairs][splits per sequence][split sequences]
-//   [merge counters][partial (m, l)][partial o]
+//   [merge counters][group list][partial (m, l)][partial o]
 //
 // The header holds the device status word (first 4 bytes), the work counter
 // the persistent decode kernels claim items from, and the plan the planning
@@ -26,7 +26,9 @@ struct WsHeader {
   int32_t max_splits;    // split capacity per sequence in this workspace
   int32_t num_split_seqs;  // sequences cut into more than one piece
   int32_t merge_counter;   // next unclaimed merge task (tensor-core kernel)
-  int32_t reserved[56];
+  int32_t num_group_items;     // group list entries x KV heads (shared prefixes)
+  int32_t group_work_counter;  // next unclaimed group item
+  int32_t reserved[54];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
@@ -54,7 +56,7 @@ inline int32_t auto_min_split(int32_t max_ctx) {
 
 struct WsLayout {
   int32_t max_splits;
-  size_t pairs_off, nsplit_off, split_off, cnt_off, ml_off, o_off, total;
+  size_t pairs_off, nsplit_off, split_off, cnt_off, gpairs_off, ml_off, o_off, total;
 };
 
 inline WsLayout ws_layout(int32_t num_seqs, int32_t num_q_heads,
@@ -77,6 +79,8 @@ inline WsLayout ws_layout(int32_t num_seqs, int32_t num_q_heads,
   off += align256(B * 4);
   w.cnt_off = off;   // merge counters [sequence][KV head] (KV heads <= query heads)
   off += align256(B * H * 4);
+  w.gpairs_off = off;   // the group list: at most one entry per (sequence, piece)
+  off += align256(B * ms * 16);
   w.ml_off = off;
   off += align256(B * H * ms * 8);
   w.o_off = off;

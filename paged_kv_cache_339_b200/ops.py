@@ -30,7 +30,8 @@ class PaKvCache(ctypes.Structure):
 
 
 class PaDecodeOptions(ctypes.Structure):
-    _fields_ = [("split_tokens", ctypes.c_int32), ("path", ctypes.c_int32)]
+    _fields_ = [("split_tokens", ctypes.c_int32), ("path", ctypes.c_int32),
+                ("share_prefixes", ctypes.c_int32)]
 
 
 class PagedAttnError(RuntimeError):
@@ -198,7 +199,8 @@ def decode_workspace(num_seqs, num_q_heads, head_dim, max_context_len, block_siz
 
 
 def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
-              workspace, split_tokens=0, path=PA_PATH_AUTO, stream=None) -> torch.Tensor:
+              workspace, split_tokens=0, path=PA_PATH_AUTO, stream=None,
+              share_prefixes=False) -> torch.Tensor:
     """out[i, h] = softmax(scale * q[i, h] . K_i^T) . V_i over context_lens[i]
     tokens reached through block_tables[i]; out is fp32 [B, Hq, D]."""
     desc = kv_cache_desc(k_cache, v_cache)
@@ -209,7 +211,7 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_
         raise ValueError("shape mismatch between q, caches and block_tables")
     if context_lens.shape != (B,):
         raise ValueError("context_lens must be [num_seqs]")
-    opts = PaDecodeOptions(int(split_tokens), int(path))
+    opts = PaDecodeOptions(int(split_tokens), int(path), int(bool(share_prefixes)))
     st = _load().pa_decode(
         ctypes.byref(desc), _dev_tensor(out, "out", torch.float32),
         _dev_tensor(q, "q", k_cache.dtype), _dev_tensor(block_tables, "block_tables", torch.int32),
@@ -221,7 +223,8 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_
 
 
 def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len,
-                      scale, split_tokens=0, path=PA_PATH_AUTO, stream=None) -> torch.Tensor:
+                      scale, split_tokens=0, path=PA_PATH_AUTO, stream=None,
+                      share_prefixes=False) -> torch.Tensor:
     """pa_decode with the library's fixed 32 MiB device scratch instead of a
     workspace, for callers that cannot allocate device memory (see
     include/pa.h). Calls must not overlap on the GPU."""
@@ -233,7 +236,7 @@ def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, max_
         raise ValueError("shape mismatch between q, caches and block_tables")
     if context_lens.shape != (B,):
         raise ValueError("context_lens must be [num_seqs]")
-    opts = PaDecodeOptions(int(split_tokens), int(path))
+    opts = PaDecodeOptions(int(split_tokens), int(path), int(bool(share_prefixes)))
     st = _load().pa_decode_noalloc(
         ctypes.byref(desc), _dev_tensor(out, "out", torch.float32),
         _dev_tensor(q, "q", k_cache.dtype), _dev_tensor(block_tables, "block_tables", torch.int32),

@@ -53,9 +53,9 @@ def _cache(ops, **kw):
 
 def _decode(lib, ops, cache, **kw):
     a = dict(out=0x30000, q=0x40000, bt=0x50000, bt_stride=4, lens=0x60000, B=2, Hq=4,
-             max_ctx=64, scale=0.1, split=0, path=0, ws=0x70000, ws_bytes=1 << 30)
+             max_ctx=64, scale=0.1, split=0, path=0, share=0, ws=0x70000, ws_bytes=1 << 30)
     a.update(kw)
-    opts = ops.PaDecodeOptions(a["split"], a["path"])
+    opts = ops.PaDecodeOptions(a["split"], a["path"], a["share"])
     return lib.pa_decode(ctypes.byref(cache), a["out"], a["q"], a["bt"], a["bt_stride"],
                          a["lens"], a["B"], a["Hq"], a["max_ctx"], a["scale"],
                          ctypes.byref(opts), a["ws"], a["ws_bytes"], None)
@@ -78,6 +78,7 @@ def test_host_side_rejections(lib):
     assert _decode(lib, ops, c, max_ctx=65) == ops.PA_ERR_INVALID_ARG      # > 4 * 16
     assert _decode(lib, ops, c, scale=float("nan")) == ops.PA_ERR_INVALID_ARG
     assert _decode(lib, ops, c, path=5) == ops.PA_ERR_INVALID_ARG
+    assert _decode(lib, ops, c, share=2) == ops.PA_ERR_INVALID_ARG
     assert _decode(lib, ops, c, out=0x30004) == ops.PA_ERR_MISALIGNED
     assert _decode(lib, ops, c, ws_bytes=100) == ops.PA_ERR_WORKSPACE_TOO_SMALL
     assert _decode(lib, ops, c, B=0) == ops.PA_OK                          # nothing to do
@@ -106,16 +107,16 @@ def test_host_side_rejections(lib):
 
 def test_workspace_size_layout(lib):
     """Header 256 B, then pairs, splits per sequence, the list of split
-    sequences, merge counters, partial (m, l) and partial o, each rounded up to
-    256 B; split capacity from the split rule."""
+    sequences, merge counters, the group list, partial (m, l) and partial o,
+    each rounded up to 256 B; split capacity from the split rule."""
     from paged_kv_cache_339_b200 import ops
 
     def expect(B, H, D, max_ctx, split):
         s = split if split > 0 else max(256, -(-(-(-max_ctx // 64)) // 128) * 128)
         ms = max(1, -(-max_ctx // s))
         r = lambda x: -(-x // 256) * 256
-        return (256 + r(B * ms * 16) + r(B * 4) + r(B * 4) + r(B * H * 4) + r(B * H * ms * 8)
-                + r(B * H * ms * D * 4))
+        return (256 + r(B * ms * 16) + r(B * 4) + r(B * 4) + r(B * H * 4) + r(B * ms * 16)
+                + r(B * H * ms * 8) + r(B * H * ms * D * 4))
 
     for args in ((64, 32, 128, 2048, 0), (256, 32, 128, 4096, 0), (8, 64, 128, 131072, 0),
                  (4, 1, 64, 33, 16), (3, 8, 128, 1000, 32)):
