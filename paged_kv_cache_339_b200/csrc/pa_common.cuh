@@ -262,7 +262,14 @@ struct __align__(16) WorkPair {
   int32_t t_end;    // one past the last token
 };
 __device__ __forceinline__ int item_split(int32_t split_n) { return split_n & 0xffff; }
-__device__ __forceinline__ int item_nsplit(int32_t split_n) { return split_n >> 16; }
+__device__ __forceinline__ int item_nsplit(int32_t split_n) { return (split_n >> 16) & 0x3fff; }
+// Set on a sequence's only piece of its own when all its other pieces are
+// shared-prefix group pieces, complete before the launch that takes it: that
+// piece folds their partial results into its own and writes the output rows.
+constexpr int32_t kFoldGroupPieces = 1 << 30;
+__device__ __forceinline__ bool item_folds(int32_t split_n) {
+  return (split_n & kFoldGroupPieces) != 0;
+}
 
 // Programmatic dependent launch: let the next kernel in the stream start its
 // prologue now / wait until the previous kernel has completed and its writes

@@ -472,13 +472,43 @@ __global__ void __launch_bounds__(SimtTraits<T, D, GPW>::NTHREADS, 2)
           }
         } else {
           const int nsp = item_nsplit(mt.split_raw);
-          const bool single = nsp == 1;
+          // the sequence's only own piece after its shared-prefix group
+          // pieces (complete before this launch) folds them in itself
+          const bool fold = item_folds(mt.split_raw);
+          const bool single = nsp == 1 || fold;   // this item writes the output rows
           const size_t row0 = static_cast<size_t>(mt.seq) * p.num_q_heads + mt.kvh * G;
           for (int idx = tid; idx < G * D; idx += Tr::NCW * 32) {
             const int h = idx / D, d = idx - (idx / D) * D;
             float M, L, O;
             combine(h, d, M, L, O);
             const size_t row = row0 + h;
+            if (fold) {
+              // (m, l, o) of pieces 0 .. split-1, 8 pieces' loads in flight
+              const size_t pr0 = row * p.max_splits;
+              for (int s0 = 0; s0 < split; s0 += 8) {
+                float2 e[8];
+                float v[8];
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                  const bool in = s0 + jj < split;
+                  e[jj] = in ? __ldcg(ml + pr0 + s0 + jj) : make_float2(-INFINITY, 0.f);
+                  v[jj] = in ? __ldcg(po + (pr0 + s0 + jj) * D + d) : 0.f;
+                }
+                float mb = M;
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) mb = fmaxf(mb, e[jj].x);
+                const float sc = exp2f(M - mb);
+                L *= sc;
+                O *= sc;
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                  const float w = exp2f(e[jj].x - mb);   // 0 for the padding entries
+                  L = fmaf(e[jj].y, w, L);
+                  O = fmaf(w, v[jj], O);
+                }
+                M = mb;
+              }
+            }
             if (single) {
               p.out[row * D + d] = O / L;
             } else {

@@ -816,9 +816,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[t]);
       const bool ok0 = tk0 < mt.valid, ok1 = tk0 + 64 < mt.valid;
-      // hardware 2^x (ex2.approx) where the registers allow it; the 16-head
-      // tile keeps exp2f, with which its registers fit without spilling
-      auto ex2 = [](float x) { return GT <= 8 ? exp2_approx(x) : exp2f(x); };
+      // hardware 2^x (ex2.approx)
+      auto ex2 = [](float x) { return exp2_approx(x); };
       float sa[GT], sb[GT];
 #pragma unroll
       for (int g = 0; g < GT; ++g) {

@@ -441,12 +441,14 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
     int kg, nA, sb, k;
     pieces_of(i, L, kg, nA, sb, k);
     const int n = kg + nA + k, base = kg * S;
+    // a member's only own piece folds the group pieces in itself
+    const int32_t fold = kg > 0 && nA + k == 1 ? kFoldGroupPieces : 0;
     WorkPair w;
     w.seq = i;
     if (nA > 0) {
       const int pos = atomicAdd(&s_fill[piece_key(S)], nA);
       for (int j = 0; j < nA; ++j) {
-        w.split_n = (kg + j) | (n << 16);
+        w.split_n = (kg + j) | (n << 16) | fold;
         w.t_begin = base + j * S;
         w.t_end = w.t_begin + S;
         pairs[pos + j] = w;
@@ -462,7 +464,7 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
       }
     }
     if (k > 0) {
-      w.split_n = (n - 1) | (n << 16);
+      w.split_n = (n - 1) | (n << 16) | fold;
       w.t_begin = base + nA * S + (k - 1) * sb;
       w.t_end = L;
       pairs[atomicAdd(&s_fill[piece_key(L - w.t_begin)], 1)] = w;
