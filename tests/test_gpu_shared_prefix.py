@@ -150,3 +150,70 @@ def test_full_size_prefix_cow_step():
             ref = sampled_reference(b, int(seq), int(h))
             got = shared[int(seq), int(h)].cpu().numpy().astype(np.float64)
             assert np.max(np.abs(got - ref)) <= 2e-3
+
+
+def test_empty_and_invalid_sequences_inside_a_run():
+    """An empty sequence and one whose length exceeds max_context_len break
+    the run they sit in: the others still match the oracle, the empty row is
+    zero, the invalid one is zero and flagged, and groups still form."""
+    b = shared_batch([(1024, [10, 20, 30, 40, 50, 60])])
+    lens = b.context_lens.clone()
+    lens[2] = 0
+    b.context_lens = lens
+    B, Hq, D = b.q.shape
+    bc = b.to("cpu")
+    ref = ORACLE.decode(f64(bc.q), pool_f64(bc.k_cache), pool_f64(bc.v_cache),
+                        bc.block_tables.numpy(), bc.context_lens.numpy(),
+                        float(np.float32(bc.scale)))
+    out, groups = decode(b, True)
+    assert groups > 0
+    assert max_abs_err(out, ref) <= TOL[b.dtype]
+    assert torch.count_nonzero(out[2]) == 0
+    # now sequence 4 claims more tokens than max_context_len allows
+    max_ctx = int(lens.max().item())
+    lens[4] = max_ctx + 1
+    ws = ops.decode_workspace(B, Hq, D, max_ctx + 16, b.block_size)
+    out2 = torch.full((B, Hq, D), float("nan"), device="cuda")
+    ops.pa_decode(out2, b.q, b.k_cache, b.v_cache, b.block_tables, lens, max_ctx, b.scale, ws,
+                  path=ops.PA_PATH_SIMT, share_prefixes=True)
+    torch.cuda.synchronize()
+    assert ops.pa_decode_status(ws) == ops.PA_ERR_INVALID_ARG
+    assert torch.count_nonzero(out2[4]) == 0
+    keep = [i for i in range(B) if i not in (2, 4)]
+    assert max_abs_err(out2[keep], ref[keep]) <= TOL[b.dtype]
+
+
+def test_largest_batch_with_groups():
+    """1024 sequences (the most pa_decode groups), runs of 5 behind 256- to
+    512-token prefixes: sampled rows against the oracle, all rows against the
+    per-sequence path."""
+    rng = np.random.default_rng(9)
+    runs = [(int(rng.choice([256, 384, 512])), [int(x) for x in rng.integers(1, 200, 5)])
+            for _ in range(204)] + [(256, [3, 30, 90, 199])]
+    b = shared_batch(runs, dtype=torch.bfloat16, Hq=8, Hkv=8)
+    assert b.q.shape[0] == 1024
+    shared, groups = decode(b, True, path=ops.PA_PATH_AUTO)
+    private, _ = decode(b, False, path=ops.PA_PATH_AUTO)
+    assert groups > 0
+    assert float((shared - private).abs().max()) <= 1e-4
+    for seq in rng.choice(1024, 8, replace=False):
+        h = int(rng.integers(0, 8))
+        ref = sampled_reference(b, int(seq), h)
+        got = shared[int(seq), h].cpu().numpy().astype(np.float64)
+        assert np.max(np.abs(got - ref)) <= 2e-3
+
+
+def test_no_alloc_entry_point_shares_too():
+    """pa_decode_noalloc takes the option through its fixed scratch."""
+    b = shared_batch([(1024, [5, 17, 300, 64, 1, 700])])
+    B, Hq, D = b.q.shape
+    bc = b.to("cpu")
+    ref = ORACLE.decode(f64(bc.q), pool_f64(bc.k_cache), pool_f64(bc.v_cache),
+                        bc.block_tables.numpy(), bc.context_lens.numpy(),
+                        float(np.float32(bc.scale)))
+    out = torch.full((B, Hq, D), float("nan"), device="cuda")
+    ops.pa_decode_noalloc(out, b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens,
+                          b.max_context_len, b.scale, path=ops.PA_PATH_SIMT, share_prefixes=True)
+    torch.cuda.synchronize()
+    assert ops.pa_decode_noalloc_status() == ops.PA_OK
+    assert max_abs_err(out, ref) <= TOL[b.dtype]
