@@ -280,6 +280,18 @@ pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
 
+  // At block size 8 the tensor-core kernel reads two KV heads' pages with one
+  // copy (its items, and the plan's, are then pairs of heads: one head of 2G
+  // query heads); not with shared prefixes, whose launches count real heads.
+  // Pairs halve the (sequence, head) units the plan deals out, so only where
+  // at least two pairs per item stream remain: with fewer, the coarser items
+  // and the extra splits cost more at the end of the call than the saved
+  // copies gain.
+  const int64_t pair_units = static_cast<int64_t>(num_seqs) * (cache->num_kv_heads / 2);
+  const bool pair = use_tc && !ch.share &&
+                    tc_pair_supported(cache->block_size, cache->num_kv_heads, group) &&
+                    pair_units >= 2 * (2 * static_cast<int64_t>(ctas));
+
   PlanParams pp;
   pp.context_lens = context_lens;
   pp.out = out;
@@ -291,6 +303,7 @@ pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
   pp.num_seqs = num_seqs;
   pp.num_q_heads = num_q_heads;
   pp.num_kv_heads = cache->num_kv_heads;
+  pp.pair_heads = pair ? 1 : 0;
   pp.head_dim = cache->head_dim;
   pp.bt_stride = bt_stride;
   pp.block_size = cache->block_size;
@@ -340,6 +353,7 @@ pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
   dp.scale_log2 = scale * 1.4426950408889634f;
   dp.dtype = cache->dtype;
   dp.gpairs_off = lay.gpairs_off;
+  dp.pair_heads = 0;
   if (ch.share) {
     // the groups' common pieces first (each member's piece is counted there),
     // then every sequence's own pieces
@@ -348,6 +362,7 @@ pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
     if (e != cudaSuccess) return cuda_fail(e);
   }
   dp.group_mode = 0;
+  dp.pair_heads = pair ? 1 : 0;
   e = use_tc ? launch_decode_tc(dp, ctas, s) : launch_decode_simt(dp, ctas, s);
   if (e != cudaSuccess) return cuda_fail(e);
 

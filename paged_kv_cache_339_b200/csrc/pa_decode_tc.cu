@@ -39,6 +39,17 @@
 //               and output column d = r for the correction O = alpha O + O_c;
 //               a split item writes its partial result to the workspace, and
 //               the last piece of a (sequence, KV head) to finish merges them.
+// Paired KV heads (block size 8, 4 query heads per KV head): the pool stores
+// a block's KV heads one after the other, so the pages of KV heads 2j and
+// 2j + 1 of a block are one contiguous 4 KiB run. The kernel then treats the
+// pair as one virtual KV head of 8 query heads whose pages hold 2 x 8
+// virtual tokens (head 2j's 8 tokens, then head 2j + 1's), loaded with one
+// box per block instead of one per (block, head): a 128-token ring position
+// holds 64 tokens of both heads. A softmax thread's token belongs to one of
+// the two heads, so it keeps the scores, probabilities and sums of that
+// head's 4 query heads only (the others' probabilities are zero). Halving
+// the copies matters at block size 8, where the copy engine's request rate,
+// not HBM, bounds 2 KiB boxes.
 // No load uses cluster multicast; every wait is bounded (see pa_common.cuh).
 #include <cudaTypedefs.h>
 
@@ -242,7 +253,8 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // GRP: the launch over the group list of shared prefixes (group items only).
-template <typename T, int GT, bool GRP>
+// PAIR: paired KV heads (items, query rows and counts per virtual KV head).
+template <typename T, int GT, bool GRP, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v,
@@ -328,8 +340,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // the group list (shared prefixes) or the work list
   const int num_items = GRP ? hdr->num_group_items : hdr->num_items;
-  const int Hkv = p.num_kv_heads, BS = p.block_size;
+  // KV heads as the items see them (virtual ones when paired), query heads
+  // per item head, tokens a page box holds and tokens per ring position
+  const int Hkv = PAIR ? p.num_kv_heads / 2 : p.num_kv_heads, BS = p.block_size;
   const int G = p.num_q_heads / Hkv;
+  const int PB = PAIR ? 2 * BS : BS;
+  constexpr int CH = PAIR ? kChunk / 2 : kChunk;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -383,10 +399,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) {
             reinterpret_cast<uint4*>(&meta[bi])[0] = m0;
             reinterpret_cast<uint4*>(&meta[bi])[1] = m1;
-            // K: one box of 2*BS half-rows per page; Q': the group's query
+            // K: one box of 2*PB half-rows per page; Q': the group's query
             // rows, first halves then second halves (NS/2 rows each)
             mbar_arrive_expect_tx(&kfull[bi],
-                                  static_cast<uint32_t>(npg * BS * 256 + Ly::NS * 128));
+                                  static_cast<uint32_t>(npg * PB * 256 + Ly::NS * 128));
             if (GRP) {
               tma_load_3d(st + 2 * kTile, &tm_q, 0, q_y, q_row, &kfull[bi]);
               tma_load_3d(st + 2 * kTile + (Ly::NS / 2) * 128, &tm_q, 64, q_y, q_row, &kfull[bi]);
@@ -397,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           __syncwarp();
           if (lane < npg)
-            tma_load_2d_hint(st + lane * BS * 256, &tm_k, 0, (blk * Hkv + kvh) * BS * 2,
+            tma_load_2d_hint(st + lane * PB * 256, &tm_k, 0, (blk * Hkv + kvh) * PB * 2,
                              &kfull[bi], pol);
         } else {
           if (lane == 0) {
@@ -415,10 +431,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         if (data) {
-          if (lane == 0) mbar_arrive_expect_tx(&vfull[bi], static_cast<uint32_t>(npg * BS * 256));
+          if (lane == 0) mbar_arrive_expect_tx(&vfull[bi], static_cast<uint32_t>(npg * PB * 256));
           __syncwarp();
           if (lane < npg)
-            tma_load_2d_hint(st + kTile + lane * BS * 256, &tm_v, 0, (blk * Hkv + kvh) * BS * 2,
+            tma_load_2d_hint(st + kTile + lane * PB * 256, &tm_v, 0, (blk * Hkv + kvh) * PB * 2,
                              &vfull[bi], pol);
         } else {
           if (lane == 0) mbar_arrive(&vfull[bi]);
@@ -545,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       int valid = 0, npg = 0, blk = 0;
       if (kind == 0) {
-        valid = min(kChunk, cur.te - cur.cs);
+        valid = min(CH, cur.te - cur.cs);
         npg = (valid + BS - 1) / BS;
         const int p0 = cur.cs / BS;
         if (p0 + npg > cur.wbase + 64) {   // chunk runs past the window: next window
@@ -565,7 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // holds an unstarted item for long (it would lengthen the tail); the
         // scheduler runs far enough ahead of the copies to cover the claim,
         // work pair and table window loads
-        if (cur.nst != 0 || cur.te - cur.cs <= kChunk) prefetch_step(cur);
+        if (cur.nst != 0 || cur.te - cur.cs <= CH) prefetch_step(cur);
       }
       const int qd = c % kQd;
       if (!mbar_wait(&desc_empty[qd], ((c / kQd) & 1u) ^ 1u, abrt, status)) return false;
@@ -578,7 +594,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           m.split_raw = cur.split_n;
           m.t0 = cur.cs;
           m.valid = valid;
-          m.flags = (cur.cs == cur.tb ? kFirst : 0) | (cur.cs + kChunk >= cur.te ? kLast : 0) |
+          m.flags = (cur.cs == cur.tb ? kFirst : 0) | (cur.cs + CH >= cur.te ? kLast : 0) |
                     (solo_mark ? kSolo : 0);
           m.pad0 = m.pad1 = 0;
           d.meta = m;
@@ -590,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           d.npg = npg;
         }
         if (lane < kMaxPages) d.blk[lane] = lane < npg ? blk : 0;
-        cur.cs += kChunk;
+        cur.cs += CH;
         solo_mark = false;
       } else if (lane == 0) {
         d.meta.flags = kind == 1 ? kEnd : kStop;
@@ -671,7 +687,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&o_free[t], par ^ 1u, abrt, status)) break;
         if (!mbar_wait(&vfull[bi], fpar, abrt, status)) break;
         tc_fence_after();
-        const int nks = (mt.valid + 15) >> 4;
+        // 16-token steps; paired, the loaded blocks' 2 x BS virtual tokens each
+        const int nks = PAIR ? (mt.valid + BS - 1) / BS * (2 * BS) / 16 : (mt.valid + 15) >> 4;
         for (int ks = 0; ks < nks; ++ks) {
           // V^T for tokens 16ks..16ks+15: 4 KB of half-rows; M atoms (column
           // halves) sh * 128 B apart, 8-token groups v_sbo apart
@@ -702,6 +719,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int hh = (r / sh) & 1;
     const int tk0 = (r / (2 * sh)) * sh + r % sh;
     const int own_t = hh ? tk0 + 64 : tk0;   // the token whose P row / V row this thread writes
+    // Paired heads (block size 8, 2 G = GT): virtual token v is token
+    // (v / 16) 8 + v % 8 of the chunk, of the pair's KV head hd = (v / 8) & 1,
+    // whose query heads are the item's columns [hd GT/2, hd GT/2 + GT/2).
+    // tk0 and tk0 + 64 are of the same head and 32 tokens apart; the lanes of
+    // one head are one half of the warp, and a lane and lane ^ 8 hold the two
+    // halves of the same tokens.
+    const int rt0 = PAIR ? (tk0 / (2 * BS)) * BS + tk0 % BS : tk0;
+    const int rt1 = PAIR ? rt0 + 32 : tk0 + 64;
+    const int own_rt = hh ? rt1 : rt0;
+    const int hd = PAIR ? (tk0 / BS) & 1 : 0;
+    constexpr int GH = GT / 2;   // query heads of one KV head of a pair
     uint8_t* pdst_base = pbuf + t * Ly::PBUF + own_t * 16;
     // own token's V half-rows in the stage: (t / sh) * sh * 256 + (t % sh) * 128, + sh * 128
     const int vrow_off = kTile + (own_t / sh) * sh * 256 + (own_t % sh) * 128;
@@ -815,47 +843,86 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[t]);
-      const bool ok0 = tk0 < mt.valid, ok1 = tk0 + 64 < mt.valid;
+      const bool ok0 = rt0 < mt.valid, ok1 = rt1 < mt.valid;
       // hardware 2^x (ex2.approx)
       auto ex2 = [](float x) { return exp2_approx(x); };
-      float sa[GT], sb[GT];
+      // scores of the thread's query columns: all GT, or paired, the GH of
+      // its own KV head
+      constexpr int NC = PAIR ? GH : GT;
+      float sa[NC], sb[NC];
 #pragma unroll
-      for (int g = 0; g < GT; ++g) {
+      for (int g = 0; g < NC; ++g) {
         float a = hh ? sv0[Ly::NS / 2 + g] : sv0[g];
         float b = hh ? sv1[Ly::NS / 2 + g] : sv1[g];
+        if constexpr (PAIR) {
+          a = hd ? (hh ? sv0[Ly::NS / 2 + GH + g] : sv0[GH + g]) : a;
+          b = hd ? (hh ? sv1[Ly::NS / 2 + GH + g] : sv1[GH + g]) : b;
+        }
         a += __shfl_xor_sync(kFull, a, sh);
         b += __shfl_xor_sync(kFull, b, sh);
-        sa[g] = (ok0 && g < rows) ? a * sl2 : -INFINITY;
-        sb[g] = (ok1 && g < rows) ? b * sl2 : -INFINITY;
+        sa[g] = (ok0 && (PAIR || g < rows)) ? a * sl2 : -INFINITY;
+        sb[g] = (ok1 && (PAIR || g < rows)) ? b * sl2 : -INFINITY;
       }
-      // ---- chunk max per head across the group's 128 threads
+      // ---- chunk max per head across the group's 128 threads (paired: per
+      // half warp, over its 8 distinct lanes)
       float* rb = red_t + par * 64;
 #pragma unroll
-      for (int g = 0; g < GT; ++g) {
+      for (int g = 0; g < NC; ++g) {
         float mx = fmaxf(sa[g], sb[g]);
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
-        if (lane == 0) rb[wq * 16 + g] = mx;
+        for (int off = PAIR ? 4 : 16; off > 0; off >>= 1)
+          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
+        if constexpr (PAIR) {
+          if ((lane & 15) == 0) rb[wq * 16 + hd * GH + g] = mx;
+        } else {
+          if (lane == 0) rb[wq * 16 + g] = mx;
+        }
       }
       if (!group_sync(gbar, gphase, abrt, status)) break;
       float alpha[GT];
       uint32_t col[NPV];   // P^T row own_t: column g = hi(p_g), column GT + g = lo(p_g)
 #pragma unroll
       for (int i = 0; i < NPV; ++i) col[i] = 0;
+      if constexpr (PAIR) {
+        // every column's running max and rescale (the correction below takes
+        // all of them), then the own head's probabilities
 #pragma unroll
-      for (int g = 0; g < GT; ++g) {
-        const float cm = fmaxf(fmaxf(rb[g], rb[16 + g]), fmaxf(rb[32 + g], rb[48 + g]));
-        const float mn = fmaxf(m_run[g], cm);
-        // rows g >= rows never see a finite score; keep them inert (alpha 0, p 0)
-        alpha[g] = (mn == -INFINITY) ? 0.f : ex2(m_run[g] - mn);
-        const float own_s = hh ? sb[g] : sa[g];
-        const float pr = (mn == -INFINITY) ? 0.f : ex2(own_s - mn);
-        m_run[g] = mn;
-        l_thr[g] = fmaf(l_thr[g], alpha[g], pr);
-        uint16_t hi, lo;
-        split16<T>(pr, hi, lo);
-        col[g] = hi;
-        col[GT + g] = lo;
+        for (int g = 0; g < GT; ++g) {
+          const float cm = fmaxf(fmaxf(rb[g], rb[16 + g]), fmaxf(rb[32 + g], rb[48 + g]));
+          const float mn = fmaxf(m_run[g], cm);
+          alpha[g] = (mn == -INFINITY) ? 0.f : ex2(m_run[g] - mn);
+          m_run[g] = mn;
+        }
+#pragma unroll
+        for (int g = 0; g < GH; ++g) {
+          const float mn = hd ? m_run[GH + g] : m_run[g];
+          const float al = hd ? alpha[GH + g] : alpha[g];
+          const float own_s = hh ? sb[g] : sa[g];
+          const float pr = (mn == -INFINITY) ? 0.f : ex2(own_s - mn);
+          l_thr[g] = fmaf(l_thr[g], al, pr);
+          uint16_t hi, lo;
+          split16<T>(pr, hi, lo);
+          col[g] = hd ? 0u : hi;
+          col[GH + g] = hd ? hi : 0u;
+          col[GT + g] = hd ? 0u : lo;
+          col[GT + GH + g] = hd ? lo : 0u;
+        }
+      } else {
+#pragma unroll
+        for (int g = 0; g < GT; ++g) {
+          const float cm = fmaxf(fmaxf(rb[g], rb[16 + g]), fmaxf(rb[32 + g], rb[48 + g]));
+          const float mn = fmaxf(m_run[g], cm);
+          // rows g >= rows never see a finite score; keep them inert (alpha 0, p 0)
+          alpha[g] = (mn == -INFINITY) ? 0.f : ex2(m_run[g] - mn);
+          const float own_s = hh ? sb[g] : sa[g];
+          const float pr = (mn == -INFINITY) ? 0.f : ex2(own_s - mn);
+          m_run[g] = mn;
+          l_thr[g] = fmaf(l_thr[g], alpha[g], pr);
+          uint16_t hi, lo;
+          split16<T>(pr, hi, lo);
+          col[g] = hi;
+          col[GT + g] = lo;
+        }
       }
 #pragma unroll
       for (int ng = 0; ng < NPV / 8; ++ng)
@@ -865,9 +932,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                        col[8 * ng + 4] | (col[8 * ng + 5] << 16),
                        col[8 * ng + 6] | (col[8 * ng + 7] << 16));
       bool vok = true;
-      if (own_t >= mt.valid && own_t < ((mt.valid + 15) & ~15)) {
-        // past the chunk's valid tokens but inside the last 16-token step of
-        // the P.V MMA: make V finite (zero) once the stage's V has landed
+      // past the chunk's valid tokens but inside the last 16-token step of
+      // the P.V MMA (paired: inside the last loaded block): make V finite
+      // (zero) once the stage's V has landed
+      const int v_end = PAIR ? (mt.valid + BS - 1) / BS * BS : (mt.valid + 15) & ~15;
+      if (own_rt >= mt.valid && own_rt < v_end) {
         vok = mbar_wait(&vfull[bi], fpar, abrt, status);
         if (vok) {
           uint8_t* vrow = smem + static_cast<size_t>(stage) * kStage + vrow_off;
@@ -906,11 +975,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         // per-warp sum of l over the group's 128 tokens
         float* lr = lred_t + (Ly::DEFER_END ? lpar : 0u) * 64;
 #pragma unroll
-        for (int g = 0; g < GT; ++g) {
+        for (int g = 0; g < (PAIR ? GH : GT); ++g) {
           float lg = l_thr[g];
 #pragma unroll
-          for (int off = 16; off > 0; off >>= 1) lg += __shfl_xor_sync(kFull, lg, off);
-          if (lane == 0) lr[wq * 16 + g] = lg;
+          for (int off = PAIR ? 8 : 16; off > 0; off >>= 1) lg += __shfl_xor_sync(kFull, lg, off);
+          if constexpr (PAIR) {
+            if ((lane & 15) == 0) lr[wq * 16 + hd * GH + g] = lg;   // the own head's sums
+          } else {
+            if (lane == 0) lr[wq * 16 + g] = lg;
+          }
         }
         if constexpr (Ly::DEFER_END) {
 #pragma unroll
@@ -1070,17 +1143,19 @@ cudaError_t make_q_group_map(CUtensorMap* m, const void* q, int num_seqs, int nu
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <typename T, int GT, bool GRP = false>
+template <typename T, int GT, bool GRP = false, bool PAIR = false>
 cudaError_t launch_t(const DecodeParams& p, int num_ctas, cudaStream_t stream) {
   using Ly = TcLayout<GT>;
   const bool bf16 = std::is_same<T, __nv_bfloat16>::value;
   CUtensorMap mk, mv, mq;
   // pools as [half-rows, 64]: a (block, head) tile is 2 * block_size
   // consecutive 128-byte half-rows in its storage order, loaded as one box
+  // (two heads' tiles when paired)
   const uint64_t half_rows =
       static_cast<uint64_t>(p.num_blocks) * p.num_kv_heads * p.block_size * 2;
-  cudaError_t e = make_map(&mk, p.k_cache, 64, half_rows, 128, 2 * p.block_size, bf16);
-  if (e == cudaSuccess) e = make_map(&mv, p.v_cache, 64, half_rows, 128, 2 * p.block_size, bf16);
+  const uint32_t box_rows = (PAIR ? 4 : 2) * p.block_size;
+  cudaError_t e = make_map(&mk, p.k_cache, 64, half_rows, 128, box_rows, bf16);
+  if (e == cudaSuccess) e = make_map(&mv, p.v_cache, 64, half_rows, 128, box_rows, bf16);
   // q as [rows, 128]: one box per column half, NS/2 query rows; for the
   // group list, the rows of G heads of 16 / G consecutive sequences
   if (e == cudaSuccess) {
@@ -1094,7 +1169,7 @@ cudaError_t launch_t(const DecodeParams& p, int num_ctas, cudaStream_t stream) {
     }
   }
   if (e != cudaSuccess) return e;
-  auto kern = tc_decode_kernel<T, GT, GRP>;
+  auto kern = tc_decode_kernel<T, GT, GRP, PAIR>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(Ly::SMEM));
   if (e != cudaSuccess) return e;
@@ -1131,9 +1206,20 @@ cudaError_t launch_decode_tc_groups(const DecodeParams& p, int num_ctas, cudaStr
   return launch_t<__half, 16, true>(p, num_ctas, stream);
 }
 
+bool tc_pair_supported(int block_size, int num_kv_heads, int group) {
+  // a pair of KV heads of 4 query heads each fills the 8-row tile exactly
+  return block_size == 8 && num_kv_heads % 2 == 0 && group == 4;
+}
+
 cudaError_t launch_decode_tc(const DecodeParams& p, int num_ctas, cudaStream_t stream) {
   const int group = p.num_q_heads / p.num_kv_heads;
   if (!tc_supported(p.dtype, p.head_dim, group)) return cudaErrorInvalidValue;
+  if (p.pair_heads) {
+    // a pair is one KV head of 2G = 8 query heads
+    if (!tc_pair_supported(p.block_size, p.num_kv_heads, group)) return cudaErrorInvalidValue;
+    if (p.dtype == 2) return launch_t<__nv_bfloat16, 8, false, true>(p, num_ctas, stream);
+    return launch_t<__half, 8, false, true>(p, num_ctas, stream);
+  }
   if (p.dtype == 2) {
     if (group <= 4) return launch_t<__nv_bfloat16, 4>(p, num_ctas, stream);
     if (group <= 8) return launch_t<__nv_bfloat16, 8>(p, num_ctas, stream);

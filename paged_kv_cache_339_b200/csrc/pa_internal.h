@@ -23,12 +23,15 @@ struct PlanParams {
   int32_t num_ctas;       // item streams of the decode kernel (CTAs x streams per CTA)
   // shared prefixes (share_prefixes = 1): groups of consecutive sequences
   // whose tables start with the same blocks; their common whole pieces go to
-  // a list of their own (gpairs_off), taken by a CUDA-core launch of
-  // group_ctas CTAs that reads each shared tile once for up to share_members
+  // a list of their own (gpairs_off), taken by a launch of group_ctas item
+  // streams that reads each shared tile once for up to share_members
   // sequences
   const int32_t* block_tables;
   int32_t share_prefixes, share_members, group_ctas;
   size_t gpairs_off;
+  // 1: the decode kernel reads KV heads in pairs; items and merge counters
+  // are per pair, pieces are cut to the same work as for one head
+  int32_t pair_heads;
 };
 
 // Everything a decode main kernel needs; filled by the C-ABI shim.
@@ -46,9 +49,12 @@ struct DecodeParams {
   int32_t dtype;     // pa_dtype
   // 1: this launch takes the group list (shared prefixes): an item is a run
   // of whole pieces common to `members` consecutive sequences, its query rows
-  // those sequences' rows of the KV head (CUDA-core kernel only)
+  // those sequences' rows of the KV head
   int32_t group_mode;
   size_t gpairs_off;
+  // 1: the tensor-core kernel reads KV heads in pairs (its items, and the
+  // plan's, count num_kv_heads / 2 virtual heads of 2G = 8 query heads)
+  int32_t pair_heads;
 };
 
 // Largest batch whose shared prefixes pa_decode looks for.
@@ -75,6 +81,9 @@ cudaError_t launch_decode_tc(const DecodeParams& p, int num_ctas,
 // The tensor-core kernel over the group list: 16-row tiles of 16 / G
 // sequences x G heads (16-bit KV, head_dim 128, G a divisor of 16 up to 8).
 bool tc_group_supported(int dtype, int head_dim, int group);
+// The tensor-core kernel can read KV heads in pairs (block size 8, an even
+// number of KV heads, 4 query heads per KV head).
+bool tc_pair_supported(int block_size, int num_kv_heads, int group);
 cudaError_t launch_decode_tc_groups(const DecodeParams& p, int num_ctas,
                                     cudaStream_t stream);
 

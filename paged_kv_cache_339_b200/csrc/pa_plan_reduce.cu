@@ -47,6 +47,7 @@ struct PieceRule {
   int S;      // whole-piece size
   int cut;    // 1: the last `e` whole pieces (and the rest) are cut into ~sB-token pieces
   int e, sB, ms;
+  int q;      // tail pieces are multiples of q tokens (one ring position)
 };
 
 // Pieces of one sequence of L tokens: nA whole pieces of S tokens, then the
@@ -69,7 +70,7 @@ __device__ __forceinline__ void seq_pieces(int L, const PieceRule& r, int& nA, i
   }
   const int room = r.ms - nA;   // >= 1: nA * S < L <= ms * S
   const int need = (rest + room - 1) / room;
-  sb = need > r.sB ? (need + 127) / 128 * 128 : r.sB;
+  sb = need > r.sB ? (need + r.q - 1) / r.q * r.q : r.sB;
   k = (rest + sb - 1) / sb;
 }
 
@@ -303,22 +304,21 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
       if (sb > S) sb = S;
       s_rule.sB = static_cast<int>(sb);
       s_rule.ms = p.max_splits;
+      s_rule.q = kAutoSplitQuantum;
       hdr->status = b ? 1 /* PA_ERR_INVALID_ARG */ : 0;
-      hdr->split_tokens = S;
       hdr->max_splits = p.max_splits;
     }
   }
   __syncthreads();
-  const int S = s_rule.S;
 
   // 2. short work: the rests (pieces shorter than S) of at most two tail
   // pieces, in tokens of one KV head
   if (p.split_tokens <= 0) {
-    const int short_max = 2 * s_rule.sB;
+    const int S1 = s_rule.S, short_max = 2 * s_rule.sB;
     long long rem = 0;
     for (int i = tid; i < p.num_seqs; i += nthreads) {
       const int L = s_len[i];
-      const int rest = valid_len(L) ? L % S : 0;
+      const int rest = valid_len(L) ? L % S1 : 0;
       if (rest <= short_max) rem += rest;
     }
 #pragma unroll
@@ -336,14 +336,29 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
       const long long target =
           2LL * p.num_ctas * s_rule.sB / p.num_kv_heads;   // tokens of one KV head
       if (lane == 0 && r < target && p.num_seqs > 0) {
-        const long long per_seq = static_cast<long long>(p.num_seqs) * S;
+        const long long per_seq = static_cast<long long>(p.num_seqs) * S1;
         s_rule.cut = 1;
         s_rule.e = static_cast<int>(min((target - r + per_seq - 1) / per_seq, 1LL << 20));
+      }
+      // Paired KV heads: an item token is a token of two heads, so the same
+      // work takes half the tokens: whole and tail pieces of half the size
+      // (whole pieces no shorter than the workspace's bound on pieces per
+      // sequence allows), twice as many cut, in multiples of one 64-token
+      // ring position.
+      if (lane == 0 && p.pair_heads) {
+        s_rule.S = max(s_rule.S / 2, p.min_split);
+        s_rule.sB = min(max(s_rule.sB / 2, kAutoSplitQuantum / 2), s_rule.S);
+        s_rule.e = min(2 * s_rule.e, 1 << 20);
+        s_rule.q = kAutoSplitQuantum / 2;
       }
     }
     __syncthreads();
   }
   const PieceRule rule = s_rule;
+  const int S = rule.S;
+  if (tid == 0) hdr->split_tokens = S;
+  // KV heads per sequence as the items count them (pairs when paired)
+  const int Hi = p.pair_heads ? p.num_kv_heads / 2 : p.num_kv_heads;
 
   if constexpr (SHARE) {
     // 2b. A group's common whole pieces: the S-token pieces inside its
@@ -397,7 +412,7 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
     const int n = kg + nA + k;
     nsplit[i] = n;
     if (n > 1) {
-      for (int h = 0; h < p.num_kv_heads; ++h) cnt[static_cast<size_t>(i) * p.num_kv_heads + h] = 0;
+      for (int h = 0; h < Hi; ++h) cnt[static_cast<size_t>(i) * Hi + h] = 0;
       split_list[atomicAdd(&s_nsplit_seqs, 1)] = i;
     }
     if (nA > 0) atomicAdd(&s_hist[piece_key(S)], nA);
@@ -421,7 +436,7 @@ __global__ void __launch_bounds__(kPlanMaxThreads, 1) plan_kernel(PlanParams p) 
     if (k1 >= 1) s_fill[k1] = excl + h0;
     if (lane == 31) {
       hdr->num_pairs = inc;
-      hdr->num_items = inc * p.num_kv_heads;
+      hdr->num_items = inc * Hi;
       if (!SHARE) hdr->num_group_items = 0;
       // every item stream takes item (its index) first without claiming it
       // (no atomic on the start-up path); claims continue from here
