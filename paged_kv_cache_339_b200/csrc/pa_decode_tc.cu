@@ -1004,12 +1004,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // ---- merges of the split sequences, one output row per task. After its
     // last item the group claims tasks, waits until every piece of the row's
-    // (sequence, KV head) has been counted, and merges the row: thread r
-    // takes column r over all pieces, 16 pieces' loads in flight. Outside the
-    // main loop, so the merge neither stalls the ring nor adds to the loop's
-    // registers; the groups that finish first share the merges out. A group
-    // waits only on pieces that streams of running CTAs have claimed (every
-    // item was claimed before any stream saw END), so every wait ends.
+    // (sequence, KV head) has been counted, and merges the row: warp w of the
+    // group folds pieces w, w + 4, ... (lane l: columns 4l .. 4l + 3, 8
+    // pieces' loads in flight), then thread r combines the four warps'
+    // results for column r. Outside the main loop, so the merge neither
+    // stalls the ring nor adds to the loop's registers; the groups that
+    // finish first share the merges out. A group waits only on pieces that
+    // streams of running CTAs have claimed (every item was claimed before any
+    // stream saw END), so every wait ends.
     // (None in the launch over the group list: its pieces are merged by the
     // launch of the members' own pieces, which runs after it.)
     if (!GRP && !*abrt) {
@@ -1017,6 +1019,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int32_t* nsplit_of = reinterpret_cast<const int32_t*>(p.ws + p.nsplit_off);
       const int Hq = p.num_q_heads;
       const int ntasks = hdr->num_split_seqs * Hq;
+      // the group's P buffer (free once its stream has ended): per warp its
+      // running max and sum, then its 128 column sums
+      float* wml = reinterpret_cast<float*>(pbuf + t * Ly::PBUF);
+      float* wacc = wml + 8;
+      static_assert(Ly::PBUF >= (8 + 4 * kD) * 4, "merge scratch fits the P buffer");
       for (;;) {
         if (wq == 0 && lane == 0) {
           int k = atomicAdd(&hdr->merge_counter, 1);
@@ -1047,33 +1054,60 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nsp = nsplit_of[sq];
         const size_t row = static_cast<size_t>(sq) * Hq + (k - j * Hq);
         const float2* mr = ml + row * p.max_splits;
-        const float* pr = po + row * p.max_splits * kD + r;
-        float M = -INFINITY, L = 0.f, acc = 0.f;
-        for (int s0 = 0; s0 < nsp; s0 += 16) {
-          float2 e[16];
-          float v[16];
+        const float4* pr4 = reinterpret_cast<const float4*>(po + row * p.max_splits * kD) + lane;
+        float M = -INFINITY, L = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s0 = wq; s0 < nsp; s0 += 32) {
+          float2 e[8];
+          float4 v[8];
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            const bool in = s0 + jj < nsp;
-            e[jj] = in ? __ldcg(mr + s0 + jj) : make_float2(-INFINITY, 0.f);
-            v[jj] = in ? __ldcg(pr + static_cast<size_t>(s0 + jj) * kD) : 0.f;
+          for (int jj = 0; jj < 8; ++jj) {
+            const int sp = s0 + 4 * jj;
+            const bool in = sp < nsp;
+            e[jj] = in ? __ldcg(mr + sp) : make_float2(-INFINITY, 0.f);
+            v[jj] = in ? __ldcg(pr4 + static_cast<size_t>(sp) * (kD / 4))
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
           }
           float mb = M;
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) mb = fmaxf(mb, e[jj].x);
+          for (int jj = 0; jj < 8; ++jj) mb = fmaxf(mb, e[jj].x);
           const float sc = exp2f(M - mb);   // M = -inf on the first batch: 0
           L *= sc;
-          acc *= sc;
+          acc.x *= sc;
+          acc.y *= sc;
+          acc.z *= sc;
+          acc.w *= sc;
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
+          for (int jj = 0; jj < 8; ++jj) {
             const float w = exp2f(e[jj].x - mb);   // 0 for the padding entries
             L = fmaf(e[jj].y, w, L);
-            acc = fmaf(w, v[jj], acc);
+            acc.x = fmaf(w, v[jj].x, acc.x);
+            acc.y = fmaf(w, v[jj].y, acc.y);
+            acc.z = fmaf(w, v[jj].z, acc.z);
+            acc.w = fmaf(w, v[jj].w, acc.w);
           }
           M = mb;
         }
-        p.out[row * kD + r] = acc / L;
-        // the task slot is rewritten only after every thread has read it
+        // a warp without pieces (nsp < 4) leaves M = -inf, L = 0: weight 0
+        if (lane == 0) {
+          wml[2 * wq] = M;
+          wml[2 * wq + 1] = L;
+        }
+        reinterpret_cast<float4*>(wacc + wq * kD)[lane] = acc;
+        if (!group_sync(gbar, gphase, abrt, status)) break;
+        float Mt = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) Mt = fmaxf(Mt, wml[2 * w]);
+        float Lt = 0.f, at = 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const float sw = exp2f(wml[2 * w] - Mt);
+          Lt = fmaf(wml[2 * w + 1], sw, Lt);
+          at = fmaf(wacc[w * kD + r], sw, at);
+        }
+        p.out[row * kD + r] = at / Lt;
+        // the task slot and the scratch are rewritten only after every
+        // thread has read them
         if (!group_sync(gbar, gphase, abrt, status)) break;
       }
     }
