@@ -124,6 +124,28 @@ def test_matches_oracle_and_per_sequence_path(name, split):
     assert float((shared - private).abs().max()) <= 1e-4
 
 
+def test_block_size_8_many_sequences_against_paired_heads():
+    """Shared prefixes at block size 8 on the tensor cores (16-row group
+    tiles of 8-token pages), in a batch large enough that, with the option
+    off, pa_decode reads its KV heads in pairs: the two paths must agree, and
+    both match the oracle on sampled rows."""
+    rng = np.random.default_rng(13)
+    runs = [(int(rng.choice([256, 512, 768])), [int(x) for x in rng.integers(1, 400, 5)])
+            for _ in range(60)]
+    b = shared_batch(runs, dtype=torch.bfloat16, Hq=16, Hkv=4, BS=8)
+    streams = 2 * torch.cuda.get_device_properties(0).multi_processor_count
+    assert b.q.shape[0] * 2 >= 2 * streams   # enough KV-head pairs to pair them
+    shared, groups = decode(b, True, path=ops.PA_PATH_TCGEN05)
+    private, none = decode(b, False, path=ops.PA_PATH_TCGEN05)
+    assert groups > 0 and none == 0
+    assert float((shared - private).abs().max()) <= 1e-4
+    for seq in rng.choice(b.q.shape[0], 6, replace=False):
+        for h in rng.choice(16, 4, replace=False):
+            ref = sampled_reference(b, int(seq), int(h))
+            got = shared[int(seq), int(h)].cpu().numpy().astype(np.float64)
+            assert np.max(np.abs(got - ref)) <= 2e-3
+
+
 def test_off_where_it_does_not_apply():
     """No groups for 16 query heads per KV head (a group would have one
     sequence), for a batch of one sequence, or for prefixes under 256 tokens."""
