@@ -245,6 +245,35 @@ __device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t& phase, volat
   return ok;
 }
 
+// Max (MAX) or sum of NC values per lane over SPAN lanes (the warp, or a half
+// warp), all NC columns at once: each step hands half of the lane's columns
+// to its partner at the step's distance and keeps the other half, so the
+// first log2(NC) shuffles cover every column; the remaining steps reduce the
+// one column left. On return, lane l holds the result for column
+// (l % SPAN) / (SPAN / NC).
+template <int NC, int SPAN, bool MAX>
+__device__ __forceinline__ float xreduce(float (&v)[NC], int lane) {
+  static_assert(NC >= 1 && NC <= SPAN && (NC & (NC - 1)) == 0, "power-of-two columns");
+  int o = SPAN / 2;
+#pragma unroll
+  for (int w = NC; w > 1; w >>= 1, o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int j = 0; j < w / 2; ++j) {
+      const float send = up ? v[j] : v[j + w / 2];
+      const float keep = up ? v[j + w / 2] : v[j];
+      const float got = __shfl_xor_sync(kFull, send, o);
+      v[j] = MAX ? fmaxf(keep, got) : keep + got;
+    }
+  }
+#pragma unroll
+  for (; o > 0; o >>= 1) {
+    const float got = __shfl_xor_sync(kFull, v[0], o);
+    v[0] = MAX ? fmaxf(v[0], got) : v[0] + got;
+  }
+  return v[0];
+}
+
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   const unsigned long long t0 = global_timer_ns();
   while (!mbar_try_wait(bar, parity)) {
@@ -843,40 +872,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[t]);
-      const bool ok0 = rt0 < mt.valid, ok1 = rt1 < mt.valid;
       // hardware 2^x (ex2.approx)
       auto ex2 = [](float x) { return exp2_approx(x); };
-      // scores of the thread's query columns: all GT, or paired, the GH of
-      // its own KV head
+      // The thread's own token's scores (hh = 0: token tk0 of tile 0, hh = 1:
+      // token tk0 + 64 of tile 1) for its query columns: all GT, or paired,
+      // the GH of its own KV head. A half-row term is K_h[t] . Q_h[g]; the
+      // thread holds half hh of both tiles' tokens, so it keeps its own
+      // token's term and trades the other tile's term with its partner
+      // (lane ^ sh), which holds the other half.
       constexpr int NC = PAIR ? GH : GT;
-      float sa[NC], sb[NC];
+      constexpr int SPAN = PAIR ? 16 : 32;   // lanes of one KV head
+      const bool own_ok = own_rt < mt.valid;
+      float so[NC];
 #pragma unroll
       for (int g = 0; g < NC; ++g) {
-        float a = hh ? sv0[Ly::NS / 2 + g] : sv0[g];
-        float b = hh ? sv1[Ly::NS / 2 + g] : sv1[g];
+        float own = hh ? sv1[Ly::NS / 2 + g] : sv0[g];
+        float send = hh ? sv0[Ly::NS / 2 + g] : sv1[g];
         if constexpr (PAIR) {
-          a = hd ? (hh ? sv0[Ly::NS / 2 + GH + g] : sv0[GH + g]) : a;
-          b = hd ? (hh ? sv1[Ly::NS / 2 + GH + g] : sv1[GH + g]) : b;
+          own = hd ? (hh ? sv1[Ly::NS / 2 + GH + g] : sv0[GH + g]) : own;
+          send = hd ? (hh ? sv0[Ly::NS / 2 + GH + g] : sv1[GH + g]) : send;
         }
-        a += __shfl_xor_sync(kFull, a, sh);
-        b += __shfl_xor_sync(kFull, b, sh);
-        sa[g] = (ok0 && (PAIR || g < rows)) ? a * sl2 : -INFINITY;
-        sb[g] = (ok1 && (PAIR || g < rows)) ? b * sl2 : -INFINITY;
+        const float full = own + __shfl_xor_sync(kFull, send, sh);
+        so[g] = (own_ok && (PAIR || g < rows)) ? full * sl2 : -INFINITY;
       }
       // ---- chunk max per head across the group's 128 threads (paired: per
-      // half warp, over its 8 distinct lanes)
+      // half warp)
       float* rb = red_t + par * 64;
+      {
+        float v[NC];
 #pragma unroll
-      for (int g = 0; g < NC; ++g) {
-        float mx = fmaxf(sa[g], sb[g]);
-#pragma unroll
-        for (int off = PAIR ? 4 : 16; off > 0; off >>= 1)
-          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
-        if constexpr (PAIR) {
-          if ((lane & 15) == 0) rb[wq * 16 + hd * GH + g] = mx;
-        } else {
-          if (lane == 0) rb[wq * 16 + g] = mx;
-        }
+        for (int g = 0; g < NC; ++g) v[g] = so[g];
+        const float mx = xreduce<NC, SPAN, true>(v, lane);
+        const int cg = (lane & (SPAN - 1)) / (SPAN / NC);
+        if ((lane & (SPAN / NC - 1)) == 0) rb[wq * 16 + hd * GH + cg] = mx;
       }
       if (!group_sync(gbar, gphase, abrt, status)) break;
       float alpha[GT];
@@ -897,8 +925,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int g = 0; g < GH; ++g) {
           const float mn = hd ? m_run[GH + g] : m_run[g];
           const float al = hd ? alpha[GH + g] : alpha[g];
-          const float own_s = hh ? sb[g] : sa[g];
-          const float pr = (mn == -INFINITY) ? 0.f : ex2(own_s - mn);
+          const float pr = (mn == -INFINITY) ? 0.f : ex2(so[g] - mn);
           l_thr[g] = fmaf(l_thr[g], al, pr);
           uint16_t hi, lo;
           split16<T>(pr, hi, lo);
@@ -914,8 +941,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float mn = fmaxf(m_run[g], cm);
           // rows g >= rows never see a finite score; keep them inert (alpha 0, p 0)
           alpha[g] = (mn == -INFINITY) ? 0.f : ex2(m_run[g] - mn);
-          const float own_s = hh ? sb[g] : sa[g];
-          const float pr = (mn == -INFINITY) ? 0.f : ex2(own_s - mn);
+          const float pr = (mn == -INFINITY) ? 0.f : ex2(so[g] - mn);
           m_run[g] = mn;
           l_thr[g] = fmaf(l_thr[g], alpha[g], pr);
           uint16_t hi, lo;
@@ -974,16 +1000,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (mt.flags & kLast) {
         // per-warp sum of l over the group's 128 tokens
         float* lr = lred_t + (Ly::DEFER_END ? lpar : 0u) * 64;
+        {
+          float v[NC];   // paired: the own head's sums
 #pragma unroll
-        for (int g = 0; g < (PAIR ? GH : GT); ++g) {
-          float lg = l_thr[g];
-#pragma unroll
-          for (int off = PAIR ? 8 : 16; off > 0; off >>= 1) lg += __shfl_xor_sync(kFull, lg, off);
-          if constexpr (PAIR) {
-            if ((lane & 15) == 0) lr[wq * 16 + hd * GH + g] = lg;   // the own head's sums
-          } else {
-            if (lane == 0) lr[wq * 16 + g] = lg;
-          }
+          for (int g = 0; g < NC; ++g) v[g] = l_thr[g];
+          const float lg = xreduce<NC, SPAN, false>(v, lane);
+          const int cg = (lane & (SPAN - 1)) / (SPAN / NC);
+          if ((lane & (SPAN / NC - 1)) == 0) lr[wq * 16 + hd * GH + cg] = lg;
         }
         if constexpr (Ly::DEFER_END) {
 #pragma unroll
