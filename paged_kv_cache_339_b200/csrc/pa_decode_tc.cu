@@ -908,6 +908,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!group_sync(gbar, gphase, abrt, status)) break;
       float alpha[GT];
+      float cmx[GT];   // the chunk's max per column over the group's four warps
+#pragma unroll
+      for (int g4 = 0; g4 < GT; g4 += 4) {
+        const float4 a = *reinterpret_cast<const float4*>(rb + g4);
+        const float4 b = *reinterpret_cast<const float4*>(rb + 16 + g4);
+        const float4 c = *reinterpret_cast<const float4*>(rb + 32 + g4);
+        const float4 d = *reinterpret_cast<const float4*>(rb + 48 + g4);
+        cmx[g4] = fmaxf(fmaxf(a.x, b.x), fmaxf(c.x, d.x));
+        cmx[g4 + 1] = fmaxf(fmaxf(a.y, b.y), fmaxf(c.y, d.y));
+        cmx[g4 + 2] = fmaxf(fmaxf(a.z, b.z), fmaxf(c.z, d.z));
+        cmx[g4 + 3] = fmaxf(fmaxf(a.w, b.w), fmaxf(c.w, d.w));
+      }
       uint32_t col[NPV];   // P^T row own_t: column g = hi(p_g), column GT + g = lo(p_g)
 #pragma unroll
       for (int i = 0; i < NPV; ++i) col[i] = 0;
@@ -916,7 +928,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // all of them), then the own head's probabilities
 #pragma unroll
         for (int g = 0; g < GT; ++g) {
-          const float cm = fmaxf(fmaxf(rb[g], rb[16 + g]), fmaxf(rb[32 + g], rb[48 + g]));
+          const float cm = cmx[g];
           const float mn = fmaxf(m_run[g], cm);
           alpha[g] = (mn == -INFINITY) ? 0.f : ex2(m_run[g] - mn);
           m_run[g] = mn;
@@ -937,7 +949,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
 #pragma unroll
         for (int g = 0; g < GT; ++g) {
-          const float cm = fmaxf(fmaxf(rb[g], rb[16 + g]), fmaxf(rb[32 + g], rb[48 + g]));
+          const float cm = cmx[g];
           const float mn = fmaxf(m_run[g], cm);
           // rows g >= rows never see a finite score; keep them inert (alpha 0, p 0)
           alpha[g] = (mn == -INFINITY) ? 0.f : ex2(m_run[g] - mn);
