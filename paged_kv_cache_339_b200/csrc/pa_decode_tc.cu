@@ -4,10 +4,13 @@
 // not fix") the G query heads that share a KV head form a real dense tile, so
 // the two contractions of a 128-token chunk run as MMAs:
 //
-//   S^T[128 tok, 16] = K[128 tok, 128 d] . Q^T[128 d, 16]     (A = K, K-major)
-//   O^T[128 d, NPV]  = V^T[128 d, 128 tok] . P^T[128 tok, NPV] (A = V^T, MN-major)
+//   S'[256 half-rows, NS] = K'[256 half-rows, 64] . Q'^T[64, NS]  (two M = 128 MMAs, A = K', K-major)
+//   O^T[128 d, NPV]       = V^T[128 d, 128 tok] . P^T[128 tok, NPV] (A = V^T, MN-major)
 //
-// Query heads sit on the N side (padded to 16; spare columns are ignored).
+// K' views the chunk's K as 128-byte half-rows (token, half h of d), Q' holds
+// the query rows' first halves then their second halves, and a token's score
+// is the sum of its two half-row terms K_h[t] . Q_h[g]. Query heads sit on
+// the N side (padded to 16; spare columns are ignored).
 // The probabilities are rounded to 16 bits for the second MMA as a sum of two
 // terms, p = hi + lo (columns [0, NPV/2) and [NPV/2, NPV) of P^T), so the
 // product keeps ~16 significant bits of p at no extra tensor-core passes.
@@ -34,11 +37,14 @@
 //   warps 1, 2  MMA issuers (one elected lane each), one per stream: S^T into
 //               the stream's TMEM columns, then O^T once its softmax group has
 //               published P; warp 1 also allocates and frees TMEM.
-//   warps 3-6,  softmax and correction groups, one per stream: thread r owns
-//   7-10        token r of a chunk for the softmax (tcgen05.ld of its S^T row)
-//               and output column d = r for the correction O = alpha O + O_c;
-//               a split item writes its partial result to the workspace, and
-//               the last piece of a (sequence, KV head) to finish merges them.
+//   warps 3-6,  softmax and correction groups, one per stream: thread r reads
+//   7-10        half-row r of both score tiles (tcgen05.ld), owns one of the
+//               two tokens in them and takes its partner lane's half of that
+//               token's score; the column maxima and sums over the group use
+//               transposed warp reductions. Thread r also owns output column
+//               d = r for the correction O = alpha O + O_c. A split item
+//               writes its partial result to the workspace; after its last
+//               item the group merges split rows (merge tasks).
 // Paired KV heads (block size 8, 4 query heads per KV head): the pool stores
 // a block's KV heads one after the other, so the pages of KV heads 2j and
 // 2j + 1 of a block are one contiguous 4 KiB run. The kernel then treats the
@@ -847,7 +853,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       const uint32_t par = n & 1u;
-      // ---- scores of tokens tk0 and tk0 + 64 (both halves summed)
+      // ---- the half-row scores of tokens tk0 (tile 0) and tk0 + 64 (tile 1)
       if (!__all_sync(kFull, mbar_wait(&s_full[t], par, abrt, status))) break;
       tc_fence_after();
       float sv0[Ly::NS], sv1[Ly::NS];

@@ -7,8 +7,9 @@
 // The header holds the device status word (first 4 bytes), the work counter
 // the persistent decode kernels claim items from, and the plan the planning
 // kernel chose (split size, number of items). A merge counter per
-// (sequence, KV head) counts the finished pieces of a split sequence; the
-// last piece merges them. Partial results are indexed
+// (sequence, KV head) counts the finished pieces of a split sequence: the
+// CUDA-core kernel's last piece to finish merges them, the tensor-core
+// kernel's merge tasks wait for the count. Partial results are indexed
 // [sequence][query head][split].
 #pragma once
 
