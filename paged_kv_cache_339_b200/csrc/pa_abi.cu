@@ -283,14 +283,23 @@ pa_status pa_decode(const pa_kv_cache* cache, float* out, const void* q,
   // At block size 8 the tensor-core kernel reads two KV heads' pages with one
   // copy (its items, and the plan's, are then pairs of heads: one head of 2G
   // query heads); not with shared prefixes, whose launches count real heads.
-  // Pairs halve the (sequence, head) units the plan deals out, so only where
-  // at least two pairs per item stream remain: with fewer, the coarser items
-  // and the extra splits cost more at the end of the call than the saved
-  // copies gain.
+  // Pairs halve the (sequence, head) units the plan deals out and the pieces
+  // it cuts, so they are used where enough items remain: with at least two
+  // pairs per item stream (many sequences), or with fewer pairs than streams
+  // (few sequences, cut into pieces) when even the longest possible context
+  // leaves the halved pieces above the workspace's smallest split (its bound
+  // on pieces per sequence); in between, and for few short sequences, the
+  // coarser items cost more at the end of the call than the saved copies gain.
   const int64_t pair_units = static_cast<int64_t>(num_seqs) * (cache->num_kv_heads / 2);
-  const bool pair = use_tc && !ch.share &&
-                    tc_pair_supported(cache->block_size, cache->num_kv_heads, group) &&
-                    pair_units >= 2 * (2 * static_cast<int64_t>(ctas));
+  const int64_t streams = 2 * static_cast<int64_t>(ctas);
+  bool pair = use_tc && !ch.share &&
+              tc_pair_supported(cache->block_size, cache->num_kv_heads, group);
+  if (pair && pair_units < 2 * streams) {
+    // an upper bound of the halved piece (the plan's half share, halved)
+    const int64_t piece = static_cast<int64_t>(num_seqs) * max_context_len *
+                          cache->num_kv_heads / streams / 4;
+    pair = pair_units < streams && piece >= auto_min_split(max_context_len);
+  }
 
   PlanParams pp;
   pp.context_lens = context_lens;

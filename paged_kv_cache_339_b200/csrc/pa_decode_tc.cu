@@ -45,15 +45,15 @@
 //               d = r for the correction O = alpha O + O_c. A split item
 //               writes its partial result to the workspace; after its last
 //               item the group merges split rows (merge tasks).
-// Paired KV heads (block size 8, 4 query heads per KV head): the pool stores
-// a block's KV heads one after the other, so the pages of KV heads 2j and
-// 2j + 1 of a block are one contiguous 4 KiB run. The kernel then treats the
-// pair as one virtual KV head of 8 query heads whose pages hold 2 x 8
+// Paired KV heads (block size 8, 4 or 8 query heads per KV head): the pool
+// stores a block's KV heads one after the other, so the pages of KV heads 2j
+// and 2j + 1 of a block are one contiguous 4 KiB run. The kernel then treats
+// the pair as one virtual KV head of 2G query heads whose pages hold 2 x 8
 // virtual tokens (head 2j's 8 tokens, then head 2j + 1's), loaded with one
 // box per block instead of one per (block, head): a 128-token ring position
 // holds 64 tokens of both heads. A softmax thread's token belongs to one of
 // the two heads, so it keeps the scores, probabilities and sums of that
-// head's 4 query heads only (the others' probabilities are zero). Halving
+// head's G query heads only (the others' probabilities are zero). Halving
 // the copies matters at block size 8, where the copy engine's request rate,
 // not HBM, bounds 2 KiB boxes.
 // No load uses cluster multicast; every wait is bounded (see pa_common.cuh).
@@ -1282,18 +1282,23 @@ cudaError_t launch_decode_tc_groups(const DecodeParams& p, int num_ctas, cudaStr
 }
 
 bool tc_pair_supported(int block_size, int num_kv_heads, int group) {
-  // a pair of KV heads of 4 query heads each fills the 8-row tile exactly
-  return block_size == 8 && num_kv_heads % 2 == 0 && group == 4;
+  // a pair of KV heads of 4 (8) query heads each fills the 8-row (16-row)
+  // tile exactly
+  return block_size == 8 && num_kv_heads % 2 == 0 && (group == 4 || group == 8);
 }
 
 cudaError_t launch_decode_tc(const DecodeParams& p, int num_ctas, cudaStream_t stream) {
   const int group = p.num_q_heads / p.num_kv_heads;
   if (!tc_supported(p.dtype, p.head_dim, group)) return cudaErrorInvalidValue;
   if (p.pair_heads) {
-    // a pair is one KV head of 2G = 8 query heads
+    // a pair is one KV head of 2G query heads
     if (!tc_pair_supported(p.block_size, p.num_kv_heads, group)) return cudaErrorInvalidValue;
-    if (p.dtype == 2) return launch_t<__nv_bfloat16, 8, false, true>(p, num_ctas, stream);
-    return launch_t<__half, 8, false, true>(p, num_ctas, stream);
+    if (p.dtype == 2) {
+      if (group == 4) return launch_t<__nv_bfloat16, 8, false, true>(p, num_ctas, stream);
+      return launch_t<__nv_bfloat16, 16, false, true>(p, num_ctas, stream);
+    }
+    if (group == 4) return launch_t<__half, 8, false, true>(p, num_ctas, stream);
+    return launch_t<__half, 16, false, true>(p, num_ctas, stream);
   }
   if (p.dtype == 2) {
     if (group <= 4) return launch_t<__nv_bfloat16, 4>(p, num_ctas, stream);

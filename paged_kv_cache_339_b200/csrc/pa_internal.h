@@ -53,7 +53,7 @@ struct DecodeParams {
   int32_t group_mode;
   size_t gpairs_off;
   // 1: the tensor-core kernel reads KV heads in pairs (its items, and the
-  // plan's, count num_kv_heads / 2 virtual heads of 2G = 8 query heads)
+  // plan's, count num_kv_heads / 2 virtual heads of 2G query heads)
   int32_t pair_heads;
 };
 
@@ -82,7 +82,7 @@ cudaError_t launch_decode_tc(const DecodeParams& p, int num_ctas,
 // sequences x G heads (16-bit KV, head_dim 128, G a divisor of 16 up to 8).
 bool tc_group_supported(int dtype, int head_dim, int group);
 // The tensor-core kernel can read KV heads in pairs (block size 8, an even
-// number of KV heads, 4 query heads per KV head).
+// number of KV heads, 4 or 8 query heads per KV head).
 bool tc_pair_supported(int block_size, int num_kv_heads, int group);
 cudaError_t launch_decode_tc_groups(const DecodeParams& p, int num_ctas,
                                     cudaStream_t stream);

@@ -4,8 +4,11 @@ A block stores its KV heads one after the other ("Paged Attention as a Memory
 Manager", "Virtual Memory as the Blueprint": a block holds the keys and
 values of a fixed number of tokens), so at block size 8 the tensor-core
 kernel loads the pages of KV heads 2j and 2j + 1 of a block with one copy and
-treats the pair as one head of 2G query heads, each score masked to its own
-KV head. The output must match the fp64 oracle element by element within the
+treats the pair as one head of 2G query heads (G = 4 or 8), each score kept
+for its own KV head's query heads only. pa_decode pairs heads with at least
+two pairs per item stream, or with fewer pairs than streams when the longest
+context allowed leaves the halved pieces above the workspace's smallest
+split. The output must match the fp64 oracle element by element within the
 decode tolerance, whatever the lengths, pieces and head layouts, and the
 plan must count the work in pairs exactly when the kernel pairs.
 """
@@ -46,6 +49,23 @@ def streams():
     return 2 * torch.cuda.get_device_properties(0).multi_processor_count
 
 
+def auto_min_split(max_ctx):
+    """The workspace's smallest automatic split (pa_workspace.h)."""
+    return max(256, -(-(-(-max_ctx // 64)) // 128) * 128)
+
+
+def expect_paired(B, Hkv, G, BS, max_ctx):
+    """pa_decode's choice to read KV heads in pairs (without shared prefixes)."""
+    if BS != 8 or Hkv % 2 or G not in (4, 8):
+        return False
+    units = B * (Hkv // 2)
+    if units >= 2 * streams():
+        return True
+    if units >= streams():
+        return False
+    return B * max_ctx * Hkv // streams() // 4 >= auto_min_split(max_ctx)
+
+
 def paired_lens(lens, Hkv):
     """`lens` repeated until the batch has at least two KV-head pairs per
     item stream (the fewest for which pa_decode pairs heads)."""
@@ -69,14 +89,15 @@ def decode(b, split):
 
 LENS = [0, 1, 2, 7, 8, 9, 31, 32, 33, 63, 64, 65, 127, 128, 129, 300, 1000, 1, 4099]
 
-# (dtype, query heads, KV heads, paired)
+# (dtype, query heads, KV heads, with at least two KV-head pairs per stream)
 LAYOUTS = [
     (torch.bfloat16, 16, 4, True),    # G = 4: two KV heads fill the 8-row tile
     (torch.float16, 16, 4, True),
     (torch.bfloat16, 8, 2, True),     # one pair
     (torch.bfloat16, 32, 8, True),    # four pairs
+    (torch.bfloat16, 32, 4, True),    # G = 8: two KV heads fill the 16-row tile
     (torch.bfloat16, 12, 3, False),   # odd KV heads: one head per item
-    (torch.float16, 32, 4, False),    # G = 8: one head per item
+    (torch.float16, 64, 4, False),    # G = 16: one head per item
 ]
 
 
@@ -87,6 +108,7 @@ _REF = {}
 @pytest.mark.parametrize("split", [0, 32, 64, 200])
 def test_matches_oracle(dtype, Hq, Hkv, paired, split):
     b = batch(paired_lens(LENS, Hkv) if paired else LENS, dtype, Hq, Hkv)
+    assert expect_paired(b.q.shape[0], Hkv, Hq // Hkv, 8, b.max_context_len) == paired
     bc = b.to("cpu")
     out, items, pairs = decode(b, split)
     # the plan counts (sequence, piece) pairs x KV heads, halved when paired
@@ -106,11 +128,36 @@ def test_matches_oracle(dtype, Hq, Hkv, paired, split):
         assert np.array_equal(o[1, h].numpy().astype(np.float64), vp[blk, h // G, 0])
 
 
-def test_few_sequences_are_not_paired():
-    """Fewer than two KV-head pairs per item stream: one head per item."""
-    b = batch(LENS, torch.bfloat16, 16, 4)
+def test_few_short_sequences_are_not_paired():
+    """Fewer than two KV-head pairs per item stream, and contexts too short
+    for halved pieces: one head per item."""
+    lens = [L for L in LENS if L <= 1000]
+    b = batch(lens, torch.bfloat16, 16, 4)
+    assert not expect_paired(len(lens), 4, 4, 8, max(lens))
     _, items, pairs = decode(b, 0)
     assert items == pairs * 4
+
+
+@pytest.mark.parametrize("Hq", [32, 64])
+def test_few_long_sequences_are_paired(Hq):
+    """Four long sequences (8 KV heads, 4 or 8 query heads each): fewer pairs
+    than streams, but long enough contexts: paired, split into pieces and
+    merged. Every query head of each sequence's first KV pair against the
+    oracle, every row against the CUDA-core path."""
+    lens = [20000, 33001, 47007, 60000]
+    b = batch(lens, torch.bfloat16, Hq, 8, seed=37)
+    G = Hq // 8
+    assert expect_paired(4, 8, G, 8, max(lens))
+    out, items, pairs = decode(b, 0)
+    assert items == pairs * 4
+    simt = run_step(b, path=ops.PA_PATH_SIMT, write=False)
+    assert float((out - simt).abs().max()) <= 2e-3
+    for seq in range(4):
+        heads = list(range(2 * G))
+        ref = reference_rows(b, seq, heads)
+        for h in heads:
+            row = out[seq, h].cpu().numpy().astype(np.float64)
+            assert np.max(np.abs(row - ref[h])) <= 2e-3, (seq, h)
 
 
 def oracle_inputs(bc):

@@ -121,27 +121,33 @@ def test_automatic_split_is_a_share_or_half_a_share(name):
 
 
 
-@pytest.mark.parametrize("few", [False, True])
-def test_paired_heads_cut_half_pieces(few):
+@pytest.mark.parametrize("case", ["many", "few_short", "few_long"])
+def test_paired_heads_cut_half_pieces(case):
     """At block size 8 the tensor-core kernel reads KV heads of 4 query heads
-    in pairs when there are at least two pairs per item stream: the items are
-    (piece, pair of KV heads), and the automatic split is half the one-head
-    split (a piece of the same work), never below the smallest split the
-    workspace allows; the pieces still tile every sequence. With fewer pairs,
-    one head per item and the one-head split."""
+    in pairs with at least two pairs per item stream ("many"), or with fewer
+    pairs than streams when the longest context allowed leaves the halved
+    pieces above the workspace's smallest split ("few_long"), not for a few
+    short sequences ("few_short"). Paired, the items are (piece, pair of KV
+    heads) and the automatic split is half the one-head split (a piece of the
+    same work), never below the smallest split the workspace allows; the
+    pieces still tile every sequence."""
     streams = 2 * torch.cuda.get_device_properties(0).multi_processor_count
-    num_seqs = 16 if few else 256
-    b = W.gqa("cuda", num_seqs=num_seqs, block_size=8)
+    if case == "many":
+        b = W.gqa("cuda", num_seqs=256, block_size=8)
+    elif case == "few_short":
+        b = W.gqa("cuda", num_seqs=16, max_len=600, block_size=8)
+    else:
+        b = W.long_context("cuda", num_q_heads=32, block_size=8)
     B, Hq, D = b.q.shape
-    assert (B * b.num_kv_heads // 2 >= 2 * streams) == (not few)
+    paired = case != "few_short"
     ws = ops.decode_workspace(B, Hq, D, b.max_context_len, b.block_size)
     run_step(b, workspace=ws, write=False)
     plan = read_plan(ws, B)
     lens = b.context_lens.cpu().tolist()
-    check_plan(plan, lens, b.num_kv_heads if few else b.num_kv_heads // 2)
+    check_plan(plan, lens, b.num_kv_heads // 2 if paired else b.num_kv_heads)
     share = -(-sum(lens) * b.num_kv_heads // streams)
     base = share if B * b.num_kv_heads >= streams else (share + 1) // 2
     up128 = lambda x: -(-x // 128) * 128
-    min_split = max(256, up128(-(-max(lens) // 64)))
+    min_split = max(256, up128(-(-b.max_context_len // 64)))
     one_head = max(up128(base), min_split)
-    assert plan["split_tokens"] == (one_head if few else max(one_head // 2, min_split))
+    assert plan["split_tokens"] == (max(one_head // 2, min_split) if paired else one_head)
