@@ -224,19 +224,23 @@ __device__ __forceinline__ float exp2_approx(float x) {
   return y;
 }
 
-// Round p to 16 bits (hi) and the remainder p - hi to 16 bits (lo): raw bits.
+// Round p to 16 bits (hi) and the remainder p - hi to 16 bits (lo), for two
+// values at once: p0 in the low half of each word, p1 in the high half (one
+// 2-wide conversion per word).
 template <typename T>
-__device__ __forceinline__ void split16(float p, uint16_t& hi, uint16_t& lo) {
-  if constexpr (sizeof(T) == 2 && std::is_same<T, __nv_bfloat16>::value) {
-    const __nv_bfloat16 h = __float2bfloat16_rn(p);
-    const __nv_bfloat16 l = __float2bfloat16_rn(p - __bfloat162float(h));
-    hi = *reinterpret_cast<const uint16_t*>(&h);
-    lo = *reinterpret_cast<const uint16_t*>(&l);
+__device__ __forceinline__ void split16x2(float p0, float p1, uint32_t& hi, uint32_t& lo) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
   } else {
-    const __half h = __float2half_rn(p);
-    const __half l = __float2half_rn(p - __half2float(h));
-    hi = *reinterpret_cast<const uint16_t*>(&h);
-    lo = *reinterpret_cast<const uint16_t*>(&l);
+    const __half2 h = __floats2half2_rn(p0, p1);
+    const float2 hf = __half22float2(h);
+    const __half2 l = __floats2half2_rn(p0 - hf.x, p1 - hf.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
   }
 }
 
@@ -926,9 +930,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         cmx[g4 + 2] = fmaxf(fmaxf(a.z, b.z), fmaxf(c.z, d.z));
         cmx[g4 + 3] = fmaxf(fmaxf(a.w, b.w), fmaxf(c.w, d.w));
       }
-      uint32_t col[NPV];   // P^T row own_t: column g = hi(p_g), column GT + g = lo(p_g)
-#pragma unroll
-      for (int i = 0; i < NPV; ++i) col[i] = 0;
+      float pv[NC];   // the thread's token's probabilities for its query columns
       if constexpr (PAIR) {
         // every column's running max and rescale (the correction below takes
         // all of them), then the own head's probabilities
@@ -945,12 +947,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float al = hd ? alpha[GH + g] : alpha[g];
           const float pr = (mn == -INFINITY) ? 0.f : ex2(so[g] - mn);
           l_thr[g] = fmaf(l_thr[g], al, pr);
-          uint16_t hi, lo;
-          split16<T>(pr, hi, lo);
-          col[g] = hd ? 0u : hi;
-          col[GH + g] = hd ? hi : 0u;
-          col[GT + g] = hd ? 0u : lo;
-          col[GT + GH + g] = hd ? lo : 0u;
+          pv[g] = pr;
         }
       } else {
 #pragma unroll
@@ -962,19 +959,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float pr = (mn == -INFINITY) ? 0.f : ex2(so[g] - mn);
           m_run[g] = mn;
           l_thr[g] = fmaf(l_thr[g], alpha[g], pr);
-          uint16_t hi, lo;
-          split16<T>(pr, hi, lo);
-          col[g] = hi;
-          col[GT + g] = lo;
+          pv[g] = pr;
+        }
+      }
+      // P^T row own_t: columns [0, GT) hold the hi parts, [GT, 2 GT) the lo
+      // parts (paired: the own head's columns; the other head's are zero),
+      // two columns to a word
+      uint32_t wd[NPV / 2];
+#pragma unroll
+      for (int i = 0; i < NPV / 2; ++i) wd[i] = 0u;
+#pragma unroll
+      for (int k = 0; k < NC / 2; ++k) {
+        uint32_t hi, lo;
+        split16x2<T>(pv[2 * k], pv[2 * k + 1], hi, lo);
+        if constexpr (PAIR) {
+          wd[k] = hd ? 0u : hi;
+          wd[GH / 2 + k] = hd ? hi : 0u;
+          wd[GT / 2 + k] = hd ? 0u : lo;
+          wd[GT / 2 + GH / 2 + k] = hd ? lo : 0u;
+        } else {
+          wd[k] = hi;
+          wd[GT / 2 + k] = lo;
         }
       }
 #pragma unroll
       for (int ng = 0; ng < NPV / 8; ++ng)
         *reinterpret_cast<uint4*>(pdst_base + ng * 2048) =
-            make_uint4(col[8 * ng + 0] | (col[8 * ng + 1] << 16),
-                       col[8 * ng + 2] | (col[8 * ng + 3] << 16),
-                       col[8 * ng + 4] | (col[8 * ng + 5] << 16),
-                       col[8 * ng + 6] | (col[8 * ng + 7] << 16));
+            make_uint4(wd[4 * ng], wd[4 * ng + 1], wd[4 * ng + 2], wd[4 * ng + 3]);
       bool vok = true;
       // past the chunk's valid tokens but inside the last 16-token step of
       // the P.V MMA (paired: inside the last loaded block): make V finite
