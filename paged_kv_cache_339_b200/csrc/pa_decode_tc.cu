@@ -860,7 +860,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- the half-row scores of tokens tk0 (tile 0) and tk0 + 64 (tile 1)
       if (!__all_sync(kFull, mbar_wait(&s_full[t], par, abrt, status))) break;
       tc_fence_after();
-      float sv0[Ly::NS], sv1[Ly::NS];
+      // The thread's own token's scores (hh = 0: token tk0 of tile 0, hh = 1:
+      // token tk0 + 64 of tile 1) for its query columns: all GT, or paired,
+      // the GH of its own KV head. A half-row term is K_h[t] . Q_h[g]; the
+      // thread holds half hh of both tiles' tokens, so it keeps its own
+      // token's term (own) and trades the other tile's term (snd) with its
+      // partner (lane ^ sh), which holds the other half. Score columns: the
+      // query rows' first halves [0, NS/2), then their second halves.
+      constexpr int NC = PAIR ? GH : GT;
+      constexpr int SPAN = PAIR ? 16 : 32;   // lanes of one KV head
+      float own[NC], snd[NC];
+      // column g of the thread's (paired: own head's) query columns in a run
+      // of first or second halves
+      auto pick = [&](const float* x, int g) { return PAIR ? (hd ? x[GH + g] : x[g]) : x[g]; };
       if constexpr (Ly::NS == 16) {
         // both score tiles requested at once, one wait
         uint32_t su0[16], su1[16];
@@ -868,41 +880,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld16_async(lane_addr + s_col + Ly::NS, su1);
         tmem_wait16(su0);
         tmem_after_wait16(su1);
+        float sv0[16], sv1[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           sv0[i] = __uint_as_float(su0[i]);
           sv1[i] = __uint_as_float(su1[i]);
         }
-      } else {   // 64 columns: one wait per load keeps the registers in bounds
-        tmem_ld16(lane_addr + s_col, sv0);
-        tmem_ld16(lane_addr + s_col + Ly::NS, sv1);
-        tmem_ld16(lane_addr + s_col + 16, sv0 + 16);
-        tmem_ld16(lane_addr + s_col + Ly::NS + 16, sv1 + 16);
+#pragma unroll
+        for (int g = 0; g < NC; ++g) {
+          own[g] = hh ? pick(sv1 + 8, g) : pick(sv0, g);
+          snd[g] = hh ? pick(sv0 + 8, g) : pick(sv1, g);
+        }
+      } else {
+        // 64 columns, 16 at a time, each kept only where the thread uses it
+        float x[16];
+        tmem_ld16(lane_addr + s_col, x);   // tile 0, first halves
+#pragma unroll
+        for (int g = 0; g < NC; ++g) own[g] = pick(x, g);
+        tmem_ld16(lane_addr + s_col + Ly::NS, x);   // tile 1, first halves
+#pragma unroll
+        for (int g = 0; g < NC; ++g) snd[g] = pick(x, g);
+        tmem_ld16(lane_addr + s_col + 16, x);   // tile 0, second halves
+#pragma unroll
+        for (int g = 0; g < NC; ++g) snd[g] = hh ? pick(x, g) : snd[g];
+        tmem_ld16(lane_addr + s_col + Ly::NS + 16, x);   // tile 1, second halves
+#pragma unroll
+        for (int g = 0; g < NC; ++g) own[g] = hh ? pick(x, g) : own[g];
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[t]);
       // hardware 2^x (ex2.approx)
       auto ex2 = [](float x) { return exp2_approx(x); };
-      // The thread's own token's scores (hh = 0: token tk0 of tile 0, hh = 1:
-      // token tk0 + 64 of tile 1) for its query columns: all GT, or paired,
-      // the GH of its own KV head. A half-row term is K_h[t] . Q_h[g]; the
-      // thread holds half hh of both tiles' tokens, so it keeps its own
-      // token's term and trades the other tile's term with its partner
-      // (lane ^ sh), which holds the other half.
-      constexpr int NC = PAIR ? GH : GT;
-      constexpr int SPAN = PAIR ? 16 : 32;   // lanes of one KV head
       const bool own_ok = own_rt < mt.valid;
       float so[NC];
 #pragma unroll
       for (int g = 0; g < NC; ++g) {
-        float own = hh ? sv1[Ly::NS / 2 + g] : sv0[g];
-        float send = hh ? sv0[Ly::NS / 2 + g] : sv1[g];
-        if constexpr (PAIR) {
-          own = hd ? (hh ? sv1[Ly::NS / 2 + GH + g] : sv0[GH + g]) : own;
-          send = hd ? (hh ? sv0[Ly::NS / 2 + GH + g] : sv1[GH + g]) : send;
-        }
-        const float full = own + __shfl_xor_sync(kFull, send, sh);
+        const float full = own[g] + __shfl_xor_sync(kFull, snd[g], sh);
         so[g] = (own_ok && (PAIR || g < rows)) ? full * sl2 : -INFINITY;
       }
       // ---- chunk max per head across the group's 128 threads (paired: per
