@@ -96,6 +96,7 @@ LAYOUTS = [
     (torch.bfloat16, 8, 2, True),     # one pair
     (torch.bfloat16, 32, 8, True),    # four pairs
     (torch.bfloat16, 32, 4, True),    # G = 8: two KV heads fill the 16-row tile
+    (torch.float16, 32, 4, True),
     (torch.bfloat16, 12, 3, False),   # odd KV heads: one head per item
     (torch.float16, 64, 4, False),    # G = 16: one head per item
 ]
